@@ -1,0 +1,201 @@
+/*
+ * muon_ns.h — C ABI of the B200 (sm_100a) Muon / NorMuon optimizer step.
+ *
+ * One optimizer step over a set of matrix parameters is four stream-ordered
+ * calls:
+ *
+ *   muon_momentum_norm    momentum + Nesterov look-ahead + per-slice ||U||_F^2
+ *   muon_ns_batched       quintic Newton-Schulz, standard form (symmetric
+ *                         products computed on one triangle)
+ *   muon_gram_ns_batched  quintic Newton-Schulz, Gram form (iterates on the
+ *                         small m x m side)
+ *   normuon_update        NorMuon per-row variance, normalization and
+ *                         norm-preserving rescale (optional), then the
+ *                         shape-scaled, decoupled-weight-decay update
+ *
+ * Sources (page titles):
+ *   [dion-121]  microsoft/dion PR #121 "Fix convolution flattening in
+ *               megabatches and NorMuon normalization"
+ *   [mcore-lsm] Megatron-Core API docs, core.optimizer.layer_sharded_muon
+ *   [ds-8437]   DeepSpeed issue #8437 "Muon under AutoTP orthogonalizes each
+ *               shard, so the update depends on the TP degree"
+ *
+ * Data model.  A call takes an array of muon_batch.  A batch is N slices of
+ * one shape [rows, cols] (rows = fan_out, cols = fan_in = prod of the
+ * parameter's other dims), each slice a row-major matrix.  A megabatch of
+ * stacked convolutions [N, out, in, kh, kw] is the batch [N, out, in*kh*kw]
+ * ([dion-121] "Problem and fix"); per-head orthogonalization of a
+ * head-blocked projection [H*d, cols] is the batch [H, d, cols] with
+ * batch_stride d*ld ([ds-8437] "What could be done", option 3).  Every
+ * slice is orthogonalized on its own.
+ *
+ * Ownership.  Every pointer in these structs is DEVICE memory owned by the
+ * caller.  The library allocates nothing, frees nothing, keeps no state
+ * between calls and does not synchronize the stream; all work is enqueued on
+ * the given stream.  Scratch memory is the caller's workspace, sized by
+ * muon_workspace_size.
+ *
+ * Errors.  Every argument is checked on the host before anything is
+ * enqueued.  On any error the call returns a non-zero status and touches no
+ * memory ("reject before mutating").  There is no fallback to another
+ * precision or kernel.  Device-side waits are bounded: a kernel that waits
+ * past its limit writes a non-zero word at workspace offset 0 and returns
+ * (see muon_workspace_error).  Empty batches (n == 0, rows == 0 or
+ * cols == 0) are accepted and enqueue nothing.
+ *
+ * Alignment.  Tensor-core operands are read by TMA: slice base pointers must
+ * be 16-byte aligned and ld, batch_stride must be multiples of 16 bytes
+ * (8 bf16 elements) for ns_in and ns_out; the workspace must be 256-byte
+ * aligned.  Violations return MUON_MISALIGNED.
+ */
+#ifndef MUON_NS_H_
+#define MUON_NS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MUON_API __attribute__((visibility("default")))
+#else
+#define MUON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MUON_OK = 0,
+  MUON_INVALID_ARG = 1,        /* null pointer where one is required, bad count */
+  MUON_BAD_SHAPE = 2,          /* ld < cols, overlapping slices, size limits */
+  MUON_UNSUPPORTED_DTYPE = 3,  /* dtype not allowed for that tensor */
+  MUON_MISALIGNED = 4,         /* 16-byte TMA rule or 256-byte workspace rule */
+  MUON_WORKSPACE_TOO_SMALL = 5,
+  MUON_CUDA_ERROR = 6,         /* a CUDA runtime call or launch failed */
+  MUON_UNSUPPORTED_DEVICE = 7  /* current device is not sm_100 */
+} muon_status;
+
+typedef enum { MUON_F32 = 0, MUON_BF16 = 1, MUON_F16 = 2 } muon_dtype;
+
+/* A strided view of the batch's N slices; element (s, i, j) is at
+ * ptr + (s*batch_stride + i*ld + j) elements.  ld >= cols. */
+typedef struct {
+  void* ptr;
+  int64_t ld;
+  int64_t batch_stride;
+  int32_t dtype;               /* muon_dtype */
+  int32_t reserved;
+} muon_view;
+
+/* N same-shape slices and every per-slice buffer the step touches.
+ * Which fields a call reads or writes is listed at each call. */
+typedef struct {
+  int64_t n;                   /* slices */
+  int64_t rows;                /* fan_out of the slice */
+  int64_t cols;                /* fan_in of the slice */
+  muon_view grad;              /* G: f32 | bf16, read */
+  muon_view momentum;          /* M: f32 | bf16, updated in place */
+  muon_view ns_in;             /* U: bf16, the Newton-Schulz input */
+  muon_view ns_out;            /* O: bf16, the Newton-Schulz output */
+  muon_view weight;            /* W: f32 | bf16, updated in place */
+  muon_view weight_copy;       /* optional bf16 copy of an f32 W (ptr NULL: none) */
+  float* sumsq;                /* [n] f32: ||U||_F^2 per slice, or NULL */
+  float* variance;             /* [n*rows] f32 NorMuon variance, slice-major; NULL without NorMuon */
+  float lr_scale;              /* shape factor of the update, from the PARAMETER's
+                                  (fan_out, fan_in): sqrt(max(1, fan_out/fan_in)) * extra
+                                  ([dion-121] review "Correctness — confirmed";
+                                  [mcore-lsm] scale_mode='spectral') */
+  int32_t reserved;
+} muon_batch;
+
+/* Hyperparameters of one step ([mcore-lsm] LayerShardedMuon constructor). */
+typedef struct {
+  float mu;                    /* momentum, 0.95 */
+  int32_t nesterov;            /* 1: U = G + mu*M_new; 0: U = M_new */
+  float ns_eps;                /* Frobenius normalization: X0 = U / (||U||_F + ns_eps) */
+  float a, b, c;               /* quintic coefficients (3.4445, -4.7750, 2.0315) */
+  int32_t ns_steps;            /* iterations, 5; 1..16 */
+  float beta2;                 /* NorMuon variance decay, 0.95 */
+  float nor_eps;               /* NorMuon: O / (sqrt(v) + nor_eps) */
+  float lr;                    /* learning rate */
+  float weight_decay;          /* decoupled: W *= 1 - lr*weight_decay before the update */
+  const float* abc_schedule;   /* optional HOST array [ns_steps][3] of per-iteration
+                                  coefficients; NULL: (a, b, c) at every iteration */
+} muon_hparams;
+
+/* Bytes of workspace the given call needs for these batches.
+ * which: 0 momentum_norm, 1 ns_batched, 2 gram_ns_batched, 3 normuon_update,
+ * -1 the maximum over all four.  Returns 0 on invalid arguments. */
+MUON_API size_t muon_workspace_size(const muon_batch* batches, int nb, int which);
+
+/*
+ * Momentum with Nesterov look-ahead and the squared Frobenius norm.
+ * [mcore-lsm] LayerShardedMuon.step(): the elementwise momentum update
+ * starts the step; momentum 0.95, nesterov=True.  [ds-8437] "Why it
+ * happens": Newton-Schulz first normalizes by the matrix norm.
+ *   M <- mu*M + G                   (stored in M's dtype, RN-even)
+ *   U  = G + mu*M   (nesterov) or M  (stored to ns_in as bf16, RN-even)
+ *   sumsq[s] = sum over slice s of bf16(U)^2   (deterministic order)
+ * Reads grad, momentum; writes momentum, ns_in, sumsq (sumsq required).
+ */
+MUON_API muon_status muon_momentum_norm(const muon_batch* batches, int nb, const muon_hparams* hp,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Standard quintic Newton-Schulz of every slice, bf16 operands, fp32
+ * accumulation on the tensor cores.
+ * [ds-8437] "Why it happens": normalize, then iterate on X X^T.
+ * [mcore-lsm] use_syrk: A = X X^T and B = b*A + c*A^2 are symmetric, one
+ * triangle of each is computed.  Per iteration X <- a*X + B X.  A slice with
+ * rows > cols is iterated transposed; the result O is in the slice's own
+ * orientation.  X0 = U / (sqrt(sumsq) + ns_eps), with sumsq from
+ * muon_momentum_norm when batch.sumsq is non-NULL, else computed here.
+ * Reads ns_in (left unchanged), sumsq; writes ns_out.
+ */
+MUON_API muon_status muon_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Gram Newton-Schulz: the same map iterated on the small side.
+ * [ds-8437] "Measurement": the Gram kernel gives the standard kernel's
+ * results.  With X0 the normalized slice (m <= n side first) and
+ * G = X0 X0^T: A = G, Q = I; per iteration P = a*I + b*A + c*A^2,
+ * Q <- P Q, A <- P A P; O = Q X0.  The m x m products use fp16 operands
+ * (10-bit mantissa) with fp32 accumulation; X-side products use bf16.
+ * Reads ns_in (left unchanged), sumsq; writes ns_out.
+ */
+MUON_API muon_status muon_gram_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * NorMuon normalization and the weight update.
+ * [dion-121] follow-on "What it does": one variance per output channel,
+ * over the last dim of the flattened [N, out, prod(rest)] view;
+ * "Compatibility": norm-preserving rescale, local to the slice.
+ * [mcore-lsm] _apply_update: one multiply-add in fp32, one downcast on store.
+ * With use_normuon:
+ *   v_i <- beta2*v_i + (1-beta2) * mean_j O_ij^2           (per slice row i)
+ *   Oh   = O_i / (sqrt(v_i) + nor_eps),  Oh *= ||O||_F / ||Oh||_F (0 stays 0)
+ * else Oh = O.  Then W <- W*(1 - lr*weight_decay) - lr*lr_scale*Oh, and
+ * weight_copy <- bf16(W) when given.
+ * Reads ns_out, variance; writes variance, weight, weight_copy.
+ */
+MUON_API muon_status normuon_update(const muon_batch* batches, int nb, const muon_hparams* hp,
+                           int use_normuon, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/* Reads the error word at workspace offset 0 after synchronizing the stream:
+ * 0 = no device-side wait timed out since the word was last cleared (each
+ * Newton-Schulz call clears it when it starts). */
+MUON_API muon_status muon_workspace_error(const void* workspace, cudaStream_t stream, int32_t* error_word);
+
+MUON_API const char* muon_status_string(muon_status status);
+
+/* Library version, "major.minor.patch". */
+MUON_API const char* muon_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MUON_NS_H_ */

@@ -1,0 +1,42 @@
+/*
+ * muon_ns_testing.h — test hook exported by libmuon_ns for unit tests of the
+ * tensor-core GEMM that the Newton-Schulz calls are built from.  The pages
+ * have no counterpart: this exists so that the sm_100a kernel can be checked
+ * one product at a time against a plain matrix product.
+ *
+ * muon_testing_gemm computes, for every slice s < slices,
+ *     C[s] = f * (alpha * opA(A[s]) opB(B[s]) + beta * D[s]) + gamma * I
+ * with opA M x K and opB K x N:
+ *     a_mn == 0: A[s] is stored [M][K] row-major;  a_mn == 1: stored [K][M]
+ *     b_mn == 0: B[s] is stored [N][K] row-major (C = A B^T); b_mn == 1: [K][N]
+ * f = f0 * (1/(sqrt(sumsq[s]) + eps))^s_pow (s_pow 0, 1 or 2; sumsq device [slices]).
+ * tri != 0 requires M == N and computes only the lower triangle, mirrored.
+ * in_dtype (MUON_BF16 | MUON_F16) is the type of A and B; out_dtype and
+ * add_dtype (MUON_BF16 | MUON_F16) the types of C and D.  D may be NULL
+ * when beta == 0.  All pointers are device memory; ld/bs are in elements.
+ * row_ss (device, may be NULL; non-tri only) receives, per slice, per
+ * 256-column block and per row, the sum of squares of the stored C values.
+ * The workspace (>= 256 bytes, 256-byte aligned) receives the error word.
+ */
+#ifndef MUON_NS_TESTING_H_
+#define MUON_NS_TESTING_H_
+
+#include "muon_ns.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+MUON_API muon_status muon_testing_gemm(int M, int N, int K, int slices, int tri, int in_dtype,
+                              const void* A, int64_t lda, int64_t bsa, int a_mn,
+                              const void* B, int64_t ldb, int64_t bsb, int b_mn,
+                              const void* D, int64_t ldd, int64_t bsd, int add_dtype,
+                              void* C, int64_t ldc, int64_t bsc, int out_dtype,
+                              float alpha, float beta, float gamma, float f0,
+                              int s_pow, const float* sumsq, float eps, float* row_ss,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MUON_NS_TESTING_H_ */

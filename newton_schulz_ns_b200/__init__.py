@@ -1,0 +1,245 @@
+"""B200-native Muon / NorMuon optimizer step: Python binding of libmuon_ns.
+
+The four calls of the C ABI (include/muon_ns.h) under the same names:
+``muon_momentum_norm``, ``muon_ns_batched``, ``muon_gram_ns_batched`` and
+``normuon_update``; plus ``muon_workspace_size``.  They take lists of
+``Batch`` objects built from torch tensors; torch provides device memory and
+streams only.  Every arithmetic step runs in the library's sm_100a kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+from typing import List, Optional, Sequence
+
+import torch
+
+from . import _capi
+from ._capi import MUON_BF16, MUON_F16, MUON_F32, MuonError  # noqa: F401
+
+__all__ = ["Batch", "Hparams", "muon_workspace_size", "muon_momentum_norm", "muon_ns_batched",
+           "muon_gram_ns_batched", "normuon_update", "workspace_error", "testing_gemm", "spectral_scale",
+           "ns_flops", "version", "MuonError", "LIB_PATH"]
+
+LIB_PATH = _capi.LIB_PATH
+
+_DT = {torch.float32: MUON_F32, torch.bfloat16: MUON_BF16, torch.float16: MUON_F16}
+
+QUINTIC = (3.4445, -4.7750, 2.0315)
+
+
+def version() -> str:
+    return _capi.lib.muon_version().decode()
+
+
+def spectral_scale(fan_out: int, fan_in: int, extra: float = 1.0) -> float:
+    """Update shape factor sqrt(max(1, fan_out/fan_in)) * extra of ONE parameter."""
+    return math.sqrt(max(1.0, fan_out / fan_in)) * extra
+
+
+def ns_flops(rows: int, cols: int, variant: str = "standard", steps: int = 5) -> float:
+    """Floating-point operations the library's kernels perform for one slice.
+
+    Standard: per step X X^T (one triangle, m^2 n), b*A + c*A^2 (one
+    triangle, m^3) and B X (2 m^2 n).  Gram: X X^T (m^2 n), per step A^2,
+    P Q (from the second step) and the two factors of P A P (up to the
+    second-to-last step), each a one-triangle m^3, then Q X (2 m^2 n).
+    """
+    m, n = min(rows, cols), max(rows, cols)
+    if variant == "standard":
+        return float(steps * (3 * m * m * n + m ** 3))
+    prods = sum(1 + (k > 0) + 2 * (k < steps - 1) for k in range(steps))
+    return float(3 * m * m * n + prods * m ** 3)
+
+
+def _view(t: Optional[torch.Tensor], n: int, rows: int, cols: int, name: str) -> _capi.MuonView:
+    v = _capi.MuonView()
+    if t is None:
+        return v
+    if t.dim() == 2:
+        t = t.unsqueeze(0)
+    if t.dim() != 3 or tuple(t.shape) != (n, rows, cols):
+        raise ValueError(f"{name}: expected shape {(n, rows, cols)}, got {tuple(t.shape)}")
+    if t.stride(2) != 1:
+        raise ValueError(f"{name}: rows must be contiguous")
+    if t.dtype not in _DT:
+        raise ValueError(f"{name}: unsupported dtype {t.dtype}")
+    v.ptr = t.data_ptr()
+    v.ld = t.stride(1)
+    v.batch_stride = t.stride(0) if n > 1 else rows * t.stride(1)
+    v.dtype = _DT[t.dtype]
+    return v
+
+
+@dataclasses.dataclass
+class Batch:
+    """Same-shape slices [n, rows, cols] and the buffers one step touches.
+
+    Tensors are 3-D [n, rows, cols] views (2-D is taken as n = 1) whose rows
+    are contiguous; ``sumsq`` is [n] and ``variance`` [n, rows], both fp32.
+    """
+    n: int
+    rows: int
+    cols: int
+    grad: Optional[torch.Tensor] = None
+    momentum: Optional[torch.Tensor] = None
+    ns_in: Optional[torch.Tensor] = None
+    ns_out: Optional[torch.Tensor] = None
+    weight: Optional[torch.Tensor] = None
+    weight_copy: Optional[torch.Tensor] = None
+    sumsq: Optional[torch.Tensor] = None
+    variance: Optional[torch.Tensor] = None
+    lr_scale: float = 1.0
+
+    def to_c(self) -> _capi.MuonBatch:
+        b = _capi.MuonBatch()
+        b.n, b.rows, b.cols = self.n, self.rows, self.cols
+        args = (self.n, self.rows, self.cols)
+        b.grad = _view(self.grad, *args, "grad")
+        b.momentum = _view(self.momentum, *args, "momentum")
+        b.ns_in = _view(self.ns_in, *args, "ns_in")
+        b.ns_out = _view(self.ns_out, *args, "ns_out")
+        b.weight = _view(self.weight, *args, "weight")
+        b.weight_copy = _view(self.weight_copy, *args, "weight_copy")
+        for name in ("sumsq", "variance"):
+            t = getattr(self, name)
+            if t is not None:
+                if t.dtype != torch.float32 or not t.is_contiguous():
+                    raise ValueError(f"{name}: contiguous float32 expected")
+                want = self.n if name == "sumsq" else self.n * self.rows
+                if t.numel() != want:
+                    raise ValueError(f"{name}: {want} elements expected, got {t.numel()}")
+                setattr(b, name, t.data_ptr())
+        b.lr_scale = float(self.lr_scale)
+        return b
+
+
+@dataclasses.dataclass
+class Hparams:
+    mu: float = 0.95
+    nesterov: bool = True
+    ns_eps: float = 1e-7
+    abc: Sequence[float] = QUINTIC
+    ns_steps: int = 5
+    beta2: float = 0.95
+    nor_eps: float = 1e-8
+    lr: float = 0.02
+    weight_decay: float = 0.0
+    abc_schedule: Optional[Sequence[Sequence[float]]] = None
+
+    def to_c(self):
+        h = _capi.MuonHparams()
+        h.mu, h.nesterov, h.ns_eps = self.mu, int(bool(self.nesterov)), self.ns_eps
+        h.a, h.b, h.c = (float(x) for x in self.abc)
+        h.ns_steps = int(self.ns_steps)
+        h.beta2, h.nor_eps, h.lr, h.weight_decay = self.beta2, self.nor_eps, self.lr, self.weight_decay
+        keep = None
+        if self.abc_schedule is not None:
+            flat = [float(v) for row in self.abc_schedule for v in row]
+            keep = (ctypes.c_float * len(flat))(*flat)
+            h.abc_schedule = ctypes.cast(keep, ctypes.POINTER(ctypes.c_float))
+        return h, keep
+
+
+def _batches(batches: Sequence[Batch]):
+    arr = (_capi.MuonBatch * max(1, len(batches)))()
+    for i, b in enumerate(batches):
+        arr[i] = b.to_c()
+    return arr, len(batches)
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def _ws(workspace: Optional[torch.Tensor]):
+    if workspace is None:
+        return None, 0
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+def muon_workspace_size(batches: Sequence[Batch], which: int = -1) -> int:
+    arr, nb = _batches(batches)
+    return int(_capi.lib.muon_workspace_size(arr, nb, which))
+
+
+def allocate_workspace(batches: Sequence[Batch], which: int = -1, device=None) -> torch.Tensor:
+    """A uint8 CUDA tensor of muon_workspace_size bytes (torch's allocator aligns it to 512 B)."""
+    return torch.empty(max(256, muon_workspace_size(batches, which)), dtype=torch.uint8,
+                       device=device or "cuda")
+
+
+def muon_momentum_norm(batches: Sequence[Batch], hp: Hparams, workspace: torch.Tensor, stream=None) -> None:
+    arr, nb = _batches(batches)
+    h, _keep = hp.to_c()
+    p, nbytes = _ws(workspace)
+    _capi.check(_capi.lib.muon_momentum_norm(arr, nb, ctypes.byref(h), p, nbytes, _stream_ptr(stream)),
+                "muon_momentum_norm")
+
+
+def muon_ns_batched(batches: Sequence[Batch], hp: Hparams, workspace: torch.Tensor, stream=None) -> None:
+    arr, nb = _batches(batches)
+    h, _keep = hp.to_c()
+    p, nbytes = _ws(workspace)
+    _capi.check(_capi.lib.muon_ns_batched(arr, nb, ctypes.byref(h), p, nbytes, _stream_ptr(stream)),
+                "muon_ns_batched")
+
+
+def muon_gram_ns_batched(batches: Sequence[Batch], hp: Hparams, workspace: torch.Tensor, stream=None) -> None:
+    arr, nb = _batches(batches)
+    h, _keep = hp.to_c()
+    p, nbytes = _ws(workspace)
+    _capi.check(_capi.lib.muon_gram_ns_batched(arr, nb, ctypes.byref(h), p, nbytes, _stream_ptr(stream)),
+                "muon_gram_ns_batched")
+
+
+def normuon_update(batches: Sequence[Batch], hp: Hparams, use_normuon: bool, workspace: torch.Tensor,
+                   stream=None) -> None:
+    arr, nb = _batches(batches)
+    h, _keep = hp.to_c()
+    p, nbytes = _ws(workspace)
+    _capi.check(_capi.lib.normuon_update(arr, nb, ctypes.byref(h), int(bool(use_normuon)), p, nbytes,
+                                         _stream_ptr(stream)), "normuon_update")
+
+
+def workspace_error(workspace: torch.Tensor, stream=None) -> int:
+    out = ctypes.c_int32(0)
+    _capi.check(_capi.lib.muon_workspace_error(workspace.data_ptr(), _stream_ptr(stream), ctypes.byref(out)),
+                "muon_workspace_error")
+    return int(out.value)
+
+
+def testing_gemm(A: torch.Tensor, a_mn: bool, B: torch.Tensor, b_mn: bool, C: torch.Tensor, *, K: int,
+                 tri: bool = False, D: Optional[torch.Tensor] = None, alpha: float = 1.0, beta: float = 0.0,
+                 gamma: float = 0.0, f0: float = 1.0, s_pow: int = 0, sumsq: Optional[torch.Tensor] = None,
+                 eps: float = 0.0, row_ss: Optional[torch.Tensor] = None, workspace: torch.Tensor = None,
+                 stream=None) -> None:
+    """Runs one tensor-core GEMM problem of the library (include/muon_ns_testing.h).
+
+    A, B, C, D are 3-D [slices, rows, cols] with contiguous rows.  C is
+    [slices, M, N]; A is [slices, M, K] (a_mn False) or [slices, K, M];
+    B is [slices, N, K] (b_mn False) or [slices, K, N].
+    """
+    S, M, N = C.shape
+    if A.dtype != B.dtype:
+        raise ValueError("A and B must share a dtype")
+
+    def ld_bs(t):
+        return (t.stride(1), t.stride(0)) if t is not None else (0, 0)
+
+    lda, bsa = ld_bs(A)
+    ldb, bsb = ld_bs(B)
+    ldc, bsc = ld_bs(C)
+    ldd, bsd = ld_bs(D)
+    p, nbytes = _ws(workspace)
+    st = _capi.lib.muon_testing_gemm(
+        M, N, K, S, int(tri), _DT[A.dtype],
+        A.data_ptr(), lda, bsa, int(a_mn), B.data_ptr(), ldb, bsb, int(b_mn),
+        D.data_ptr() if D is not None else None, ldd, bsd, _DT[D.dtype] if D is not None else MUON_BF16,
+        C.data_ptr(), ldc, bsc, _DT[C.dtype], alpha, beta, gamma, f0, s_pow,
+        sumsq.data_ptr() if sumsq is not None else None, eps,
+        row_ss.data_ptr() if row_ss is not None else None, p, nbytes, _stream_ptr(stream))
+    _capi.check(st, "muon_testing_gemm")

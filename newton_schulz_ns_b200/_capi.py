@@ -1,0 +1,98 @@
+"""ctypes declarations of libmuon_ns (include/muon_ns.h, include/muon_ns_testing.h).
+
+Argument marshalling only: every step of the optimizer runs in the CUDA
+library.  Importing this module loads the library and fails loudly if it is
+missing or lacks a symbol; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libmuon_ns.so")
+
+MUON_F32, MUON_BF16, MUON_F16 = 0, 1, 2
+
+STATUS = {
+    0: "MUON_OK", 1: "MUON_INVALID_ARG", 2: "MUON_BAD_SHAPE", 3: "MUON_UNSUPPORTED_DTYPE",
+    4: "MUON_MISALIGNED", 5: "MUON_WORKSPACE_TOO_SMALL", 6: "MUON_CUDA_ERROR", 7: "MUON_UNSUPPORTED_DEVICE",
+}
+
+
+class MuonError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+class MuonView(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("ld", ctypes.c_int64), ("batch_stride", ctypes.c_int64),
+                ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class MuonBatch(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int64), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("grad", MuonView), ("momentum", MuonView), ("ns_in", MuonView), ("ns_out", MuonView),
+                ("weight", MuonView), ("weight_copy", MuonView),
+                ("sumsq", ctypes.c_void_p), ("variance", ctypes.c_void_p),
+                ("lr_scale", ctypes.c_float), ("reserved", ctypes.c_int32)]
+
+
+class MuonHparams(ctypes.Structure):
+    _fields_ = [("mu", ctypes.c_float), ("nesterov", ctypes.c_int32), ("ns_eps", ctypes.c_float),
+                ("a", ctypes.c_float), ("b", ctypes.c_float), ("c", ctypes.c_float),
+                ("ns_steps", ctypes.c_int32), ("beta2", ctypes.c_float), ("nor_eps", ctypes.c_float),
+                ("lr", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("abc_schedule", ctypes.POINTER(ctypes.c_float))]
+
+
+EXPORTS = ("muon_workspace_size", "muon_momentum_norm", "muon_ns_batched", "muon_gram_ns_batched",
+           "normuon_update", "muon_workspace_error", "muon_status_string", "muon_version",
+           "muon_testing_gemm")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m newton_schulz_ns_b200.build` "
+            "(the Muon step has no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name in EXPORTS:
+        if not hasattr(lib, name):
+            raise ImportError(f"{LIB_PATH} does not export {name}")
+    P = ctypes.c_void_p
+    B = ctypes.POINTER(MuonBatch)
+    H = ctypes.POINTER(MuonHparams)
+    lib.muon_workspace_size.argtypes = [B, ctypes.c_int, ctypes.c_int]
+    lib.muon_workspace_size.restype = ctypes.c_size_t
+    for fn in (lib.muon_momentum_norm, lib.muon_ns_batched, lib.muon_gram_ns_batched):
+        fn.argtypes = [B, ctypes.c_int, H, P, ctypes.c_size_t, P]
+        fn.restype = ctypes.c_int
+    lib.normuon_update.argtypes = [B, ctypes.c_int, H, ctypes.c_int, P, ctypes.c_size_t, P]
+    lib.normuon_update.restype = ctypes.c_int
+    lib.muon_workspace_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+    lib.muon_workspace_error.restype = ctypes.c_int
+    lib.muon_status_string.argtypes = [ctypes.c_int]
+    lib.muon_status_string.restype = ctypes.c_char_p
+    lib.muon_version.argtypes = []
+    lib.muon_version.restype = ctypes.c_char_p
+    i64, i32, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    lib.muon_testing_gemm.argtypes = [i32, i32, i32, i32, i32, i32,
+                                      P, i64, i64, i32, P, i64, i64, i32, P, i64, i64, i32,
+                                      P, i64, i64, i32, f32, f32, f32, f32, i32, P, f32, P,
+                                      P, ctypes.c_size_t, P]
+    lib.muon_testing_gemm.restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.muon_status_string(int(status)).decode()
+
+
+def check(status: int, what: str) -> None:
+    if status != 0:
+        raise MuonError(status, what)

@@ -1,0 +1,325 @@
+// Bandwidth-bound kernels of the Muon / NorMuon step (sm_100a):
+//   momentum + Nesterov + per-chunk sum of squares, the per-slice
+//   finalization of those sums, NorMuon row statistics and slice factors,
+//   and the weight update.
+//
+// Work is split into fixed chunks of CHUNK elements of one slice's
+// row-major [rows, cols] index space, so every reduction has a fixed order
+// (a chunk's partial is reduced by a fixed tree; a slice's partials are then
+// summed in chunk order): results are bitwise reproducible and independent
+// of the batch a slice is in.  Threads move 8 consecutive elements of a row
+// at a time (16-byte loads for bf16) when the row length and strides allow,
+// else one element.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace muon {
+
+constexpr int EW_THREADS = 256;
+constexpr int CHUNK = 8192;       // elements per chunk (a multiple of EW_THREADS * 8)
+constexpr int MAX_SEGS = 16;      // batches per elementwise launch
+
+struct EwSeg {
+  long long n, rows, cols;
+  long long chunks_per_slice;
+  long long chunk_begin;          // first global chunk of this segment
+  long long slice_begin;          // first global slice of this segment (for per-slice arrays)
+  long long row_begin;            // first global row of this segment (for per-row arrays)
+  int vec8;                       // 1: cols, strides and pointers allow 8-wide vectors
+  // tensors: (ptr, ld, batch stride, dtype: 0 f32, 1 bf16)
+  const void* g; long long g_ld, g_bs; int g_dt;
+  void* m; long long m_ld, m_bs; int m_dt;
+  void* u; long long u_ld, u_bs;                 // bf16
+  const void* o; long long o_ld, o_bs;           // bf16 (update: Newton-Schulz output)
+  void* w; long long w_ld, w_bs; int w_dt;
+  void* wc; long long wc_ld, wc_bs;              // optional bf16 copy
+  float* variance;                               // [n*rows]
+  float lr_scale;
+};
+
+struct EwParams {
+  EwSeg seg[MAX_SEGS];
+  int nseg;
+  long long total_chunks;
+  long long total_slices;
+  long long total_rows;
+  float mu;
+  int nesterov;
+  float* partials;                // [total_chunks]
+  float* sumsq_ws;                // [total_slices] (finalize writes here when a segment has no sumsq)
+  float* sumsq_out[MAX_SEGS];     // per segment output (may be null -> sumsq_ws)
+  // NorMuon / update
+  float beta2, nor_eps, lr, wd;
+  int use_normuon;
+  float* row_ss;                  // [total_rows]
+  float* row_d;                   // [total_rows]
+  float* slice_factor;            // [total_slices]
+};
+
+__device__ __forceinline__ int find_seg_by_chunk(const EwParams& P, long long c) {
+  int s = 0;
+  while (s + 1 < P.nseg && c >= P.seg[s + 1].chunk_begin) ++s;
+  return s;
+}
+
+__device__ __forceinline__ float ld_f(const void* p, long long off, int dt) {
+  if (dt == 0) return reinterpret_cast<const float*>(p)[off];
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[off]);
+}
+
+__device__ __forceinline__ void st_f(void* p, long long off, float v, int dt) {
+  if (dt == 0)
+    reinterpret_cast<float*>(p)[off] = v;
+  else
+    reinterpret_cast<__nv_bfloat16*>(p)[off] = __float2bfloat16_rn(v);
+}
+
+// 8 consecutive values (16-byte aligned) in f32 or bf16.
+__device__ __forceinline__ void ld8(const void* p, long long off, int dt, float (&v)[8]) {
+  if (dt == 0) {
+    const float4* q = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + off);
+    float4 a = q[0], b = q[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    uint4 a = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p) + off);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __bfloat162float(__ushort_as_bfloat16(static_cast<uint16_t>(w[i] & 0xFFFFu)));
+      v[2 * i + 1] = __bfloat162float(__ushort_as_bfloat16(static_cast<uint16_t>(w[i] >> 16)));
+    }
+  }
+}
+
+// Stores 8 values; returns them as rounded to the stored type.
+__device__ __forceinline__ void st8(void* p, long long off, int dt, float (&v)[8]) {
+  if (dt == 0) {
+    float4* q = reinterpret_cast<float4*>(reinterpret_cast<float*>(p) + off);
+    q[0] = make_float4(v[0], v[1], v[2], v[3]);
+    q[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat16 lo = __float2bfloat16_rn(v[2 * i]), hi = __float2bfloat16_rn(v[2 * i + 1]);
+      v[2 * i] = __bfloat162float(lo);
+      v[2 * i + 1] = __bfloat162float(hi);
+      w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+    }
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p) + off) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Fixed-order block sum (butterfly within warps, then warp 0 over warp sums).
+__device__ __forceinline__ float block_sum(float v, float* scratch) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  float t = 0.0f;
+  if (warp == 0) {
+    t = lane < (blockDim.x >> 5) ? scratch[lane] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  }
+  return t;  // valid in thread 0
+}
+
+// ---------------------------------------------------------------------------
+// Momentum, Nesterov, U = bf16, partial sum of U^2 per chunk.
+// With mode == 1 the kernel only reads U (ns_in) and forms the partial sums
+// (the Frobenius norm of a Newton-Schulz input that came without one).
+// ---------------------------------------------------------------------------
+template <int MODE>
+__global__ void __launch_bounds__(EW_THREADS) momentum_chunks_kernel(const __grid_constant__ EwParams P) {
+  __shared__ float scratch[32];
+  for (long long c = blockIdx.x; c < P.total_chunks; c += gridDim.x) {
+    const int si = find_seg_by_chunk(P, c);
+    const EwSeg& S = P.seg[si];
+    const long long local = c - S.chunk_begin;
+    const long long slice = local / S.chunks_per_slice;
+    const long long lc = local - slice * S.chunks_per_slice;
+    const long long total = S.rows * S.cols;
+    const long long e0 = lc * CHUNK;
+    const long long e1 = min(e0 + CHUNK, total);
+    float acc = 0.0f;
+    if (S.vec8) {
+      for (long long e = e0 + threadIdx.x * 8; e < e1; e += EW_THREADS * 8) {
+        const long long r = e / S.cols, col = e - r * S.cols;
+        float u[8];
+        if (MODE == 0) {
+          float g[8], m[8];
+          ld8(S.g, slice * S.g_bs + r * S.g_ld + col, S.g_dt, g);
+          ld8(S.m, slice * S.m_bs + r * S.m_ld + col, S.m_dt, m);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m[i] = P.mu * m[i] + g[i];
+          float mn[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mn[i] = m[i];
+          st8(S.m, slice * S.m_bs + r * S.m_ld + col, S.m_dt, m);   // m now holds the stored values
+#pragma unroll
+          for (int i = 0; i < 8; ++i) u[i] = P.nesterov ? g[i] + P.mu * mn[i] : mn[i];
+          st8(S.u, slice * S.u_bs + r * S.u_ld + col, 1, u);         // u now holds bf16(U)
+        } else {
+          ld8(S.u, slice * S.u_bs + r * S.u_ld + col, 1, u);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc += u[i] * u[i];
+      }
+    } else {
+      for (long long e = e0 + threadIdx.x; e < e1; e += EW_THREADS) {
+        const long long r = e / S.cols, col = e - r * S.cols;
+        float uv;
+        if (MODE == 0) {
+          const float g = ld_f(S.g, slice * S.g_bs + r * S.g_ld + col, S.g_dt);
+          const float mo = ld_f(S.m, slice * S.m_bs + r * S.m_ld + col, S.m_dt);
+          const float mn = P.mu * mo + g;
+          st_f(S.m, slice * S.m_bs + r * S.m_ld + col, mn, S.m_dt);
+          const float u = P.nesterov ? g + P.mu * mn : mn;
+          const __nv_bfloat16 ub = __float2bfloat16_rn(u);
+          reinterpret_cast<__nv_bfloat16*>(S.u)[slice * S.u_bs + r * S.u_ld + col] = ub;
+          uv = __bfloat162float(ub);
+        } else {
+          uv = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(S.u)[slice * S.u_bs + r * S.u_ld + col]);
+        }
+        acc += uv * uv;
+      }
+    }
+    const float tot = block_sum(acc, scratch);
+    if (threadIdx.x == 0) P.partials[c] = tot;
+  }
+}
+
+// One warp per slice sums that slice's chunk partials in chunk order.
+__global__ void __launch_bounds__(EW_THREADS) sumsq_finalize_kernel(const __grid_constant__ EwParams P) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (EW_THREADS / 32);
+  for (long long gs = blockIdx.x * (EW_THREADS / 32) + (threadIdx.x >> 5); gs < P.total_slices; gs += warps) {
+    int si = 0;
+    while (si + 1 < P.nseg && gs >= P.seg[si + 1].slice_begin) ++si;
+    const EwSeg& S = P.seg[si];
+    const long long slice = gs - S.slice_begin;
+    const float* part = P.partials + S.chunk_begin + slice * S.chunks_per_slice;
+    float acc = 0.0f;
+    for (long long k = lane; k < S.chunks_per_slice; k += 32) acc += part[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      float* dst = P.sumsq_out[si] ? P.sumsq_out[si] : (P.sumsq_ws + S.slice_begin);
+      dst[slice] = acc;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// NorMuon row statistics: one warp per row of O.
+//   ss = sum_j O_ij^2;  v <- beta2*v + (1-beta2)*ss/cols;  d = 1/(sqrt(v)+eps)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(EW_THREADS) normuon_rows_kernel(const __grid_constant__ EwParams P) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (EW_THREADS / 32);
+  for (long long gr = blockIdx.x * (EW_THREADS / 32) + (threadIdx.x >> 5); gr < P.total_rows; gr += warps) {
+    int si = 0;
+    while (si + 1 < P.nseg && gr >= P.seg[si + 1].row_begin) ++si;
+    const EwSeg& S = P.seg[si];
+    const long long lr = gr - S.row_begin;
+    const long long slice = lr / S.rows, r = lr - slice * S.rows;
+    const __nv_bfloat16* o = reinterpret_cast<const __nv_bfloat16*>(S.o) + slice * S.o_bs + r * S.o_ld;
+    float acc = 0.0f;
+    if (S.vec8) {
+      for (long long j = lane * 8; j < S.cols; j += 256) {
+        float v[8];
+        ld8(o, j, 1, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc += v[i] * v[i];
+      }
+    } else {
+      for (long long j = lane; j < S.cols; j += 32) {
+        const float v = __bfloat162float(o[j]);
+        acc += v * v;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      float* vp = S.variance + lr;
+      const float vn = P.beta2 * (*vp) + (1.0f - P.beta2) * (acc / static_cast<float>(S.cols));
+      *vp = vn;
+      P.row_ss[gr] = acc;
+      P.row_d[gr] = 1.0f / (sqrtf(vn) + P.nor_eps);
+    }
+  }
+}
+
+// One block per slice: factor = ||O||_F / ||O * d||_F (0 when the latter is 0).
+__global__ void __launch_bounds__(EW_THREADS) normuon_slices_kernel(const __grid_constant__ EwParams P) {
+  __shared__ float scratch[32];
+  for (long long gs = blockIdx.x; gs < P.total_slices; gs += gridDim.x) {
+    int si = 0;
+    while (si + 1 < P.nseg && gs >= P.seg[si + 1].slice_begin) ++si;
+    const EwSeg& S = P.seg[si];
+    const long long slice = gs - S.slice_begin;
+    const long long r0 = S.row_begin + slice * S.rows;
+    float s1 = 0.0f, s2 = 0.0f;
+    for (long long r = threadIdx.x; r < S.rows; r += EW_THREADS) {
+      const float ss = P.row_ss[r0 + r], d = P.row_d[r0 + r];
+      s1 += ss;
+      s2 += ss * d * d;
+    }
+    const float t1 = block_sum(s1, scratch);
+    const float t2 = block_sum(s2, scratch);
+    if (threadIdx.x == 0) P.slice_factor[gs] = t2 > 0.0f ? sqrtf(t1 / t2) : 0.0f;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// W <- W*(1 - lr*wd) - lr*lr_scale*factor*d_row * O ; optional bf16 copy.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(EW_THREADS) update_kernel(const __grid_constant__ EwParams P) {
+  const float keep = 1.0f - P.lr * P.wd;
+  for (long long c = blockIdx.x; c < P.total_chunks; c += gridDim.x) {
+    const int si = find_seg_by_chunk(P, c);
+    const EwSeg& S = P.seg[si];
+    const long long local = c - S.chunk_begin;
+    const long long slice = local / S.chunks_per_slice;
+    const long long lc = local - slice * S.chunks_per_slice;
+    const long long total = S.rows * S.cols;
+    const long long e0 = lc * CHUNK;
+    const long long e1 = min(e0 + CHUNK, total);
+    const float base = P.lr * S.lr_scale * (P.use_normuon ? P.slice_factor[S.slice_begin + slice] : 1.0f);
+    const float* rowd = P.use_normuon ? P.row_d + S.row_begin + slice * S.rows : nullptr;
+    if (S.vec8) {
+      for (long long e = e0 + threadIdx.x * 8; e < e1; e += EW_THREADS * 8) {
+        const long long r = e / S.cols, col = e - r * S.cols;
+        const float coef = rowd ? base * rowd[r] : base;
+        float o[8], w[8];
+        ld8(S.o, slice * S.o_bs + r * S.o_ld + col, 1, o);
+        ld8(S.w, slice * S.w_bs + r * S.w_ld + col, S.w_dt, w);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = fmaf(-coef, o[i], w[i] * keep);
+        st8(S.w, slice * S.w_bs + r * S.w_ld + col, S.w_dt, w);
+        if (S.wc) st8(S.wc, slice * S.wc_bs + r * S.wc_ld + col, 1, w);
+      }
+    } else {
+      for (long long e = e0 + threadIdx.x; e < e1; e += EW_THREADS) {
+        const long long r = e / S.cols, col = e - r * S.cols;
+        const float coef = rowd ? base * rowd[r] : base;
+        const float o = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(S.o)[slice * S.o_bs + r * S.o_ld + col]);
+        const long long wo = slice * S.w_bs + r * S.w_ld + col;
+        float w = ld_f(S.w, wo, S.w_dt);
+        w = fmaf(-coef, o, w * keep);
+        st_f(S.w, wo, w, S.w_dt);
+        if (S.wc) {
+          const float ws = S.w_dt == 0 ? w : __bfloat162float(__float2bfloat16_rn(w));
+          reinterpret_cast<__nv_bfloat16*>(S.wc)[slice * S.wc_bs + r * S.wc_ld + col] = __float2bfloat16_rn(ws);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace muon

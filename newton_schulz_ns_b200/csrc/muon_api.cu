@@ -1,0 +1,890 @@
+// C ABI of the Muon / NorMuon step: host-side validation, workspace layout,
+// TMA descriptor encoding and the launch sequence of every call.
+//
+// Nothing here allocates, frees or synchronizes: every kernel and memset is
+// enqueued on the caller's stream, and all scratch lives in the caller's
+// workspace.  Arguments are checked before the first enqueue; a call that
+// returns an error has enqueued nothing.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/muon_ns.h"
+#include "../../include/muon_ns_testing.h"
+#include "elementwise.cuh"
+#include "ns_gemm.cuh"
+
+using namespace muon;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kErrBytes = 256;                         // error word + padding at offset 0
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
+constexpr float kGramScale = 16384.0f;                    // A is kept as kGramScale*A in fp16
+constexpr int kMaxDevices = 64;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline int64_t round_up64(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------- device state
+struct DeviceInfo {
+  bool ready = false;
+  bool ok = false;
+  int sms = 0;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+muon_status device_setup(int* sms_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MUON_CUDA_ERROR;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    d.ready = true;
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      d.ready = false;
+      return MUON_CUDA_ERROR;
+    }
+    d.sms = sms;
+    d.ok = (major == 10 && minor == 0);
+    if (d.ok) {
+      if (cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) !=
+          cudaSuccess) {
+        d.ready = false;
+        return MUON_CUDA_ERROR;
+      }
+    }
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr) {
+        d.ready = false;
+        return MUON_CUDA_ERROR;
+      }
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  if (!d.ok) return MUON_UNSUPPORTED_DEVICE;
+  *sms_out = d.sms;
+  return MUON_OK;
+}
+
+// ---------------------------------------------------------------- validation
+inline bool dtype_is(int32_t dt, std::initializer_list<int> allowed) {
+  for (int a : allowed)
+    if (dt == a) return true;
+  return false;
+}
+inline int esize(int32_t dt) { return dt == MUON_F32 ? 4 : 2; }
+
+bool batch_empty(const muon_batch& b) { return b.n == 0 || b.rows == 0 || b.cols == 0; }
+
+muon_status check_shape(const muon_batch& b) {
+  if (b.n < 0 || b.rows < 0 || b.cols < 0) return MUON_BAD_SHAPE;
+  if (b.rows > (1 << 20) || b.cols > (1 << 20) || b.rows * b.cols > INT32_MAX || b.n > INT32_MAX)
+    return MUON_BAD_SHAPE;
+  return MUON_OK;
+}
+
+muon_status check_view(const muon_batch& b, const muon_view& v, std::initializer_list<int> dts, bool tma) {
+  if (v.ptr == nullptr) return MUON_INVALID_ARG;
+  if (!dtype_is(v.dtype, dts)) return MUON_UNSUPPORTED_DTYPE;
+  if (v.ld < b.cols) return MUON_BAD_SHAPE;
+  if (b.n > 1 && v.batch_stride < v.ld * (b.rows - 1) + b.cols) return MUON_BAD_SHAPE;
+  if (v.batch_stride < 0) return MUON_BAD_SHAPE;
+  const int es = esize(v.dtype);
+  if (reinterpret_cast<uintptr_t>(v.ptr) % es) return MUON_MISALIGNED;
+  if (tma) {
+    if (reinterpret_cast<uintptr_t>(v.ptr) % 16 || (v.ld * es) % 16 || (b.n > 1 && (v.batch_stride * es) % 16))
+      return MUON_MISALIGNED;
+  }
+  return MUON_OK;
+}
+
+bool vec8_ok(const muon_batch& b, std::initializer_list<const muon_view*> views) {
+  if (b.cols % 8) return false;
+  for (const muon_view* v : views) {
+    if (v->ptr == nullptr) continue;
+    const int es = esize(v->dtype);
+    if (reinterpret_cast<uintptr_t>(v->ptr) % 16 || (v->ld * es) % 16 || (v->batch_stride * es) % 16) return false;
+  }
+  return true;
+}
+
+muon_status check_hp(const muon_hparams* hp) {
+  if (!hp) return MUON_INVALID_ARG;
+  if (hp->ns_steps < 1 || hp->ns_steps > 16) return MUON_INVALID_ARG;
+  const float vals[] = {hp->mu, hp->ns_eps, hp->a, hp->b, hp->c, hp->beta2, hp->nor_eps, hp->lr, hp->weight_decay};
+  for (float v : vals)
+    if (!std::isfinite(v)) return MUON_INVALID_ARG;
+  if (hp->abc_schedule)
+    for (int i = 0; i < 3 * hp->ns_steps; ++i)
+      if (!std::isfinite(hp->abc_schedule[i])) return MUON_INVALID_ARG;
+  return MUON_OK;
+}
+
+muon_status check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return MUON_OK;
+  if (ws == nullptr) return MUON_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign) return MUON_MISALIGNED;
+  if (have < need) return MUON_WORKSPACE_TOO_SMALL;
+  return MUON_OK;
+}
+
+// ---------------------------------------------------------------- workspace layout
+struct NsBatchWs {
+  size_t off[5] = {0, 0, 0, 0, 0};   // standard: A, B, X ; gram: Ah, P, Qa, Qb, R
+  int64_t ldm = 0, bsm = 0;         // m x m buffers
+  int64_t ldx = 0, bsx = 0;         // X buffer
+};
+
+struct Layout {
+  size_t total = 0;
+  size_t partials = 0, sumsq = 0;   // norm reduction scratch
+  size_t row_ss = 0, row_d = 0, factor = 0;
+  std::vector<NsBatchWs> nsb;
+  int64_t total_chunks = 0, total_slices = 0, total_rows = 0;
+};
+
+Layout plan_layout(const muon_batch* bs, int nb, int which) {
+  Layout L;
+  size_t cur = kErrBytes;
+  for (int i = 0; i < nb; ++i) {
+    const muon_batch& b = bs[i];
+    if (batch_empty(b)) continue;
+    L.total_chunks += b.n * cdiv(b.rows * b.cols, CHUNK);
+    L.total_slices += b.n;
+    L.total_rows += b.n * b.rows;
+  }
+  auto take = [&](size_t bytes) {
+    const size_t o = cur;
+    cur = align_up(cur + bytes, kAlign);
+    return o;
+  };
+  L.nsb.resize(nb > 0 ? nb : 0);
+  if (which == 0 || which == 1 || which == 2) {
+    L.partials = take(sizeof(float) * std::max<int64_t>(L.total_chunks, 1));
+    L.sumsq = take(sizeof(float) * std::max<int64_t>(L.total_slices, 1));
+  }
+  if (which == 1 || which == 2) {
+    for (int i = 0; i < nb; ++i) {
+      const muon_batch& b = bs[i];
+      if (batch_empty(b)) continue;
+      const int64_t m = std::min(b.rows, b.cols);
+      NsBatchWs& w = L.nsb[i];
+      w.ldm = round_up64(m, 64);
+      w.bsm = w.ldm * m;
+      const size_t mm = sizeof(uint16_t) * static_cast<size_t>(w.bsm) * static_cast<size_t>(b.n);
+      if (which == 1) {
+        w.ldx = round_up64(b.cols, 64);
+        w.bsx = w.ldx * b.rows;
+        w.off[0] = take(mm);
+        w.off[1] = take(mm);
+        w.off[2] = take(sizeof(uint16_t) * static_cast<size_t>(w.bsx) * static_cast<size_t>(b.n));
+      } else {
+        for (int k = 0; k < 5; ++k) w.off[k] = take(mm);
+      }
+    }
+  }
+  if (which == 3) {
+    L.row_ss = take(sizeof(float) * std::max<int64_t>(L.total_rows, 1));
+    L.row_d = take(sizeof(float) * std::max<int64_t>(L.total_rows, 1));
+    L.factor = take(sizeof(float) * std::max<int64_t>(L.total_slices, 1));
+  }
+  L.total = cur;
+  return L;
+}
+
+// ---------------------------------------------------------------- tensor maps
+struct Mat {                 // a strided batch of row-major [rows][cols] matrices
+  const void* ptr;
+  int64_t rows, cols, ld, bs, n;
+  int f16;                   // element type: 1 fp16, 0 bf16
+};
+
+bool encode_map(CUtensorMap* map, const Mat& m, int box_x, int box_y) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(m.cols), static_cast<cuuint64_t>(m.rows),
+                        static_cast<cuuint64_t>(m.n)};
+  const int64_t bs = m.n > 1 ? m.bs : m.ld * m.rows;
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(m.ld * 2), static_cast<cuuint64_t>(round_up64(bs * 2, 16))};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_x), static_cast<cuuint32_t>(box_y), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, m.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                              const_cast<void*>(m.ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// One GEMM problem as the planner describes it.
+struct ProblemSpec {
+  int M, N, K, slices;
+  int tri;
+  Mat a;
+  int a_mn;                  // a is [M][K] (0) or [K][M] (1)
+  Mat b;
+  int b_mn;                  // b is [N][K] (0) or [K][N] (1)
+  int in_f16;
+  float alpha, beta, gamma, f0;
+  int s_pow;
+  float eps;
+  const float* sumsq;
+  const void* addend;
+  int64_t add_ld, add_bs;
+  int add_f16;
+  void* out;
+  int64_t out_ld, out_bs;
+  int out_f16;
+  float* row_ss;
+};
+
+muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* err, cudaStream_t stream) {
+  size_t i = 0;
+  while (i < specs.size()) {
+    GemmParams P;
+    std::memset(&P, 0, sizeof(P));
+    P.err = err;
+    P.timeout_ns = kWaitLimitNs;
+    int tiles = 0;
+    int np = 0;
+    for (; i < specs.size() && np < MAX_PROBLEMS; ++i) {
+      const ProblemSpec& s = specs[i];
+      if (s.slices == 0 || s.M == 0 || s.N == 0) continue;
+      GemmProblem& g = P.prob[np];
+      g.M = s.M;
+      g.N = s.N;
+      g.K = s.K;
+      g.slices = s.slices;
+      g.mt = static_cast<int>(cdiv(s.M, BM));
+      g.nt = static_cast<int>(cdiv(s.N, BN));
+      g.kt = static_cast<int>(cdiv(s.K, BK));
+      g.tri = s.tri;
+      if (s.tri) {
+        int cnt = 0;
+        for (int j = 0; j < g.nt; ++j) cnt += std::max(0, g.mt - 2 * j);
+        g.tiles_per_slice = cnt;
+      } else {
+        g.tiles_per_slice = g.mt * g.nt;
+      }
+      g.tile_begin = tiles;
+      g.a_mn = s.a_mn;
+      g.b_mn = s.b_mn;
+      g.idesc = mma_idesc_f16(s.in_f16 ? 0u : 1u, static_cast<uint32_t>(s.a_mn), static_cast<uint32_t>(s.b_mn), BM,
+                              BN);
+      g.alpha = s.alpha;
+      g.beta = s.beta;
+      g.gamma = s.gamma;
+      g.f0 = s.f0;
+      g.s_pow = s.s_pow;
+      g.eps = s.eps;
+      g.sumsq = s.sumsq;
+      g.addend = s.addend;
+      g.add_ld = s.add_ld;
+      g.add_bs = s.add_bs;
+      g.add_f16 = s.add_f16;
+      g.out = s.out;
+      g.out_ld = s.out_ld;
+      g.out_bs = s.out_bs;
+      g.out_f16 = s.out_f16;
+      g.row_ss = s.row_ss;
+      // A operand: K-major box 64 (K) x 128 rows; MN-major box 64 (M) x 64 (K rows).
+      if (!encode_map(&P.mapA[np], s.a, 64, s.a_mn ? 64 : BM)) return MUON_CUDA_ERROR;
+      if (!encode_map(&P.mapB[np], s.b, 64, s.b_mn ? 64 : BN)) return MUON_CUDA_ERROR;
+      const long long t = static_cast<long long>(g.tiles_per_slice) * s.slices;
+      if (tiles + t > INT32_MAX) return MUON_BAD_SHAPE;
+      tiles += static_cast<int>(t);
+      ++np;
+    }
+    if (np == 0) continue;
+    P.num_problems = np;
+    P.total_tiles = tiles;
+    const int grid = std::min(tiles, sms);
+    ns_gemm_kernel<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(P);
+    if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+  }
+  return MUON_OK;
+}
+
+// ---------------------------------------------------------------- elementwise launches
+void fill_seg_common(EwSeg& S, const muon_batch& b, long long& chunk, long long& slice, long long& row) {
+  S.n = b.n;
+  S.rows = b.rows;
+  S.cols = b.cols;
+  S.chunks_per_slice = cdiv(b.rows * b.cols, CHUNK);
+  S.chunk_begin = chunk;
+  S.slice_begin = slice;
+  S.row_begin = row;
+  chunk += b.n * S.chunks_per_slice;
+  slice += b.n;
+  row += b.n * b.rows;
+}
+
+int ew_grid(long long work, int sms) {
+  const long long cap = static_cast<long long>(sms) * 8;
+  return static_cast<int>(std::max<long long>(1, std::min(work, cap)));
+}
+
+// Launches the per-chunk U^2 partials (mode 0 also does the momentum) and the
+// per-slice finalization for one list of batches.  sumsq_ws_dev receives the
+// sums of batches whose own sumsq pointer is null.
+muon_status launch_norm(const muon_batch* bs, int nb, const muon_hparams* hp, int mode, float* partials,
+                        float* sumsq_ws_dev, int sms, cudaStream_t stream) {
+  int i = 0;
+  while (i < nb) {
+    EwParams P;
+    std::memset(&P, 0, sizeof(P));
+    long long chunk = 0, slice = 0, row = 0;
+    int ns = 0;
+    for (; i < nb && ns < MAX_SEGS; ++i) {
+      const muon_batch& b = bs[i];
+      if (batch_empty(b)) continue;
+      EwSeg& S = P.seg[ns];
+      fill_seg_common(S, b, chunk, slice, row);
+      S.g = b.grad.ptr;
+      S.g_ld = b.grad.ld;
+      S.g_bs = b.grad.batch_stride;
+      S.g_dt = b.grad.dtype == MUON_F32 ? 0 : 1;
+      S.m = b.momentum.ptr;
+      S.m_ld = b.momentum.ld;
+      S.m_bs = b.momentum.batch_stride;
+      S.m_dt = b.momentum.dtype == MUON_F32 ? 0 : 1;
+      S.u = b.ns_in.ptr;
+      S.u_ld = b.ns_in.ld;
+      S.u_bs = b.ns_in.batch_stride;
+      S.vec8 = mode == 0 ? vec8_ok(b, {&b.grad, &b.momentum, &b.ns_in}) : vec8_ok(b, {&b.ns_in});
+      P.sumsq_out[ns] = b.sumsq;
+      ++ns;
+    }
+    if (ns == 0) continue;
+    P.nseg = ns;
+    P.total_chunks = chunk;
+    P.total_slices = slice;
+    P.total_rows = row;
+    P.mu = hp ? hp->mu : 0.0f;
+    P.nesterov = hp ? hp->nesterov : 0;
+    P.partials = partials;
+    P.sumsq_ws = sumsq_ws_dev;
+    if (mode == 0)
+      momentum_chunks_kernel<0><<<ew_grid(chunk, sms), EW_THREADS, 0, stream>>>(P);
+    else
+      momentum_chunks_kernel<1><<<ew_grid(chunk, sms), EW_THREADS, 0, stream>>>(P);
+    if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+    sumsq_finalize_kernel<<<ew_grid(cdiv(slice, EW_THREADS / 32), sms), EW_THREADS, 0, stream>>>(P);
+    if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+    partials += chunk;
+    sumsq_ws_dev += slice;
+  }
+  return MUON_OK;
+}
+
+// ---------------------------------------------------------------- Newton-Schulz planning
+struct Coefs {
+  float a, b, c;
+};
+
+Coefs coefs_at(const muon_hparams* hp, int it) {
+  if (hp->abc_schedule) return Coefs{hp->abc_schedule[3 * it], hp->abc_schedule[3 * it + 1], hp->abc_schedule[3 * it + 2]};
+  return Coefs{hp->a, hp->b, hp->c};
+}
+
+Mat view_mat(const muon_batch& b, const muon_view& v) {
+  return Mat{v.ptr, b.rows, b.cols, v.ld, v.batch_stride, b.n, 0};
+}
+
+// SYRK of the slice storage X ([rows][cols]) on the short side: out = f * X X^T (rows <= cols)
+// or f * X^T X (rows > cols), lower triangle + mirror.
+ProblemSpec syrk_spec(const muon_batch& b, const Mat& x, void* out, int64_t ldm, int64_t bsm, int out_f16, float f0,
+                      int s_pow, const float* sumsq, float eps) {
+  const bool T = b.rows > b.cols;
+  const int m = static_cast<int>(std::min(b.rows, b.cols)), n = static_cast<int>(std::max(b.rows, b.cols));
+  ProblemSpec s{};
+  s.M = m;
+  s.N = m;
+  s.K = n;
+  s.slices = static_cast<int>(b.n);
+  s.tri = 1;
+  s.a = x;
+  s.a_mn = T ? 1 : 0;
+  s.b = x;
+  s.b_mn = T ? 1 : 0;
+  s.in_f16 = x.f16;
+  s.alpha = 1.0f;
+  s.f0 = f0;
+  s.s_pow = s_pow;
+  s.eps = eps;
+  s.sumsq = sumsq;
+  s.out = out;
+  s.out_ld = ldm;
+  s.out_bs = bsm;
+  s.out_f16 = out_f16;
+  return s;
+}
+
+// Symmetric m x m product out = f * (alpha * P S + beta * D) + gamma I (lower + mirror);
+// both factors are symmetric, so both are read K-major.
+ProblemSpec sym_spec(int m, int slices, const Mat& p, const Mat& q, void* out, int64_t ldm, int64_t bsm, int out_f16,
+                     float alpha, float beta, const void* add, int add_f16, float gamma) {
+  ProblemSpec s{};
+  s.M = m;
+  s.N = m;
+  s.K = m;
+  s.slices = slices;
+  s.tri = 1;
+  s.a = p;
+  s.a_mn = 0;
+  s.b = q;
+  s.b_mn = 0;
+  s.in_f16 = p.f16;
+  s.alpha = alpha;
+  s.beta = beta;
+  s.gamma = gamma;
+  s.f0 = 1.0f;
+  s.addend = add;
+  s.add_ld = ldm;
+  s.add_bs = bsm;
+  s.add_f16 = add_f16;
+  s.out = out;
+  s.out_ld = ldm;
+  s.out_bs = bsm;
+  s.out_f16 = out_f16;
+  return s;
+}
+
+// Applies the symmetric m x m factor F (bf16) to the slice storage X on the
+// short side: out = f * (F X + beta X) when rows <= cols, or
+// out = f * (X F + beta X) in the transposed case; out has X's layout.
+ProblemSpec apply_spec(const muon_batch& b, const Mat& f, const Mat& x, void* out, int64_t out_ld, int64_t out_bs,
+                       float beta, int s_pow, const float* sumsq, float eps, float* row_ss) {
+  const bool T = b.rows > b.cols;
+  const int m = static_cast<int>(std::min(b.rows, b.cols));
+  ProblemSpec s{};
+  s.slices = static_cast<int>(b.n);
+  s.tri = 0;
+  s.in_f16 = 0;
+  if (!T) {
+    s.M = m;
+    s.N = static_cast<int>(b.cols);
+    s.K = m;
+    s.a = f;
+    s.a_mn = 0;
+    s.b = x;
+    s.b_mn = 1;
+  } else {
+    s.M = static_cast<int>(b.rows);
+    s.N = m;
+    s.K = m;
+    s.a = x;
+    s.a_mn = 0;
+    s.b = f;
+    s.b_mn = 0;
+  }
+  s.alpha = 1.0f;
+  s.beta = beta;
+  s.f0 = 1.0f;
+  s.s_pow = s_pow;
+  s.eps = eps;
+  s.sumsq = sumsq;
+  s.addend = beta != 0.0f ? x.ptr : nullptr;
+  s.add_ld = x.ld;
+  s.add_bs = x.bs;
+  s.add_f16 = 0;
+  s.out = out;
+  s.out_ld = out_ld;
+  s.out_bs = out_bs;
+  s.out_f16 = 0;
+  s.row_ss = row_ss;
+  return s;
+}
+
+muon_status validate_ns(const muon_batch* bs, int nb, const muon_hparams* hp) {
+  if (nb < 0 || (nb > 0 && bs == nullptr)) return MUON_INVALID_ARG;
+  muon_status st = check_hp(hp);
+  if (st != MUON_OK) return st;
+  for (int i = 0; i < nb; ++i) {
+    const muon_batch& b = bs[i];
+    if ((st = check_shape(b)) != MUON_OK) return st;
+    if (batch_empty(b)) continue;
+    if ((st = check_view(b, b.ns_in, {MUON_BF16}, true)) != MUON_OK) return st;
+    if ((st = check_view(b, b.ns_out, {MUON_BF16}, true)) != MUON_OK) return st;
+    if (b.ns_in.ptr == b.ns_out.ptr) return MUON_INVALID_ARG;
+  }
+  return MUON_OK;
+}
+
+// Clears the error word and makes sure every batch has a per-slice sum of squares.
+// Returns the per-batch sumsq pointers to use.
+muon_status prepare_norms(const muon_batch* bs, int nb, const Layout& L, uint8_t* ws, int sms, cudaStream_t stream,
+                          std::vector<const float*>& sumsq) {
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), stream) != cudaSuccess) return MUON_CUDA_ERROR;
+  sumsq.assign(nb, nullptr);
+  std::vector<muon_batch> missing;
+  float* base = reinterpret_cast<float*>(ws + L.sumsq);
+  float* cur = base;
+  for (int i = 0; i < nb; ++i) {
+    if (batch_empty(bs[i])) continue;
+    if (bs[i].sumsq) {
+      sumsq[i] = bs[i].sumsq;
+    } else {
+      muon_batch c = bs[i];
+      c.sumsq = nullptr;
+      missing.push_back(c);
+      sumsq[i] = cur;
+      cur += bs[i].n;
+    }
+  }
+  if (!missing.empty())
+    return launch_norm(missing.data(), static_cast<int>(missing.size()), nullptr, 1,
+                       reinterpret_cast<float*>(ws + L.partials), base, sms, stream);
+  return MUON_OK;
+}
+
+}  // namespace
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+const char* muon_version(void) { return "0.1.0"; }
+
+const char* muon_status_string(muon_status s) {
+  switch (s) {
+    case MUON_OK: return "ok";
+    case MUON_INVALID_ARG: return "invalid argument";
+    case MUON_BAD_SHAPE: return "bad shape or strides";
+    case MUON_UNSUPPORTED_DTYPE: return "unsupported dtype";
+    case MUON_MISALIGNED: return "misaligned pointer or stride (16-byte TMA rule, 256-byte workspace rule)";
+    case MUON_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MUON_CUDA_ERROR: return "CUDA error";
+    case MUON_UNSUPPORTED_DEVICE: return "current device is not sm_100 (B200)";
+  }
+  return "unknown status";
+}
+
+size_t muon_workspace_size(const muon_batch* batches, int nb, int which) {
+  if (nb < 0 || (nb > 0 && !batches) || which < -1 || which > 3) return 0;
+  for (int i = 0; i < nb; ++i)
+    if (check_shape(batches[i]) != MUON_OK) return 0;
+  if (which == -1) {
+    size_t m = 0;
+    for (int w = 0; w < 4; ++w) m = std::max(m, plan_layout(batches, nb, w).total);
+    return m;
+  }
+  return plan_layout(batches, nb, which).total;
+}
+
+muon_status muon_workspace_error(const void* workspace, cudaStream_t stream, int32_t* error_word) {
+  if (!workspace || !error_word) return MUON_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MUON_CUDA_ERROR;
+  if (cudaMemcpy(error_word, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MUON_CUDA_ERROR;
+  return MUON_OK;
+}
+
+muon_status muon_momentum_norm(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
+                               size_t workspace_bytes, cudaStream_t stream) {
+  if (nb < 0 || (nb > 0 && !batches)) return MUON_INVALID_ARG;
+  muon_status st = check_hp(hp);
+  if (st != MUON_OK) return st;
+  bool any = false;
+  for (int i = 0; i < nb; ++i) {
+    const muon_batch& b = batches[i];
+    if ((st = check_shape(b)) != MUON_OK) return st;
+    if (batch_empty(b)) continue;
+    any = true;
+    if ((st = check_view(b, b.grad, {MUON_F32, MUON_BF16}, false)) != MUON_OK) return st;
+    if ((st = check_view(b, b.momentum, {MUON_F32, MUON_BF16}, false)) != MUON_OK) return st;
+    if ((st = check_view(b, b.ns_in, {MUON_BF16}, false)) != MUON_OK) return st;
+    if (!b.sumsq) return MUON_INVALID_ARG;
+  }
+  if (!any) return MUON_OK;
+  const Layout L = plan_layout(batches, nb, 0);
+  if ((st = check_ws(workspace, workspace_bytes, L.total)) != MUON_OK) return st;
+  int sms = 0;
+  if ((st = device_setup(&sms)) != MUON_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return launch_norm(batches, nb, hp, 0, reinterpret_cast<float*>(ws + L.partials),
+                     reinterpret_cast<float*>(ws + L.sumsq), sms, stream);
+}
+
+muon_status muon_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream) {
+  muon_status st = validate_ns(batches, nb, hp);
+  if (st != MUON_OK) return st;
+  bool any = false;
+  for (int i = 0; i < nb; ++i) any |= !batch_empty(batches[i]);
+  if (!any) return MUON_OK;
+  const Layout L = plan_layout(batches, nb, 1);
+  if ((st = check_ws(workspace, workspace_bytes, L.total)) != MUON_OK) return st;
+  int sms = 0;
+  if ((st = device_setup(&sms)) != MUON_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  std::vector<const float*> sumsq;
+  if ((st = prepare_norms(batches, nb, L, ws, sms, stream, sumsq)) != MUON_OK) return st;
+  int* err = reinterpret_cast<int*>(ws);
+
+  const int S = hp->ns_steps;
+  for (int it = 0; it < S; ++it) {
+    const Coefs cf = coefs_at(hp, it);
+    std::vector<ProblemSpec> syrk, poly, apply;
+    for (int i = 0; i < nb; ++i) {
+      const muon_batch& b = batches[i];
+      if (batch_empty(b)) continue;
+      const NsBatchWs& w = L.nsb[i];
+      const int m = static_cast<int>(std::min(b.rows, b.cols));
+      void* Abuf = ws + w.off[0];
+      void* Bbuf = ws + w.off[1];
+      void* Xws = ws + w.off[2];
+      // Writes alternate between ns_out and the X workspace so the last lands in ns_out.
+      auto buf = [&](int k) -> Mat {
+        if (k < 0) return view_mat(b, b.ns_in);
+        if ((S - 1 - k) % 2 == 0) return view_mat(b, b.ns_out);
+        return Mat{Xws, b.rows, b.cols, w.ldx, w.bsx, b.n, 0};
+      };
+      const Mat src = buf(it - 1), dst = buf(it);
+      const Mat Am{Abuf, m, m, w.ldm, w.bsm, b.n, 0};
+      const Mat Bm{Bbuf, m, m, w.ldm, w.bsm, b.n, 0};
+      syrk.push_back(syrk_spec(b, src, Abuf, w.ldm, w.bsm, 0, 1.0f, it == 0 ? 2 : 0, sumsq[i], hp->ns_eps));
+      poly.push_back(sym_spec(m, static_cast<int>(b.n), Am, Am, Bbuf, w.ldm, w.bsm, 0, cf.c, cf.b, Abuf, 0, 0.0f));
+      apply.push_back(apply_spec(b, Bm, src, const_cast<void*>(dst.ptr), dst.ld, dst.bs, cf.a, it == 0 ? 1 : 0,
+                                 sumsq[i], hp->ns_eps, nullptr));
+    }
+    if ((st = launch_gemms(syrk, sms, err, stream)) != MUON_OK) return st;
+    if ((st = launch_gemms(poly, sms, err, stream)) != MUON_OK) return st;
+    if ((st = launch_gemms(apply, sms, err, stream)) != MUON_OK) return st;
+  }
+  return MUON_OK;
+}
+
+muon_status muon_gram_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+  muon_status st = validate_ns(batches, nb, hp);
+  if (st != MUON_OK) return st;
+  bool any = false;
+  for (int i = 0; i < nb; ++i) any |= !batch_empty(batches[i]);
+  if (!any) return MUON_OK;
+  const Layout L = plan_layout(batches, nb, 2);
+  if ((st = check_ws(workspace, workspace_bytes, L.total)) != MUON_OK) return st;
+  int sms = 0;
+  if ((st = device_setup(&sms)) != MUON_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  std::vector<const float*> sumsq;
+  if ((st = prepare_norms(batches, nb, L, ws, sms, stream, sumsq)) != MUON_OK) return st;
+  int* err = reinterpret_cast<int*>(ws);
+  const int S = hp->ns_steps;
+  const float kap = kGramScale;
+
+  // G: kappa * s^2 * X X^T (short side) in fp16.
+  {
+    std::vector<ProblemSpec> g;
+    for (int i = 0; i < nb; ++i) {
+      const muon_batch& b = batches[i];
+      if (batch_empty(b)) continue;
+      const NsBatchWs& w = L.nsb[i];
+      g.push_back(syrk_spec(b, view_mat(b, b.ns_in), ws + w.off[0], w.ldm, w.bsm, 1, kap, 2, sumsq[i], hp->ns_eps));
+    }
+    if ((st = launch_gemms(g, sms, err, stream)) != MUON_OK) return st;
+  }
+  // Buffers: 0 Ah (kappa*A), 1 P, 2 Qa, 3 Qb, 4 R.  P of step 0 is written to Qa (Q_1 = P_1).
+  int qcur = 2;
+  for (int k = 0; k < S; ++k) {
+    const Coefs cf = coefs_at(hp, k);
+    const bool last = (k == S - 1);
+    std::vector<ProblemSpec> t_l, qr_l, a_l;
+    int qnext = qcur;
+    for (int i = 0; i < nb; ++i) {
+      const muon_batch& b = batches[i];
+      if (batch_empty(b)) continue;
+      const NsBatchWs& w = L.nsb[i];
+      const int m = static_cast<int>(std::min(b.rows, b.cols));
+      const int sl = static_cast<int>(b.n);
+      auto M16 = [&](int idx, int f16) { return Mat{ws + w.off[idx], m, m, w.ldm, w.bsm, b.n, f16}; };
+      const int pidx = (k == 0) ? 2 : 1;
+      // P = a I + (b/kappa) Ah + (c/kappa^2) Ah^2 ; bf16 when it is the final Q (one step only).
+      const int p_f16 = (k == 0 && last) ? 0 : 1;
+      t_l.push_back(sym_spec(m, sl, M16(0, 1), M16(0, 1), ws + w.off[pidx], w.ldm, w.bsm, p_f16, cf.c / (kap * kap),
+                             cf.b / kap, ws + w.off[0], 1, cf.a));
+      if (k > 0) {
+        qnext = (qcur == 2) ? 3 : 2;
+        qr_l.push_back(sym_spec(m, sl, M16(1, 1), M16(qcur, 1), ws + w.off[qnext], w.ldm, w.bsm, last ? 0 : 1, 1.0f,
+                                0.0f, nullptr, 1, 0.0f));
+      }
+      if (!last) {
+        qr_l.push_back(sym_spec(m, sl, M16(pidx, 1), M16(0, 1), ws + w.off[4], w.ldm, w.bsm, 1, 1.0f, 0.0f, nullptr,
+                                1, 0.0f));
+        a_l.push_back(sym_spec(m, sl, M16(pidx, 1), M16(4, 1), ws + w.off[0], w.ldm, w.bsm, 1, 1.0f, 0.0f, nullptr,
+                               1, 0.0f));
+      }
+    }
+    if ((st = launch_gemms(t_l, sms, err, stream)) != MUON_OK) return st;
+    if ((st = launch_gemms(qr_l, sms, err, stream)) != MUON_OK) return st;
+    if ((st = launch_gemms(a_l, sms, err, stream)) != MUON_OK) return st;
+    qcur = qnext;
+  }
+  // O = s * Q X0 on the short side, Q in bf16.
+  {
+    std::vector<ProblemSpec> o;
+    for (int i = 0; i < nb; ++i) {
+      const muon_batch& b = batches[i];
+      if (batch_empty(b)) continue;
+      const NsBatchWs& w = L.nsb[i];
+      const int m = static_cast<int>(std::min(b.rows, b.cols));
+      const Mat Q{ws + w.off[qcur], m, m, w.ldm, w.bsm, b.n, 0};
+      const Mat out = view_mat(b, b.ns_out);
+      o.push_back(apply_spec(b, Q, view_mat(b, b.ns_in), const_cast<void*>(out.ptr), out.ld, out.bs, 0.0f, 1,
+                             sumsq[i], hp->ns_eps, nullptr));
+    }
+    if ((st = launch_gemms(o, sms, err, stream)) != MUON_OK) return st;
+  }
+  return MUON_OK;
+}
+
+muon_status normuon_update(const muon_batch* batches, int nb, const muon_hparams* hp, int use_normuon,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (nb < 0 || (nb > 0 && !batches)) return MUON_INVALID_ARG;
+  muon_status st = check_hp(hp);
+  if (st != MUON_OK) return st;
+  bool any = false;
+  for (int i = 0; i < nb; ++i) {
+    const muon_batch& b = batches[i];
+    if ((st = check_shape(b)) != MUON_OK) return st;
+    if (batch_empty(b)) continue;
+    any = true;
+    if ((st = check_view(b, b.ns_out, {MUON_BF16}, false)) != MUON_OK) return st;
+    if ((st = check_view(b, b.weight, {MUON_F32, MUON_BF16}, false)) != MUON_OK) return st;
+    if (b.weight_copy.ptr && (st = check_view(b, b.weight_copy, {MUON_BF16}, false)) != MUON_OK) return st;
+    if (use_normuon && !b.variance) return MUON_INVALID_ARG;
+    if (!std::isfinite(b.lr_scale)) return MUON_INVALID_ARG;
+  }
+  if (!any) return MUON_OK;
+  const Layout L = plan_layout(batches, nb, 3);
+  if ((st = check_ws(workspace, workspace_bytes, L.total)) != MUON_OK) return st;
+  int sms = 0;
+  if ((st = device_setup(&sms)) != MUON_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* row_ss = reinterpret_cast<float*>(ws + L.row_ss);
+  float* row_d = reinterpret_cast<float*>(ws + L.row_d);
+  float* factor = reinterpret_cast<float*>(ws + L.factor);
+  int i = 0;
+  while (i < nb) {
+    EwParams P;
+    std::memset(&P, 0, sizeof(P));
+    long long chunk = 0, slice = 0, row = 0;
+    int ns = 0;
+    for (; i < nb && ns < MAX_SEGS; ++i) {
+      const muon_batch& b = batches[i];
+      if (batch_empty(b)) continue;
+      EwSeg& S = P.seg[ns];
+      fill_seg_common(S, b, chunk, slice, row);
+      S.o = b.ns_out.ptr;
+      S.o_ld = b.ns_out.ld;
+      S.o_bs = b.ns_out.batch_stride;
+      S.w = b.weight.ptr;
+      S.w_ld = b.weight.ld;
+      S.w_bs = b.weight.batch_stride;
+      S.w_dt = b.weight.dtype == MUON_F32 ? 0 : 1;
+      S.wc = b.weight_copy.ptr;
+      S.wc_ld = b.weight_copy.ld;
+      S.wc_bs = b.weight_copy.batch_stride;
+      S.variance = b.variance;
+      S.lr_scale = b.lr_scale;
+      S.vec8 = vec8_ok(b, {&b.ns_out, &b.weight, &b.weight_copy});
+      ++ns;
+    }
+    if (ns == 0) continue;
+    P.nseg = ns;
+    P.total_chunks = chunk;
+    P.total_slices = slice;
+    P.total_rows = row;
+    P.beta2 = hp->beta2;
+    P.nor_eps = hp->nor_eps;
+    P.lr = hp->lr;
+    P.wd = hp->weight_decay;
+    P.use_normuon = use_normuon ? 1 : 0;
+    P.row_ss = row_ss;
+    P.row_d = row_d;
+    P.slice_factor = factor;
+    if (use_normuon) {
+      normuon_rows_kernel<<<ew_grid(cdiv(row, EW_THREADS / 32), sms), EW_THREADS, 0, stream>>>(P);
+      if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+      normuon_slices_kernel<<<ew_grid(slice, sms), EW_THREADS, 0, stream>>>(P);
+      if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+    }
+    update_kernel<<<ew_grid(chunk, sms), EW_THREADS, 0, stream>>>(P);
+    if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+  }
+  return MUON_OK;
+}
+
+muon_status muon_testing_gemm(int M, int N, int K, int slices, int tri, int in_dtype, const void* A, int64_t lda,
+                              int64_t bsa, int a_mn, const void* B, int64_t ldb, int64_t bsb, int b_mn,
+                              const void* D, int64_t ldd, int64_t bsd, int add_dtype, void* C, int64_t ldc,
+                              int64_t bsc, int out_dtype, float alpha, float beta, float gamma, float f0, int s_pow,
+                              const float* sumsq, float eps, float* row_ss, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
+  if (M < 0 || N < 0 || K < 1 || slices < 0) return MUON_BAD_SHAPE;
+  if (tri && M != N) return MUON_BAD_SHAPE;
+  if (!A || !B || !C) return MUON_INVALID_ARG;
+  if (beta != 0.0f && !D) return MUON_INVALID_ARG;
+  if (s_pow < 0 || s_pow > 2 || (s_pow > 0 && !sumsq)) return MUON_INVALID_ARG;
+  if (!dtype_is(in_dtype, {MUON_BF16, MUON_F16}) || !dtype_is(out_dtype, {MUON_BF16, MUON_F16}) ||
+      !dtype_is(add_dtype, {MUON_BF16, MUON_F16}))
+    return MUON_UNSUPPORTED_DTYPE;
+  auto al = [](const void* p, int64_t ld, int64_t bs) {
+    return reinterpret_cast<uintptr_t>(p) % 16 == 0 && (ld * 2) % 16 == 0 && (bs * 2) % 16 == 0;
+  };
+  if (!al(A, lda, bsa) || !al(B, ldb, bsb) || !al(C, ldc, bsc) || (D && !al(D, ldd, bsd))) return MUON_MISALIGNED;
+  muon_status st = check_ws(workspace, workspace_bytes, kErrBytes);
+  if (st != MUON_OK) return st;
+  if (M == 0 || N == 0 || slices == 0) return MUON_OK;
+  int sms = 0;
+  if ((st = device_setup(&sms)) != MUON_OK) return st;
+  if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), stream) != cudaSuccess) return MUON_CUDA_ERROR;
+  const int f16 = in_dtype == MUON_F16;
+  ProblemSpec s{};
+  s.M = M;
+  s.N = N;
+  s.K = K;
+  s.slices = slices;
+  s.tri = tri;
+  s.a = a_mn ? Mat{A, K, M, lda, bsa, slices, f16} : Mat{A, M, K, lda, bsa, slices, f16};
+  s.a_mn = a_mn;
+  s.b = b_mn ? Mat{B, K, N, ldb, bsb, slices, f16} : Mat{B, N, K, ldb, bsb, slices, f16};
+  s.b_mn = b_mn;
+  s.in_f16 = f16;
+  s.alpha = alpha;
+  s.beta = beta;
+  s.gamma = gamma;
+  s.f0 = f0;
+  s.s_pow = s_pow;
+  s.eps = eps;
+  s.sumsq = sumsq;
+  s.addend = D;
+  s.add_ld = ldd;
+  s.add_bs = bsd;
+  s.add_f16 = add_dtype == MUON_F16;
+  s.out = C;
+  s.out_ld = ldc;
+  s.out_bs = bsc;
+  s.out_f16 = out_dtype == MUON_F16;
+  s.row_ss = tri ? nullptr : row_ss;
+  std::vector<ProblemSpec> v{s};
+  return launch_gemms(v, sms, reinterpret_cast<int*>(workspace), stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,424 @@
+// Persistent grouped tensor-core GEMM for the Newton-Schulz iteration (sm_100a).
+//
+// One launch runs up to MAX_PROBLEMS "problems"; a problem is a batch of
+// same-shape slices C[s] = epilogue(opA(A[s]) * opB(B[s])) with
+//   opA: M x K, stored K-major ([M][K] row-major) or MN-major ([K][M]);
+//   opB: K x N, stored K-major ([N][K], i.e. C = A B^T) or MN-major ([K][N]).
+// Tiles are 128 x 256 (BM x BN) with 64-wide K blocks.  Operands are
+// brought into shared memory by TMA (128-byte swizzle, zero fill outside the
+// slice), multiplied by tcgen05.mma (bf16 or fp16 in, fp32 accumulate in
+// TMEM), and the epilogue applies
+//   C = f * (alpha * acc + beta * D) + gamma * [row == col]
+// where D is an addend with C's shape and f = f0 * s^p per slice, with
+// s = 1 / (sqrt(sumsq[slice]) + eps) and p in {0, 1, 2}.
+//
+// Symmetric problems ("tri") compute only the 128x256 tiles that touch the
+// lower triangle and write each lower element and its mirror, so A = X X^T
+// and B = b*A + c*A^2 cost about half of a full product (the one-triangle
+// products of the Megatron-Core layer_sharded_muon docs, use_syrk).
+//
+// Roles (192 threads, one CTA per SM, persistent over a static tile stride):
+//   warp 0 lane 0 : TMA producer over a STAGES-deep shared-memory ring
+//   warp 1        : TMEM allocation; lane 0 issues the MMAs
+//   warps 2..5    : epilogue, one TMEM lane (= output row) per thread;
+//                   two 256-column accumulators let the epilogue of one
+//                   tile overlap the main loop of the next.
+// Every wait is bounded (see mbar_wait_bounded); a role that gives up
+// records an error code in *err, raises the CTA's abort flag and leaves;
+// in-flight TMA loads and MMAs are waited for (bounded) before TMEM is freed.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "ptx_sm100.cuh"
+
+namespace muon {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_STAGE_BYTES = BM * BK * 2;
+constexpr int B_STAGE_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int MN_BLOCK_BYTES = 64 * BK * 2;      // one [64 K rows][64 MN] swizzled block
+constexpr uint32_t TMEM_COLS = 2 * BN;           // two accumulators
+constexpr int GEMM_THREADS = 192;
+constexpr int MAX_PROBLEMS = 8;
+constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+enum GemmError : int { kErrNone = 0, kErrProducer = 1, kErrMma = 2, kErrEpilogue = 3 };
+
+struct GemmProblem {
+  int M, N, K;
+  int slices;
+  int mt, nt, kt;           // tile counts along M, N, K
+  int tiles_per_slice;
+  int tile_begin;           // first linear tile of this problem in the launch
+  int tri;                  // symmetric output: lower-triangle tiles + mirror
+  int a_mn, b_mn;           // operand majors (1 = MN-major)
+  uint32_t idesc;           // tcgen05 instruction descriptor
+  float alpha, beta, gamma, f0;
+  int s_pow;                // exponent of the per-slice normalization factor
+  float eps;
+  const float* sumsq;       // [slices] when s_pow > 0
+  const void* addend;       // D (same dtype as C), may be null when beta == 0
+  long long add_ld, add_bs;
+  void* out;
+  long long out_ld, out_bs;
+  int out_f16;              // 1: C is fp16, 0: bf16
+  int add_f16;              // 1: D is fp16, 0: bf16
+  float* row_ss;            // optional [slices][nt][M]: sum over the tile's columns of bf16(C)^2
+};
+
+struct __align__(64) GemmParams {
+  CUtensorMap mapA[MAX_PROBLEMS];
+  CUtensorMap mapB[MAX_PROBLEMS];
+  GemmProblem prob[MAX_PROBLEMS];
+  int num_problems;
+  int total_tiles;
+  int* err;
+  unsigned long long timeout_ns;
+};
+
+struct TileCoord {
+  int p, slice, tm, tn;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const GemmParams& P, int t) {
+  int p = 0;
+  while (p + 1 < P.num_problems && t >= P.prob[p + 1].tile_begin) ++p;
+  const GemmProblem& pr = P.prob[p];
+  const int local = t - pr.tile_begin;
+  const int slice = local / pr.tiles_per_slice;
+  int r = local - slice * pr.tiles_per_slice;
+  int tm, tn;
+  if (pr.tri) {
+    // Column j of 256 output columns needs row tiles 2j .. mt-1.
+    int j = 0;
+    while (r >= pr.mt - 2 * j) {
+      r -= pr.mt - 2 * j;
+      ++j;
+    }
+    tn = j;
+    tm = 2 * j + r;
+  } else {
+    tm = r % pr.mt;
+    tn = r / pr.mt;
+  }
+  return TileCoord{p, slice, tm, tn};
+}
+
+__device__ __forceinline__ void record_error(int* err, volatile int* abort_flag, int code) {
+  *abort_flag = 1;
+  if (err) atomicCAS(err, 0, code);
+}
+
+__device__ __forceinline__ float load_elem(const void* base, long long off, int f16) {
+  if (f16) return __half2float(reinterpret_cast<const __half*>(base)[off]);
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[off]);
+}
+
+// Rounds v to the output type, stores it, and returns the rounded value.
+__device__ __forceinline__ float store_elem(void* base, long long off, float v, int f16) {
+  if (f16) {
+    __half h = __float2half_rn(v);
+    reinterpret_cast<__half*>(base)[off] = h;
+    return __half2float(h);
+  }
+  __nv_bfloat16 h = __float2bfloat16_rn(v);
+  reinterpret_cast<__nv_bfloat16*>(base)[off] = h;
+  return __bfloat162float(h);
+}
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_constant__ GemmParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t limit = P.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int p = 0; p < P.num_problems; ++p) {
+      tma_prefetch_desc(&P.mapA[p]);
+      tma_prefetch_desc(&P.mapB[p]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t last_par[STAGES];
+      bool used[STAGES];
+      for (int s = 0; s < STAGES; ++s) {
+        used[s] = false;
+        last_par[s] = 0;
+      }
+      bool ok = true;
+      for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = decode_tile(P, t);
+        const GemmProblem& pr = P.prob[tc.p];
+        for (int kb = 0; kb < pr.kt; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit)) {
+            record_error(P.err, abort_flag, kErrProducer);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          uint8_t* a_dst = sA + stage * A_STAGE_BYTES;
+          uint8_t* b_dst = sB + stage * B_STAGE_BYTES;
+          const int k0 = kb * BK;
+          if (!pr.a_mn) {
+            tma_load_3d(a_dst, &P.mapA[tc.p], &full[stage], k0, tc.tm * BM, tc.slice);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BM / 64; ++c)
+              tma_load_3d(a_dst + c * MN_BLOCK_BYTES, &P.mapA[tc.p], &full[stage], tc.tm * BM + 64 * c, k0,
+                          tc.slice);
+          }
+          if (!pr.b_mn) {
+            tma_load_3d(b_dst, &P.mapB[tc.p], &full[stage], k0, tc.tn * BN, tc.slice);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_3d(b_dst + c * MN_BLOCK_BYTES, &P.mapB[tc.p], &full[stage], tc.tn * BN + 64 * c, k0,
+                          tc.slice);
+          }
+          used[stage] = true;
+          last_par[stage] = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Leave no bulk copy in flight into shared memory.
+        for (int s = 0; s < STAGES; ++s)
+          if (used[s]) {
+            volatile int never = 0;
+            mbar_wait_bounded(&full[s], last_par[s], &never, limit);
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int iter = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x, ++iter) {
+        const TileCoord tc = decode_tile(P, t);
+        const GemmProblem& pr = P.prob[tc.p];
+        const int acc = iter & 1;
+        const uint32_t acc_par = (iter >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[acc], acc_par ^ 1u, abort_flag, limit)) {
+          record_error(P.err, abort_flag, kErrMma);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < pr.kt; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, limit)) {
+            record_error(P.err, abort_flag, kErrMma);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * B_STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            // K-major: 16 elements = 32 bytes along the swizzled row.
+            // MN-major: 16 K rows = two 8-row groups of 1024 bytes.
+            const uint64_t ad = pr.a_mn ? smem_desc_sw128(a_base + k * 2048, MN_BLOCK_BYTES, 1024)
+                                        : smem_desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = pr.b_mn ? smem_desc_sw128(b_base + k * 2048, MN_BLOCK_BYTES, 1024)
+                                        : smem_desc_sw128(b_base + k * 32, 16, 1024);
+            tc_mma_f16(d_tmem, ad, bd, pr.idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+      }
+      // Every MMA this thread issued has finished before TMEM can be freed.
+      tc_commit(drain);
+      volatile int never = 0;
+      if (!mbar_wait_bounded(drain, 0, &never, limit)) record_error(P.err, abort_flag, kErrMma);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    int iter = 0;
+    for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++iter) {
+      const TileCoord tc = decode_tile(P, t);
+      const GemmProblem& pr = P.prob[tc.p];
+      const int acc = iter & 1;
+      const uint32_t acc_par = (iter >> 1) & 1;
+      bool ok = mbar_wait_bounded(&tfull[acc], acc_par, abort_flag, limit);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) record_error(P.err, abort_flag, kErrEpilogue);
+        break;
+      }
+      tc_fence_after();
+
+      const int row = tc.tm * BM + q * 32 + lane;
+      const bool row_ok = row < pr.M;
+      float f = pr.f0;
+      if (pr.s_pow > 0) {
+        const float s = 1.0f / (sqrtf(pr.sumsq[tc.slice]) + pr.eps);
+        f *= (pr.s_pow == 2) ? s * s : s;
+      }
+      const long long out_slice = static_cast<long long>(tc.slice) * pr.out_bs;
+      const long long add_slice = static_cast<long long>(tc.slice) * pr.add_bs;
+      const bool use_add = pr.beta != 0.0f && pr.addend != nullptr;
+      float rss = 0.0f;
+
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + c * 32),
+                           r);
+        tmem_ld_wait();
+        const int col0 = tc.tn * BN + c * 32;
+        if (col0 >= pr.N || !row_ok) continue;
+        const bool full_chunk = col0 + 32 <= pr.N;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = pr.alpha * __uint_as_float(r[j]);
+        if (use_add) {
+          const long long aoff = add_slice + static_cast<long long>(row) * pr.add_ld + col0;
+          if (full_chunk) {
+            const uint4* src = reinterpret_cast<const uint4*>(
+                reinterpret_cast<const uint16_t*>(pr.addend) + aoff);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              uint4 u = src[w];
+              const uint32_t words[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const uint16_t lo = static_cast<uint16_t>(words[h] & 0xFFFFu);
+                const uint16_t hi = static_cast<uint16_t>(words[h] >> 16);
+                float flo, fhi;
+                if (pr.add_f16) {
+                  flo = __half2float(__ushort_as_half(lo));
+                  fhi = __half2float(__ushort_as_half(hi));
+                } else {
+                  flo = __bfloat162float(__ushort_as_bfloat16(lo));
+                  fhi = __bfloat162float(__ushort_as_bfloat16(hi));
+                }
+                v[w * 8 + h * 2] += pr.beta * flo;
+                v[w * 8 + h * 2 + 1] += pr.beta * fhi;
+              }
+            }
+          } else {
+            for (int j = 0; j < 32 && col0 + j < pr.N; ++j) v[j] += pr.beta * load_elem(pr.addend, aoff + j, pr.add_f16);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] *= f;
+        if (pr.tri) {
+          for (int j = 0; j < 32; ++j) {
+            const int col = col0 + j;
+            if (col >= pr.N || col > row) break;
+            float x = v[j];
+            if (col == row) x += pr.gamma;
+            store_elem(pr.out, out_slice + static_cast<long long>(row) * pr.out_ld + col, x, pr.out_f16);
+            if (col < row) store_elem(pr.out, out_slice + static_cast<long long>(col) * pr.out_ld + row, x, pr.out_f16);
+          }
+        } else {
+          const long long ooff = out_slice + static_cast<long long>(row) * pr.out_ld + col0;
+          if (full_chunk) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              uint16_t lo, hi;
+              float rlo, rhi;
+              if (pr.out_f16) {
+                __half a = __float2half_rn(v[2 * j]), b = __float2half_rn(v[2 * j + 1]);
+                lo = __half_as_ushort(a);
+                hi = __half_as_ushort(b);
+                rlo = __half2float(a);
+                rhi = __half2float(b);
+              } else {
+                __nv_bfloat16 a = __float2bfloat16_rn(v[2 * j]), b = __float2bfloat16_rn(v[2 * j + 1]);
+                lo = __bfloat16_as_ushort(a);
+                hi = __bfloat16_as_ushort(b);
+                rlo = __bfloat162float(a);
+                rhi = __bfloat162float(b);
+              }
+              rss += rlo * rlo + rhi * rhi;
+              packed[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(pr.out) + ooff);
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+              dst[w] = make_uint4(packed[4 * w], packed[4 * w + 1], packed[4 * w + 2], packed[4 * w + 3]);
+          } else {
+            for (int j = 0; j < 32 && col0 + j < pr.N; ++j) {
+              const float x = store_elem(pr.out, ooff + j, v[j], pr.out_f16);
+              rss += x * x;
+            }
+          }
+        }
+      }
+      if (pr.row_ss != nullptr && row_ok)
+        pr.row_ss[(static_cast<long long>(tc.slice) * pr.nt + tc.tn) * pr.M + row] = rss;
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace muon

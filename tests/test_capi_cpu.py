@@ -1,0 +1,148 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load, export every function the public headers declare,
+size workspaces, and reject bad arguments before it touches a device.
+No call here reaches a kernel launch.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def mn():
+    from newton_schulz_ns_b200 import build
+    build.build()
+    import newton_schulz_ns_b200 as m
+    return m
+
+
+def _declared():
+    names = []
+    for h in ("muon_ns.h", "muon_ns_testing.h"):
+        text = open(os.path.join(ROOT, "include", h)).read()
+        names += re.findall(r"MUON_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    return names
+
+
+def test_library_exports_every_declared_symbol(mn):
+    from newton_schulz_ns_b200 import _capi
+    names = _declared()
+    assert set(names) >= {"muon_momentum_norm", "muon_ns_batched", "muon_gram_ns_batched", "normuon_update",
+                          "muon_workspace_size"}
+    lib = ctypes.CDLL(_capi.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert mn.version().count(".") == 2
+
+
+def test_status_strings(mn):
+    from newton_schulz_ns_b200 import _capi
+    for s in range(8):
+        assert _capi.status_string(s) and _capi.status_string(s) != "unknown status"
+
+
+def _fake_batch(mn, n, r, c, **kw):
+    from newton_schulz_ns_b200 import _capi
+    b = _capi.MuonBatch()
+    b.n, b.rows, b.cols = n, r, c
+    ld = kw.get("ld", c)
+    for i, f in enumerate(("grad", "momentum", "ns_in", "ns_out", "weight")):
+        v = getattr(b, f)
+        base = kw.get("ptr", 0x7F0000000000)
+        v.ptr = base + i * 0x10000000 if base else 0
+        v.ld = ld
+        v.batch_stride = kw.get("bs", r * ld)
+        v.dtype = kw.get(f + "_dt", _capi.MUON_BF16)
+    b.sumsq = 0x7F0000100000
+    b.variance = 0x7F0000200000
+    b.lr_scale = 1.0
+    return b
+
+
+def _call(mn, fn, batches, ws=None, nbytes=0, hp=None, **kw):
+    from newton_schulz_ns_b200 import _capi
+    arr = (_capi.MuonBatch * max(1, len(batches)))(*batches)
+    h, keep = (hp or mn.Hparams(**kw)).to_c()
+    lib = _capi.lib
+    if fn == "normuon_update":
+        return lib.normuon_update(arr, len(batches), ctypes.byref(h), 1, ws, nbytes, None)
+    return getattr(lib, fn)(arr, len(batches), ctypes.byref(h), ws, nbytes, None)
+
+
+def test_workspace_size_grows_with_batches(mn):
+    from newton_schulz_ns_b200 import _capi
+    b1 = _fake_batch(mn, 2, 64, 576)
+    b2 = _fake_batch(mn, 4, 1024, 512)
+    arr1 = (_capi.MuonBatch * 1)(b1)
+    arr2 = (_capi.MuonBatch * 2)(b1, b2)
+    for which in (0, 1, 2, 3):
+        s1 = _capi.lib.muon_workspace_size(arr1, 1, which)
+        s2 = _capi.lib.muon_workspace_size(arr2, 2, which)
+        assert s1 >= 256 and s2 > s1 and s1 % 256 == 0
+    # standard: two m x m bf16 buffers + one X-sized buffer per slice
+    ns = _capi.lib.muon_workspace_size(arr2, 2, 1)
+    assert ns >= 2 * (2 * 2 * 64 * 64 + 2 * 64 * 576) + 4 * (2 * 2 * 512 * 512 + 2 * 1024 * 512)
+    allmax = _capi.lib.muon_workspace_size(arr2, 2, -1)
+    assert allmax == max(_capi.lib.muon_workspace_size(arr2, 2, w) for w in range(4))
+    assert _capi.lib.muon_workspace_size(arr2, 2, 7) == 0
+
+
+@pytest.mark.parametrize("fn", ["muon_momentum_norm", "muon_ns_batched", "muon_gram_ns_batched", "normuon_update"])
+def test_rejects_bad_arguments_before_any_device_work(mn, fn):
+    good = _fake_batch(mn, 2, 64, 576)
+    # ld smaller than cols
+    assert _call(mn, fn, [_fake_batch(mn, 2, 64, 576, ld=500)], 0x7F0000300000, 1 << 30) == 2
+    # negative sizes
+    assert _call(mn, fn, [_fake_batch(mn, -1, 64, 576)], 0x7F0000300000, 1 << 30) == 2
+    # null data pointer
+    assert _call(mn, fn, [_fake_batch(mn, 2, 64, 576, ptr=0)], 0x7F0000300000, 1 << 30) == 1
+    # workspace: missing, misaligned, too small
+    assert _call(mn, fn, [good], None, 0) == 1
+    assert _call(mn, fn, [good], 0x7F0000300010, 1 << 30) == 4
+    assert _call(mn, fn, [good], 0x7F0000300000, 256) == 5
+    # ns_steps out of range and non-finite hyperparameters
+    assert _call(mn, fn, [good], 0x7F0000300000, 1 << 30, ns_steps=0) == 1
+    assert _call(mn, fn, [good], 0x7F0000300000, 1 << 30, lr=float("nan")) == 1
+
+
+def test_dtype_and_alignment_rules(mn):
+    from newton_schulz_ns_b200 import _capi
+    # Newton-Schulz operands must be bf16 and meet the 16-byte TMA rule.
+    assert _call(mn, "muon_ns_batched", [_fake_batch(mn, 2, 64, 576, ns_in_dt=_capi.MUON_F32)],
+                 0x7F0000300000, 1 << 30) == 3
+    assert _call(mn, "muon_ns_batched", [_fake_batch(mn, 2, 64, 570, ld=570)], 0x7F0000300000, 1 << 30) == 4
+    assert _call(mn, "muon_ns_batched", [_fake_batch(mn, 2, 64, 576, ptr=0x7F0000000008)],
+                 0x7F0000300000, 1 << 30) == 4
+    # the elementwise calls take f32 or bf16 and any 2-byte-aligned layout
+    b = _fake_batch(mn, 2, 64, 570, ld=570, grad_dt=_capi.MUON_F32, momentum_dt=_capi.MUON_F32)
+    st = _call(mn, "muon_momentum_norm", [b], 0x7F0000300000, 1 << 30)
+    assert st in (6, 7)      # passed validation; no device here (CUDA error) or not a B200
+
+
+def test_empty_batches_enqueue_nothing(mn):
+    for fn in ("muon_momentum_norm", "muon_ns_batched", "muon_gram_ns_batched", "normuon_update"):
+        assert _call(mn, fn, [_fake_batch(mn, 0, 64, 576)], None, 0) == 0
+        assert _call(mn, fn, [_fake_batch(mn, 3, 0, 576)], None, 0) == 0
+        assert _call(mn, fn, [], None, 0) == 0
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    import subprocess
+    import sys
+    code = ("import sys, importlib; sys.path.insert(0, %r); import newton_schulz_ns_b200._capi as c; "
+            "print('loaded')") % ROOT
+    env = dict(os.environ)
+    # Point the loader at a copy of the package without the shared object.
+    pkg = tmp_path / "newton_schulz_ns_b200"
+    pkg.mkdir()
+    src = os.path.join(ROOT, "newton_schulz_ns_b200")
+    for f in ("__init__.py", "_capi.py"):
+        (pkg / f).write_text(open(os.path.join(src, f)).read())
+    code = "import sys; sys.path.insert(0, %r); import newton_schulz_ns_b200" % str(tmp_path)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env)
+    assert r.returncode != 0 and "libmuon_ns.so is missing" in r.stderr

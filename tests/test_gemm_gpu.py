@@ -1,0 +1,156 @@
+"""The tcgen05 GEMM of the library against a float64 matrix product.
+
+Each case runs one GEMM problem through the C ABI's test hook on slices that
+span several 128x256 tiles with ragged tails, in every operand-major
+combination the Newton-Schulz calls use, and checks the epilogue terms
+(alpha, addend, identity, per-slice norm factor, row sums of squares).
+"""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def mn():
+    import newton_schulz_ns_b200 as m
+    return m
+
+
+def _ws():
+    return torch.zeros(256, dtype=torch.uint8, device=DEV)
+
+
+def _rnd(shape, dtype, seed, scale=1.0):
+    """Seeded N(0, scale^2) [S, R, C] on the device, rows padded to a multiple of 8 elements (TMA rule)."""
+    g = torch.Generator().manual_seed(seed)
+    S, R, C = shape
+    ld = (C + 7) // 8 * 8
+    x = torch.zeros((S, R, ld), dtype=dtype, device=DEV)
+    x[:, :, :C] = (torch.randn(shape, generator=g) * scale).to(dtype).to(DEV)
+    return x[:, :, :C]
+
+
+def _empty(shape, dtype, fill=float("nan")):
+    S, R, C = shape
+    ld = (C + 7) // 8 * 8
+    return torch.full((S, R, ld), fill, dtype=dtype, device=DEV)[:, :, :C]
+
+
+def _f64(t):
+    return t.detach().float().cpu().double().numpy()
+
+
+def _check(C, ref, rel_tol=4e-3):
+    C = _f64(C)
+    err = np.linalg.norm(C - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert err < rel_tol, f"relative error {err:.3e}"
+    assert np.max(np.abs(C - ref)) <= 2e-2 * np.max(np.abs(ref)) + 1e-6
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("M,N,K,S", [(300, 520, 200, 2), (128, 256, 64, 1), (77, 40, 33, 3), (513, 300, 520, 1)])
+def test_gemm_majors(mn, a_mn, b_mn, dtype, M, N, K, S):
+    A = _rnd((S, K, M) if a_mn else (S, M, K), dtype, 1)
+    B = _rnd((S, K, N) if b_mn else (S, N, K), dtype, 2)
+    C = _empty((S, M, N), torch.bfloat16)
+    ws = _ws()
+    mn.testing_gemm(A, bool(a_mn), B, bool(b_mn), C, K=K, alpha=0.5, workspace=ws)
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0
+    a = _f64(A)
+    b = _f64(B)
+    a = np.swapaxes(a, 1, 2) if a_mn else a                 # [S, M, K]
+    b = b if b_mn else np.swapaxes(b, 1, 2)                 # [S, K, N]
+    _check(C, 0.5 * a @ b)
+
+
+def test_gemm_strided_slices_and_padding(mn):
+    # Slices with ld > cols and batch stride > rows*ld; padding must stay untouched.
+    S, M, N, K = 3, 200, 260, 136
+    Abig = _rnd((S, M + 8, K + 24), torch.bfloat16, 3)
+    A = Abig[:, :M, :K]
+    Bbig = _rnd((S, K, N + 44), torch.bfloat16, 4)
+    B = Bbig[:, :, :N]
+    Cbig = torch.full((S, M + 5, N + 60), 7.0, dtype=torch.bfloat16, device=DEV)
+    C = Cbig[:, :M, :N]
+    ws = _ws()
+    mn.testing_gemm(A, False, B, True, C, K=K, workspace=ws)
+    torch.cuda.synchronize()
+    _check(C, _f64(A) @ _f64(B))
+    rest = _f64(Cbig)
+    rest[:, :M, :N] = 7.0
+    assert np.all(rest == 7.0)
+
+
+@pytest.mark.parametrize("mnmaj", [0, 1])
+@pytest.mark.parametrize("m,n", [(384, 500), (200, 1000), (64, 576), (513, 130)])
+def test_syrk_triangle_mirror(mn, mnmaj, m, n):
+    S = 2
+    X = _rnd((S, n, m) if mnmaj else (S, m, n), torch.bfloat16, 5)
+    C = _empty((S, m, m), torch.bfloat16)
+    ss = torch.tensor([4.0, 9.0], device=DEV)
+    ws = _ws()
+    mn.testing_gemm(X, bool(mnmaj), X, bool(mnmaj), C, K=n, tri=True, s_pow=2, sumsq=ss, eps=0.0, f0=3.0,
+                    workspace=ws)
+    torch.cuda.synchronize()
+    x = _f64(X)
+    x = np.swapaxes(x, 1, 2) if mnmaj else x
+    ref = x @ np.swapaxes(x, 1, 2) * 3.0 / np.array([4.0, 9.0])[:, None, None]
+    Cn = _f64(C)
+    assert np.array_equal(Cn, np.swapaxes(Cn, 1, 2))        # mirror is exact
+    _check(C, ref)
+
+
+def test_symmetric_epilogue_addend_identity_fp16(mn):
+    # P = a I + (b/k) A + (c/k^2) A A with fp16 A, as the Gram iteration forms it.
+    S, m = 2, 300
+    X = _rnd((S, m, 2 * m), torch.float32, 6)
+    A32 = X @ X.transpose(1, 2) / (2 * m)
+    A = _empty((S, m, m), torch.float16, 0.0)
+    A.copy_(A32.to(torch.float16))
+    P = _empty((S, m, m), torch.float16)
+    a, b, c, k = 3.4445, -4.7750, 2.0315, 4.0
+    ws = _ws()
+    mn.testing_gemm(A, False, A, False, P, K=m, tri=True, D=A, alpha=c / k ** 2, beta=b / k, gamma=a,
+                    workspace=ws)
+    torch.cuda.synchronize()
+    an = _f64(A)
+    ref = a * np.eye(m)[None] + (b / k) * an + (c / k ** 2) * an @ an
+    _check(P, ref, rel_tol=2e-3)
+
+
+def test_row_sums_of_squares(mn):
+    S, M, N, K = 2, 260, 600, 100
+    A = _rnd((S, M, K), torch.bfloat16, 7)
+    B = _rnd((S, K, N), torch.bfloat16, 8)
+    C = _empty((S, M, N), torch.bfloat16)
+    nt = (N + 255) // 256
+    rss = torch.full((S, nt, M), float("nan"), device=DEV)
+    ws = _ws()
+    mn.testing_gemm(A, False, B, True, C, K=K, row_ss=rss, workspace=ws)
+    torch.cuda.synchronize()
+    c = _f64(C)
+    for t in range(nt):
+        ref = np.sum(c[:, :, 256 * t:256 * (t + 1)] ** 2, axis=2)
+        assert np.allclose(_f64(rss)[:, t], ref, rtol=1e-5)
+
+
+def test_gemm_deterministic_and_batch_invariant(mn):
+    M, N, K = 384, 512, 640
+    A = _rnd((4, M, K), torch.bfloat16, 9)
+    B = _rnd((4, K, N), torch.bfloat16, 10)
+    ws = _ws()
+    C1 = torch.empty((4, M, N), dtype=torch.bfloat16, device=DEV)
+    C2 = torch.empty_like(C1)
+    mn.testing_gemm(A, False, B, True, C1, K=K, workspace=ws)
+    mn.testing_gemm(A, False, B, True, C2, K=K, workspace=ws)
+    C3 = torch.empty((1, M, N), dtype=torch.bfloat16, device=DEV)
+    mn.testing_gemm(A[2:3], False, B[2:3], True, C3, K=K, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(C1, C2)
+    assert torch.equal(C1[2:3], C3)

@@ -1,0 +1,336 @@
+"""Parity of the CUDA Muon / NorMuon step with the fp64 oracle.
+
+Bars (from the method's problem statement):
+* Newton-Schulz output: relative Frobenius error <= 3e-2 per slice against
+  the oracle on the same seeded inputs (bf16 tensor-core arithmetic);
+* momentum, NorMuon and update stages fed the same Newton-Schulz output:
+  <= 1e-5 relative on fp32 results (momentum, variance, weight update
+  delta), and at most one bf16 ulp per element with >= 99.99% exact on
+  bf16-stored results (momentum, weights, weight copy).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+NS_TOL = 3e-2
+
+
+@pytest.fixture(scope="module")
+def mn():
+    import newton_schulz_ns_b200 as m
+    return m
+
+
+def f64(t):
+    return t.detach().float().cpu().double().numpy()
+
+
+def rel(a, b):
+    nb = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / nb) if nb > 0 else float(np.linalg.norm(a))
+
+
+def _aligned(n, r, c, dtype, fill=0.0):
+    ld = (c + 7) // 8 * 8
+    return torch.full((n, r, ld), fill, dtype=dtype, device=DEV)[:, :, :c]
+
+
+def _seeded(n, r, c, seed, dtype, std=1.0):
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn((n, r, c), generator=g) * std).to(dtype)
+    t = _aligned(n, r, c, dtype)
+    t.copy_(x.to(DEV))
+    return t
+
+
+def _ns_batch(mn, U):
+    n, r, c = U.shape
+    out = _aligned(n, r, c, torch.bfloat16, float("nan"))
+    return mn.Batch(n, r, c, ns_in=U, ns_out=out)
+
+
+def _run_ns(mn, batches, variant, hp):
+    ws = mn.allocate_workspace(batches, 1 if variant == "standard" else 2)
+    fn = mn.muon_ns_batched if variant == "standard" else mn.muon_gram_ns_batched
+    fn(batches, hp, ws)
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0
+    return ws
+
+
+def _oracle_ns(U, variant, steps=5, abc=oracle.QUINTIC_ABC):
+    return oracle.ns_batched(f64(U), variant, steps=steps, abc=abc)
+
+
+# ----------------------------------------------------------------- Newton-Schulz
+
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+@pytest.mark.parametrize("shape", workloads.small_shapes())
+def test_ns_matches_oracle_small_shapes(mn, variant, shape):
+    r, c = shape
+    U = _seeded(3, r, c, 100 + r + c, torch.bfloat16)
+    b = _ns_batch(mn, U)
+    _run_ns(mn, [b], variant, mn.Hparams())
+    ref = _oracle_ns(U, variant)
+    got = f64(b.ns_out)
+    for i in range(3):
+        assert rel(got[i], ref[i]) < NS_TOL, (variant, shape, i, rel(got[i], ref[i]))
+
+
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+@pytest.mark.parametrize("steps", [1, 2, 3])
+def test_ns_step_counts(mn, variant, steps):
+    U = _seeded(2, 130, 300, 7, torch.bfloat16)
+    b = _ns_batch(mn, U)
+    _run_ns(mn, [b], variant, mn.Hparams(ns_steps=steps))
+    ref = _oracle_ns(U, variant, steps=steps)
+    got = f64(b.ns_out)
+    for i in range(2):
+        assert rel(got[i], ref[i]) < NS_TOL
+
+
+def test_ns_coefficient_schedule(mn):
+    sched = [(3.4445, -4.7750, 2.0315), (3.0, -3.2, 1.2), (2.5, -2.0, 0.5)]
+    U = _seeded(2, 96, 200, 8, torch.bfloat16)
+    b = _ns_batch(mn, U)
+    _run_ns(mn, [b], "standard", mn.Hparams(ns_steps=3, abc_schedule=sched))
+    X = f64(U)
+    for i in range(2):
+        x = oracle.frobenius_normalize(X[i], 1e-7)
+        for (a, bb, cc) in sched:
+            A = x @ x.T
+            x = a * x + (bb * A + cc * A @ A) @ x
+        assert rel(f64(b.ns_out)[i], x) < NS_TOL
+
+
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+def test_ns_mixed_batches_one_call(mn, variant):
+    shapes = [(64, 576, 4), (300, 200, 2), (256, 256, 1), (128, 1000, 3)]
+    bs, Us = [], []
+    for k, (r, c, n) in enumerate(shapes):
+        U = _seeded(n, r, c, 300 + k, torch.bfloat16)
+        Us.append(U)
+        bs.append(_ns_batch(mn, U))
+    _run_ns(mn, bs, variant, mn.Hparams())
+    for U, b in zip(Us, bs):
+        ref = _oracle_ns(U, variant)
+        got = f64(b.ns_out)
+        for i in range(U.shape[0]):
+            assert rel(got[i], ref[i]) < NS_TOL
+
+
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+def test_ns_batch_invariance_and_determinism(mn, variant):
+    U = _seeded(5, 200, 330, 11, torch.bfloat16)
+    b = _ns_batch(mn, U)
+    _run_ns(mn, [b], variant, mn.Hparams())
+    first = b.ns_out.clone()
+    _run_ns(mn, [b], variant, mn.Hparams())
+    assert torch.equal(first, b.ns_out)                      # run to run
+    one = _ns_batch(mn, U[3:4])
+    _run_ns(mn, [one], variant, mn.Hparams())
+    assert torch.equal(one.ns_out[0], first[3])              # N = 1 vs N = 5
+    rev = _aligned(5, 200, 330, torch.bfloat16)
+    rev.copy_(U.flip(0))
+    br = _ns_batch(mn, rev)
+    _run_ns(mn, [br], variant, mn.Hparams())
+    assert torch.equal(br.ns_out.flip(0), first)             # reversed batch order
+
+
+def test_ns_zero_and_rank_deficient(mn):
+    Z = _aligned(2, 64, 128, torch.bfloat16)
+    b = _ns_batch(mn, Z)
+    for variant in ("standard", "gram"):
+        _run_ns(mn, [b], variant, mn.Hparams())
+        assert torch.all(b.ns_out == 0)
+    g = torch.Generator().manual_seed(12)
+    low = (torch.randn(2, 100, 3, generator=g) @ torch.randn(2, 3, 160, generator=g)).to(torch.bfloat16)
+    L = _aligned(2, 100, 160, torch.bfloat16)
+    L.copy_(low.to(DEV))
+    b = _ns_batch(mn, L)
+    for variant in ("standard", "gram"):
+        _run_ns(mn, [b], variant, mn.Hparams())
+        ref = _oracle_ns(L, variant)
+        for i in range(2):
+            assert rel(f64(b.ns_out)[i], ref[i]) < NS_TOL
+
+
+def test_ns_zero_padding_invariance(mn):
+    # Zero columns appended to a slice leave the real columns' result unchanged
+    # (up to the kernel's own rounding: it is a different problem shape).
+    U = _seeded(2, 96, 300, 13, torch.bfloat16)
+    P = _aligned(2, 96, 360, torch.bfloat16)
+    P[:, :, :300].copy_(U)
+    b1, b2 = _ns_batch(mn, U), _ns_batch(mn, P)
+    _run_ns(mn, [b1, b2], "standard", mn.Hparams())
+    assert torch.all(b2.ns_out[:, :, 300:] == 0)
+    assert rel(f64(b2.ns_out[:, :, :300]), f64(b1.ns_out)) < 1e-2
+
+
+def test_per_head_view_equals_head_blocks(mn):
+    # Per-head NS of a [H*d, c] projection through a strided view equals NS of
+    # each head block as its own slice, bit for bit.
+    H, d, c = 8, 64, 384
+    W = _seeded(1, H * d, c, 14, torch.bfloat16)[0]
+    heads = W.view(H, d, c) if W.is_contiguous() else W.reshape(H, d, c)
+    bh = _ns_batch(mn, heads)
+    _run_ns(mn, [bh], "standard", mn.Hparams())
+    shard = _ns_batch(mn, heads[2:6])
+    _run_ns(mn, [shard], "standard", mn.Hparams())
+    assert torch.equal(shard.ns_out, bh.ns_out[2:6])
+    ref = oracle.per_head_ns(f64(W), H)
+    assert rel(f64(bh.ns_out).reshape(H * d, c), ref) < NS_TOL
+
+
+# ----------------------------------------------------------------- momentum
+
+@pytest.mark.parametrize("gdt,mdt", [(torch.float32, torch.float32), (torch.bfloat16, torch.bfloat16),
+                                     (torch.bfloat16, torch.float32)])
+@pytest.mark.parametrize("shape", [(3, 64, 576), (2, 37, 51), (1, 300, 200)])
+@pytest.mark.parametrize("nesterov", [True, False])
+def test_momentum_norm(mn, gdt, mdt, shape, nesterov):
+    n, r, c = shape
+    G = _seeded(n, r, c, 20, gdt)
+    M = _seeded(n, r, c, 21, mdt, std=0.5)
+    M0 = M.clone()
+    U = _aligned(n, r, c, torch.bfloat16, float("nan"))
+    ss = torch.full((n,), float("nan"), device=DEV)
+    b = mn.Batch(n, r, c, grad=G, momentum=M, ns_in=U, sumsq=ss)
+    ws = mn.allocate_workspace([b], 0)
+    mn.muon_momentum_norm([b], mn.Hparams(mu=0.95, nesterov=nesterov), ws)
+    torch.cuda.synchronize()
+    store = "bf16" if mdt == torch.bfloat16 else "f32"
+    Mref, Uref = oracle.momentum_nesterov(f64(G), f64(M0), 0.95, nesterov, store)
+    Mg, Ug = f64(M), f64(U)
+    if mdt == torch.float32:
+        assert rel(Mg, Mref) < 1e-6
+    else:
+        _bf16_close(Mg, Mref)
+    _bf16_close(Ug, oracle.bf16_round(Uref))
+    # sum of squares of the stored bf16 U, per slice
+    for i in range(n):
+        assert abs(float(ss[i]) / np.sum(Ug[i] ** 2) - 1) < 1e-5
+
+
+def _bf16_close(got, want):
+    """<= 1 bf16 ulp everywhere and >= 99.99% identical."""
+    ulp = np.abs(oracle.bf16_round(np.abs(want) * (1 + 2.0 ** -7)) - oracle.bf16_round(np.abs(want)))
+    ulp = np.maximum(ulp, 1e-38)
+    diff = np.abs(got - want)
+    assert np.all(diff <= ulp * 1.0001), float(np.max(diff / ulp))
+    assert np.mean(diff == 0) >= 0.9999, float(np.mean(diff == 0))
+
+
+# ----------------------------------------------------------------- NorMuon + update
+
+@pytest.mark.parametrize("wdt,copy", [(torch.float32, True), (torch.bfloat16, False), (torch.float32, False)])
+@pytest.mark.parametrize("normuon", [True, False])
+@pytest.mark.parametrize("shape", [(4, 64, 576), (2, 300, 200), (1, 33, 45)])
+def test_update_fed_same_ns_output(mn, wdt, copy, normuon, shape):
+    n, r, c = shape
+    O = _seeded(n, r, c, 30, torch.bfloat16, std=1 / math.sqrt(c)) * torch.linspace(0.2, 3, r, device=DEV)[None, :, None]
+    O = O.to(torch.bfloat16)
+    Ob = _aligned(n, r, c, torch.bfloat16)
+    Ob.copy_(O)
+    W = _seeded(n, r, c, 31, wdt, std=0.02)
+    W0 = W.clone()
+    Wc = _aligned(n, r, c, torch.bfloat16, float("nan")) if copy else None
+    V = torch.rand((n, r), generator=torch.Generator().manual_seed(32)).mul(1e-3).to(DEV)
+    V0 = V.clone()
+    scale = mn.spectral_scale(r, c)
+    b = mn.Batch(n, r, c, ns_out=Ob, weight=W, weight_copy=Wc, variance=V if normuon else None, lr_scale=scale)
+    hp = mn.Hparams(lr=0.02, weight_decay=0.01)
+    ws = mn.allocate_workspace([b], 3)
+    mn.normuon_update([b], hp, normuon, ws)
+    torch.cuda.synchronize()
+    ref = oracle.muon_step_slices(np.zeros((n, r, c)), np.zeros((n, r, c)), f64(W0), f64(V0), normuon=normuon,
+                                  lr=0.02, weight_decay=0.01, lr_scale=scale, O_override=f64(Ob))
+    if normuon:
+        assert rel(f64(V), ref["v"]) < 1e-5
+    if wdt == torch.float32:
+        dW = f64(W) - f64(W0)
+        assert rel(dW, ref["W"] - f64(W0)) < 1e-5
+        if copy:
+            _bf16_close(f64(Wc), oracle.bf16_round(oracle.fp32_round(ref["W"])))
+    else:
+        _bf16_close(f64(W), oracle.bf16_round(ref["W"]))
+
+
+# ----------------------------------------------------------------- whole step
+
+def _workload_batches(mn, w, step_states=None):
+    """Device buffers for every group of a workload (one Batch per group)."""
+    out = []
+    for g in w.groups:
+        n, r, c = g.slices, g.slice_rows, g.cols
+        G = torch.stack([workloads.gradient(w, g, i, 0).reshape(g.rows, g.cols) for i in range(g.count)])
+        G = G.reshape(n, r, c)
+        W = torch.stack([workloads.initial_weight(w, g, i).reshape(g.rows, g.cols) for i in range(g.count)])
+        W = W.reshape(n, r, c)
+        d = dict(grad=_aligned(n, r, c, w.grad_dtype), momentum=_aligned(n, r, c, w.mom_dtype),
+                 weight=_aligned(n, r, c, w.weight_dtype),
+                 ns_in=_aligned(n, r, c, torch.bfloat16), ns_out=_aligned(n, r, c, torch.bfloat16),
+                 sumsq=torch.zeros(n, device=DEV),
+                 variance=torch.zeros(n * r, device=DEV) if w.normuon else None,
+                 weight_copy=_aligned(n, r, c, torch.bfloat16) if w.weight_copy_bf16 else None)
+        d["grad"].copy_(G.to(DEV))
+        d["weight"].copy_(W.to(DEV))
+        out.append((g, mn.Batch(n, r, c, lr_scale=mn.spectral_scale(g.rows, g.cols), **d)))
+    return out
+
+
+@pytest.mark.parametrize("key", ["single_256", "conv_megabatch", "per_head"])
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+def test_full_step_matches_oracle(mn, key, variant):
+    w = workloads.WORKLOADS[key]
+    gb = _workload_batches(mn, w)
+    batches = [b for _, b in gb]
+    hp = mn.Hparams(mu=w.momentum, nesterov=w.nesterov, ns_eps=w.ns_eps, ns_steps=w.ns_steps, beta2=w.beta2,
+                    nor_eps=w.nor_eps, lr=w.lr, weight_decay=w.weight_decay)
+    ws = mn.allocate_workspace(batches, -1)
+    states = [dict(M=np.zeros((b.n, b.rows, b.cols)), W=f64(b.weight),
+                   v=np.zeros((b.n, b.rows)) if w.normuon else None) for b in batches]
+    ns_fn = mn.muon_ns_batched if variant == "standard" else mn.muon_gram_ns_batched
+    for step in range(w.steps):
+        if step > 0:
+            for (g, b) in gb:
+                G = torch.stack([workloads.gradient(w, g, i, step).reshape(g.rows, g.cols) for i in range(g.count)])
+                b.grad.copy_(G.reshape(b.n, b.rows, b.cols).to(DEV))
+        Gs = [f64(b.grad) for b in batches]
+        mn.muon_momentum_norm(batches, hp, ws)
+        ns_fn(batches, hp, ws)
+        W_before = [f64(b.weight) for b in batches]
+        mn.normuon_update(batches, hp, w.normuon, ws)
+        torch.cuda.synchronize()
+        assert mn.workspace_error(ws) == 0
+        mstore = "bf16" if w.mom_dtype == torch.bfloat16 else "f32"
+        wstore = "bf16" if w.weight_dtype == torch.bfloat16 else "f32"
+        for k, b in enumerate(batches):
+            st = states[k]
+            ref = oracle.muon_step_slices(Gs[k], st["M"], st["W"], st["v"], mu=w.momentum, nesterov=w.nesterov,
+                                          variant=variant, normuon=w.normuon, beta2=w.beta2, nor_eps=w.nor_eps,
+                                          lr=w.lr, weight_decay=w.weight_decay, lr_scale=b.lr_scale,
+                                          mom_store=mstore, w_store=wstore)
+            O = f64(b.ns_out)
+            for i in range(b.n):
+                assert rel(O[i], ref["O"][i]) < NS_TOL, (key, variant, step, k, i, rel(O[i], ref["O"][i]))
+            # downstream stages on the device's own Newton-Schulz output
+            ref2 = oracle.muon_step_slices(Gs[k], st["M"], W_before[k], st["v"], mu=w.momentum,
+                                           nesterov=w.nesterov, normuon=w.normuon, beta2=w.beta2,
+                                           nor_eps=w.nor_eps, lr=w.lr, weight_decay=w.weight_decay,
+                                           lr_scale=b.lr_scale, mom_store=mstore, w_store="f64", O_override=O)
+            if w.normuon:
+                assert rel(f64(b.variance).reshape(b.n, b.rows), ref2["v"]) < 1e-5
+            if wstore == "f32":
+                assert rel(f64(b.weight) - W_before[k], ref2["W"] - W_before[k]) < 1e-5
+            # carry the device's state forward (the oracle's own trajectory is checked per step above)
+            st["M"] = f64(b.momentum)
+            st["W"] = f64(b.weight)
+            st["v"] = f64(b.variance).reshape(b.n, b.rows) if w.normuon else None
