@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Throughput of the B200 Muon / NorMuon optimizer step.
+
+One step = momentum + Nesterov + Frobenius norm (muon_momentum_norm), quintic
+Newton-Schulz of every slice (muon_ns_batched or muon_gram_ns_batched) and
+NorMuon + weight update (normuon_update), over every matrix of the workload,
+with all inputs resident in HBM.  Prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b]
+                    [--variant standard|gram] [--impl ours|reference]
+
+Metric: Newton-Schulz TFLOP/s of the whole step (the algorithmic flops of
+the variant run -- one-triangle symmetric products -- divided by the step
+time), with its fraction of the measured bf16 dense tensor-core peak and the
+matrices (Newton-Schulz slices) per second.  Multi-GPU runs are independent
+replicas (the step has no exchange): value = all ranks' work / max time.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Muon step NS TFLOP/s & % bf16 TC peak; matrices/s at 1 B200 vs CPU oracle"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+DESCRIPTIONS = {
+    "llama8b": "Llama-8B-shaped Muon step, 32 layers: q,o 4096x4096, k,v 1024x4096, gate,up 14336x4096, "
+               "down 4096x14336 (224 matrices); bf16 G and M, fp32 master W + bf16 copy; NorMuon; lr 0.02",
+    "moe": "MoE megabatch: 64 experts x (w1 2048x7168, w2 7168x2048) bf16; per-expert grad scale "
+           "log-uniform [1e-2,1]; NorMuon; lr 0.02",
+    "per_head": "q_proj 4096x4096 as 32 heads [32,128,4096] + 512x1024 + 1024x512, bf16, plain Muon",
+    "conv_megabatch": "16 stacked Conv2d [16,64,64,3,3] -> [16,64,576] bf16, NorMuon, lr 0.02, wd 0.01",
+    "single_256": "one 256x256 fp32 gradient, Muon, lr 0.05",
+}
+
+# Oracle sample per workload for the CPU baseline: (group index, parameters of it).
+CPU_SAMPLE = {
+    "llama8b": [(0, 1), (1, 1), (2, 1)],          # layer 0 q_proj, k_proj, v_proj
+    "moe": [(0, 1), (1, 1)],                      # expert 0 w1 and w2
+    "per_head": [(0, 1), (1, 1), (2, 1)],         # all of it
+    "conv_megabatch": [(0, 16)],
+    "single_256": [(0, 1)],
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama8b", choices=sorted(DESCRIPTIONS))
+    ap.add_argument("--variant", choices=["standard", "gram"], default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--scale-down", type=int, default=1, help="divide every parameter count (smoke runs only)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def ns_flops(rows, cols, variant, steps):
+    """Work of one slice's orthogonalization, as the metric counts it (m = short side, n = long side).
+
+    Standard, one triangle of each symmetric product: per step m^2 n (X X^T)
+    + m^3 (b*A + c*A^2) + 2 m^2 n (B X).  Gram: m^2 n for X X^T, 2 m^2 n for
+    the final Q X, and per step one-triangle m^3 products: A^2, P Q (from the
+    second step), and the two factors of P A P (up to the second-to-last).
+    Both arms of the benchmark count the same work for the same variant.
+    """
+    m, n = min(rows, cols), max(rows, cols)
+    if variant == "standard":
+        return float(steps * (3 * m * m * n + m ** 3))
+    prods = sum(1 + (k > 0) + 2 * (k < steps - 1) for k in range(steps))
+    return float(3 * m * m * n + prods * m ** 3)
+
+
+def default_variant(wl):
+    return "gram" if wl.key == "moe" else "standard"
+
+
+# ----------------------------------------------------------------------------- CPU oracle (baseline)
+
+def oracle_sample(wl, variant, budget_s=30.0):
+    """Runs the fp64 oracle's full step on the workload's sample; returns (flops, slices, seconds, cores, desc)."""
+    import numpy as np
+    import threadpoolctl
+    import oracle
+    import workloads
+
+    ncores = os.cpu_count() or 1
+    with threadpoolctl.threadpool_limits(limits=ncores):
+        info = threadpoolctl.threadpool_info()
+        cores = max([i.get("num_threads", 1) for i in info] or [1])
+        flops = 0.0
+        slices = 0
+        parts = []
+        t0 = time.perf_counter()
+        for gi, count in CPU_SAMPLE[wl.key]:
+            g = wl.groups[gi]
+            for p in range(count):
+                G = workloads.gradient(wl, g, p, 0).float().double().numpy().reshape(g.slices // g.count,
+                                                                                     g.slice_rows, g.cols)
+                W = workloads.initial_weight(wl, g, p).float().double().numpy().reshape(G.shape)
+                M = np.zeros_like(G)
+                v = np.zeros(G.shape[:2]) if wl.normuon else None
+                oracle.muon_step_slices(G, M, W, v, mu=wl.momentum, nesterov=wl.nesterov, ns_eps=wl.ns_eps,
+                                        ns_steps=wl.ns_steps, variant=variant, normuon=wl.normuon,
+                                        beta2=wl.beta2, nor_eps=wl.nor_eps, lr=wl.lr,
+                                        weight_decay=wl.weight_decay,
+                                        lr_scale=math.sqrt(max(1.0, g.rows / g.cols)))
+                flops += G.shape[0] * ns_flops(g.slice_rows, g.cols, variant, wl.ns_steps)
+                slices += G.shape[0]
+            parts.append(f"{g.name} x{count}")
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+    desc = (f"oracle (numpy fp64, full step incl. momentum/NorMuon/update) on {', '.join(parts)} of "
+            f"{wl.key}; {slices} slices")
+    return flops, slices, dt, cores, desc
+
+
+# ----------------------------------------------------------------------------- GPU state
+
+def build_state(wl, variant, dev):
+    import torch
+    import newton_schulz_ns_b200 as mn
+    import workloads
+
+    groups = []
+    for g in wl.groups:
+        n, r, c = g.slices, g.slice_rows, g.cols
+        G = torch.empty((g.count, g.rows, g.cols), dtype=wl.grad_dtype, device=dev)
+        W = torch.empty((g.count, g.rows, g.cols), dtype=wl.weight_dtype, device=dev)
+        for i in range(g.count):
+            G[i].copy_(workloads.gradient(wl, g, i, 0, device=dev).reshape(g.rows, g.cols))
+            W[i].copy_(workloads.initial_weight(wl, g, i, device=dev).reshape(g.rows, g.cols))
+        b = mn.Batch(n, r, c,
+                     grad=G.view(n, r, c), momentum=torch.zeros((n, r, c), dtype=wl.mom_dtype, device=dev),
+                     ns_in=torch.empty((n, r, c), dtype=torch.bfloat16, device=dev),
+                     ns_out=torch.empty((n, r, c), dtype=torch.bfloat16, device=dev),
+                     weight=W.view(n, r, c),
+                     weight_copy=torch.empty((n, r, c), dtype=torch.bfloat16, device=dev)
+                     if wl.weight_copy_bf16 else None,
+                     sumsq=torch.zeros(n, dtype=torch.float32, device=dev),
+                     variance=torch.zeros(n * r, dtype=torch.float32, device=dev) if wl.normuon else None,
+                     lr_scale=mn.spectral_scale(g.rows, g.cols))
+        groups.append(b)
+    hp = mn.Hparams(mu=wl.momentum, nesterov=wl.nesterov, ns_eps=wl.ns_eps, ns_steps=wl.ns_steps,
+                    beta2=wl.beta2, nor_eps=wl.nor_eps, lr=wl.lr, weight_decay=wl.weight_decay)
+    ws = mn.allocate_workspace(groups, -1, dev)
+    return groups, hp, ws
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(gpu_id)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power = [], [], []
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, wl, variant, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import newton_schulz_ns_b200 as mn
+
+    dev = f"cuda:{local_rank}"
+    torch.cuda.set_device(dev)
+    groups, hp, ws = build_state(wl, variant, dev)
+    ns_fn = mn.muon_ns_batched if variant == "standard" else mn.muon_gram_ns_batched
+    stream = torch.cuda.current_stream()
+
+    ns_flop = sum(b.n * ns_flops(b.rows, b.cols, variant, wl.ns_steps) for b in groups)
+    slices = sum(b.n for b in groups)
+
+    def step(ev=None):
+        mn.muon_momentum_norm(groups, hp, ws, stream)
+        if ev is not None:
+            ev[0].record(stream)
+        ns_fn(groups, hp, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        mn.normuon_update(groups, hp, wl.normuon, ws, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0, "device-side wait timed out"
+
+    # ---- device-resident timing
+    gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[local_rank] \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else str(local_rank)
+    ns_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks = Clocks(gpu_id)
+    launches0 = mn.kernel_launches()
+    start.record(stream)
+    for k in range(args.steps):
+        step(ns_events[k])
+    end.record(stream)
+    torch.cuda.synchronize()
+    launches = mn.kernel_launches() - launches0
+    clk = clocks.stop()
+    barrier()
+    ms_total = start.elapsed_time(end)
+    ns_ms = [a.elapsed_time(b) for a, b in ns_events]
+    assert mn.workspace_error(ws) == 0, "device-side wait timed out"
+
+    # ---- end to end: gradients H2D from pinned host memory, step, result D2H
+    e2e = None
+    need = sum(b.grad.numel() * b.grad.element_size() for b in groups)
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:  # noqa: BLE001
+        avail = 0
+    e2e_skip = None if avail > 4 * need * max(1, world) else f"host memory {avail/1e9:.0f} GB too small for pinned gradients"
+    if not args.no_e2e and e2e_skip is None:
+        host_g = [torch.empty(b.grad.shape, dtype=b.grad.dtype, pin_memory=True) for b in groups]
+        for h, b in zip(host_g, groups):
+            h.copy_(b.grad)
+        host_out = [torch.empty(b.n, dtype=torch.float32, pin_memory=True) for b in groups]
+        h2d = sum(t.numel() * t.element_size() for t in host_g)
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+        for k in range(2):
+            for b, h in zip(groups, host_g):
+                b.grad.copy_(h, non_blocking=True)
+            step()
+            for b, h in zip(groups, host_out):
+                h.copy_(b.sumsq, non_blocking=True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for k in range(args.steps):
+            for b, h in zip(groups, host_g):
+                b.grad.copy_(h, non_blocking=True)
+            step()
+            for b, h in zip(groups, host_out):
+                h.copy_(b.sumsq, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
+
+    # ---- max over ranks
+    vals = torch.tensor([ms_total, statistics.mean(ns_ms), e2e["ms"] if e2e else 0.0], device=dev,
+                        dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms_total, ns_mean, e2e_ms = (float(x) for x in vals.tolist())
+    if rank != 0:
+        return None
+
+    peaks, src = load_peaks()
+    sec = ms_total / 1e3
+    value = world * ns_flop * args.steps / sec / 1e12
+    ms_step = ms_total / args.steps
+    achieved = ns_flop / (ns_mean / 1e3) / 1e12          # per NS call, averaged over the timed steps
+    peak_s = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_b = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch Philox on the device)",
+        "config": {"workload": DESCRIPTIONS[wl.key], "key": wl.key, "variant": variant, "slices": slices,
+                   "ns_flop_per_step": ns_flop, "l2": "inputs larger than L2 (126 MB), no flush",
+                   "parallelism": f"replicas x{world} (no exchange)"},
+        "pct_bf16_peak": round(100 * value / world / peak_s, 2),
+        "pct_bf16_peak_burst": round(100 * value / world / peak_b, 2),
+        "matrices_per_s": round(world * slices * args.steps / sec, 2),
+        "ms_breakdown": {"ns": round(ns_mean, 3), "momentum_and_update": round(ms_step - ns_mean, 3)},
+        "roofline": {"bound": "tensor", "kernel": "ns_gemm_kernel (all launches of one Newton-Schulz call)",
+                     "achieved": round(achieved, 2), "peak": peak_s, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_s, 4), "frac_of_burst": round(achieved / peak_b, 4),
+                     "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a long step)",
+                     "traffic": None},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if e2e_skip:
+        out["e2e"] = {"value": None, "unit": "TFLOP/s", "skipped": e2e_skip}
+    if e2e:
+        out["e2e"] = {"value": round(world * ns_flop * args.steps / (e2e_ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
+                      "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                      "ms_per_step": round(e2e_ms / args.steps, 3),
+                      "path": "public C-ABI calls; gradients copied H2D from pinned host memory and the per-slice "
+                              "norms read back D2H inside the timed region"}
+    if world == 1 and not args.no_cpu_baseline:
+        flops, sl, dt, cores, desc = oracle_sample(wl, variant)
+        out["cpu_baseline"] = {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+                               "kind": "oracle", "sample": desc, "seconds": round(dt, 2),
+                               "matrices_per_s": round(sl / dt, 4)}
+    return out
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, wl, variant):
+    peaks, _ = load_peaks()
+    budget = max(5.0, 60.0 / max(1, args.steps + args.warmup))
+    per_step = []
+    flops = sl = 0
+    cores, desc = 1, ""
+    for k in range(args.warmup + args.steps):
+        f, s, dt, cores, desc = oracle_sample(wl, variant, budget)
+        if k >= args.warmup:
+            per_step.append(dt)
+            flops, sl = f, s
+    sec = sum(per_step)
+    value = flops * args.steps / sec / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sec / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": DESCRIPTIONS[wl.key], "key": wl.key, "variant": variant,
+                   "sample": desc},
+        "pct_bf16_peak": round(100 * value / peaks.get("bf16_tflops_sustained", 1400.0), 6),
+        "matrices_per_s": round(sl * args.steps / sec, 4),
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    import workloads
+    wl = workloads.WORKLOADS[args.workload]
+    if args.scale_down > 1:
+        wl = workloads.scaled(wl, args.scale_down)
+    variant = args.variant or default_variant(wl)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, wl, variant)), flush=True)
+        return 0
+
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(f"cuda:{local_rank}"))
+    try:
+        out = run_ours(args, wl, variant, rank, world, local_rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -192,6 +192,11 @@ MUON_API muon_status muon_workspace_error(const void* workspace, cudaStream_t st
 
 MUON_API const char* muon_status_string(muon_status status);
 
+/* Kernels this library has enqueued in this process so far (all devices,
+ * all threads).  Instrumentation only: lets a caller count the launches of a
+ * region without a profiler. */
+MUON_API uint64_t muon_kernel_launches(void);
+
 /* Library version, "major.minor.patch". */
 MUON_API const char* muon_version(void);
 

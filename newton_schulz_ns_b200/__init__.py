@@ -20,7 +20,7 @@ from ._capi import MUON_BF16, MUON_F16, MUON_F32, MuonError  # noqa: F401
 
 __all__ = ["Batch", "Hparams", "muon_workspace_size", "muon_momentum_norm", "muon_ns_batched",
            "muon_gram_ns_batched", "normuon_update", "workspace_error", "testing_gemm", "spectral_scale",
-           "ns_flops", "version", "MuonError", "LIB_PATH"]
+           "ns_flops", "version", "kernel_launches", "allocate_workspace", "MuonError", "LIB_PATH"]
 
 LIB_PATH = _capi.LIB_PATH
 
@@ -31,6 +31,11 @@ QUINTIC = (3.4445, -4.7750, 2.0315)
 
 def version() -> str:
     return _capi.lib.muon_version().decode()
+
+
+def kernel_launches() -> int:
+    """Kernels the library has enqueued in this process so far."""
+    return int(_capi.lib.muon_kernel_launches())
 
 
 def spectral_scale(fan_out: int, fan_in: int, extra: float = 1.0) -> float:

@@ -49,13 +49,13 @@ class MuonHparams(ctypes.Structure):
 
 EXPORTS = ("muon_workspace_size", "muon_momentum_norm", "muon_ns_batched", "muon_gram_ns_batched",
            "normuon_update", "muon_workspace_error", "muon_status_string", "muon_version",
-           "muon_testing_gemm")
+           "muon_testing_gemm", "muon_kernel_launches")
 
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m newton_schulz_ns_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python newton_schulz_ns_b200/build.py` "
             "(the Muon step has no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     for name in EXPORTS:
@@ -75,6 +75,8 @@ def _load() -> ctypes.CDLL:
     lib.muon_workspace_error.restype = ctypes.c_int
     lib.muon_status_string.argtypes = [ctypes.c_int]
     lib.muon_status_string.restype = ctypes.c_char_p
+    lib.muon_kernel_launches.argtypes = []
+    lib.muon_kernel_launches.restype = ctypes.c_uint64
     lib.muon_version.argtypes = []
     lib.muon_version.restype = ctypes.c_char_p
     i64, i32, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_float

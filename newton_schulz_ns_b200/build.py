@@ -1,6 +1,7 @@
 """Builds libmuon_ns.so in-tree for sm_100a with nvcc.
 
-Usage: ``python -m newton_schulz_ns_b200.build [--verbose] [--ptxas-info]``.
+Usage: ``python newton_schulz_ns_b200/build.py [--verbose] [--ptxas-info] [--force]``.
+Run it by path: importing the package loads the library this script builds.
 The library links the CUDA runtime statically and resolves the driver's
 tensor-map encoder at run time, so it loads on a machine without a GPU
 driver (symbol checks) and runs on a B200.

@@ -10,6 +10,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -44,6 +45,14 @@ struct DeviceInfo {
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::atomic<unsigned long long> g_launches{0};
+
+// Checks the launch just enqueued and counts it.
+inline bool launched() {
+  if (cudaGetLastError() != cudaSuccess) return false;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return true;
+}
 
 muon_status device_setup(int* sms_out) {
   int dev = 0;
@@ -315,7 +324,7 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
     P.total_tiles = tiles;
     const int grid = std::min(tiles, sms);
     ns_gemm_kernel<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(P);
-    if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+    if (!launched()) return MUON_CUDA_ERROR;
   }
   return MUON_OK;
 }
@@ -383,9 +392,9 @@ muon_status launch_norm(const muon_batch* bs, int nb, const muon_hparams* hp, in
       momentum_chunks_kernel<0><<<ew_grid(chunk, sms), EW_THREADS, 0, stream>>>(P);
     else
       momentum_chunks_kernel<1><<<ew_grid(chunk, sms), EW_THREADS, 0, stream>>>(P);
-    if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+    if (!launched()) return MUON_CUDA_ERROR;
     sumsq_finalize_kernel<<<ew_grid(cdiv(slice, EW_THREADS / 32), sms), EW_THREADS, 0, stream>>>(P);
-    if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+    if (!launched()) return MUON_CUDA_ERROR;
     partials += chunk;
     sumsq_ws_dev += slice;
   }
@@ -561,6 +570,8 @@ muon_status prepare_norms(const muon_batch* bs, int nb, const Layout& L, uint8_t
 extern "C" {
 
 const char* muon_version(void) { return "0.1.0"; }
+
+uint64_t muon_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* muon_status_string(muon_status s) {
   switch (s) {
@@ -821,12 +832,12 @@ muon_status normuon_update(const muon_batch* batches, int nb, const muon_hparams
     P.slice_factor = factor;
     if (use_normuon) {
       normuon_rows_kernel<<<ew_grid(cdiv(row, EW_THREADS / 32), sms), EW_THREADS, 0, stream>>>(P);
-      if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+      if (!launched()) return MUON_CUDA_ERROR;
       normuon_slices_kernel<<<ew_grid(slice, sms), EW_THREADS, 0, stream>>>(P);
-      if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+      if (!launched()) return MUON_CUDA_ERROR;
     }
     update_kernel<<<ew_grid(chunk, sms), EW_THREADS, 0, stream>>>(P);
-    if (cudaGetLastError() != cudaSuccess) return MUON_CUDA_ERROR;
+    if (!launched()) return MUON_CUDA_ERROR;
   }
   return MUON_OK;
 }

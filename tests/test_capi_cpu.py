@@ -15,8 +15,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def mn():
-    from newton_schulz_ns_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._builder().build()
     import newton_schulz_ns_b200 as m
     return m
 
