@@ -188,6 +188,36 @@ MUON_API muon_status normuon_update(const muon_batch* batches, int nb, const muo
 /* Reads the error word at workspace offset 0 after synchronizing the stream:
  * 0 = no device-side wait timed out since the word was last cleared (each
  * Newton-Schulz call clears it when it starts). */
+/*
+ * muon_momentum_norm without a workspace argument.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory at the point where they run the step, such as code running
+ * under a framework or runtime that owns all device memory and hands out
+ * none after start-up, or a real-time or replay loop where allocation is
+ * not permitted, and that have nowhere to keep a workspace between calls.
+ *
+ * It computes exactly what muon_momentum_norm computes (same kernels, same
+ * arguments apart from the workspace) and keeps its per-chunk partial sums
+ * in a scratch array of MUON_NOALLOC_SCRATCH_FLOATS floats (4 MiB) that the
+ * library holds in static device memory on every GPU that loads it, until
+ * the process exits.  Nothing is allocated or freed by the call.
+ *
+ * Limits and sharing:
+ *  - the batches may hold at most MUON_NOALLOC_SCRATCH_FLOATS chunks of 8192
+ *    elements in total (about 8.6e9 elements); larger calls return
+ *    MUON_WORKSPACE_TOO_SMALL and enqueue nothing;
+ *  - every call on a device uses the same array, so calls whose kernels can
+ *    overlap on the GPU (different streams without ordering between them)
+ *    race on it; calls ordered on one stream are safe.  Each call overwrites
+ *    every partial it later reads, so nothing needs clearing between calls;
+ *  - the first call on a device looks up the array's device address (a
+ *    runtime query that does not allocate); make that first call before any
+ *    stream capture on that device.
+ */
+#define MUON_NOALLOC_SCRATCH_FLOATS (1 << 20)
+MUON_API muon_status muon_momentum_norm_noalloc(const muon_batch* batches, int nb, const muon_hparams* hp,
+                                                cudaStream_t stream);
+
 MUON_API muon_status muon_workspace_error(const void* workspace, cudaStream_t stream, int32_t* error_word);
 
 MUON_API const char* muon_status_string(muon_status status);

@@ -20,7 +20,7 @@ from ._capi import MUON_BF16, MUON_F16, MUON_F32, MuonError  # noqa: F401
 
 __all__ = ["Batch", "Hparams", "muon_workspace_size", "muon_momentum_norm", "muon_ns_batched",
            "muon_gram_ns_batched", "normuon_update", "workspace_error", "testing_gemm", "spectral_scale",
-           "ns_flops", "version", "kernel_launches", "allocate_workspace", "MuonError", "LIB_PATH"]
+           "ns_flops", "version", "kernel_launches", "muon_momentum_norm_noalloc", "allocate_workspace", "MuonError", "LIB_PATH"]
 
 LIB_PATH = _capi.LIB_PATH
 
@@ -183,6 +183,19 @@ def muon_momentum_norm(batches: Sequence[Batch], hp: Hparams, workspace: torch.T
     p, nbytes = _ws(workspace)
     _capi.check(_capi.lib.muon_momentum_norm(arr, nb, ctypes.byref(h), p, nbytes, _stream_ptr(stream)),
                 "muon_momentum_norm")
+
+
+def muon_momentum_norm_noalloc(batches: Sequence[Batch], hp: Hparams, stream=None) -> None:
+    """muon_momentum_norm with the library's static device scratch instead of a workspace.
+
+    For callers that cannot allocate device memory where they run the step.
+    Calls that may overlap on the GPU share the scratch and race; the first
+    call on a device should come before any stream capture on it.
+    """
+    arr, nb = _batches(batches)
+    h, _keep = hp.to_c()
+    _capi.check(_capi.lib.muon_momentum_norm_noalloc(arr, nb, ctypes.byref(h), _stream_ptr(stream)),
+                "muon_momentum_norm_noalloc")
 
 
 def muon_ns_batched(batches: Sequence[Batch], hp: Hparams, workspace: torch.Tensor, stream=None) -> None:

@@ -49,7 +49,7 @@ class MuonHparams(ctypes.Structure):
 
 EXPORTS = ("muon_workspace_size", "muon_momentum_norm", "muon_ns_batched", "muon_gram_ns_batched",
            "normuon_update", "muon_workspace_error", "muon_status_string", "muon_version",
-           "muon_testing_gemm", "muon_kernel_launches")
+           "muon_testing_gemm", "muon_kernel_launches", "muon_momentum_norm_noalloc")
 
 
 def _load() -> ctypes.CDLL:
@@ -69,6 +69,8 @@ def _load() -> ctypes.CDLL:
     for fn in (lib.muon_momentum_norm, lib.muon_ns_batched, lib.muon_gram_ns_batched):
         fn.argtypes = [B, ctypes.c_int, H, P, ctypes.c_size_t, P]
         fn.restype = ctypes.c_int
+    lib.muon_momentum_norm_noalloc.argtypes = [B, ctypes.c_int, H, P]
+    lib.muon_momentum_norm_noalloc.restype = ctypes.c_int
     lib.normuon_update.argtypes = [B, ctypes.c_int, H, ctypes.c_int, P, ctypes.c_size_t, P]
     lib.normuon_update.restype = ctypes.c_int
     lib.muon_workspace_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]

@@ -564,6 +564,32 @@ muon_status prepare_norms(const muon_batch* bs, int nb, const Layout& L, uint8_t
 
 }  // namespace
 
+// Scratch of muon_momentum_norm_noalloc: per-chunk partial sums in static
+// device memory, so that entry point allocates nothing.  Host code must not
+// pass the symbol itself to a kernel (on the host it names a shadow
+// variable); it passes the device address looked up per device below.
+static __device__ __align__(256) float g_noalloc_partials[MUON_NOALLOC_SCRATCH_FLOATS];
+
+namespace {
+std::mutex g_noalloc_mu;
+float* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_partials on the current device, looked up once
+// per device with that device current.
+muon_status noalloc_scratch(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MUON_CUDA_ERROR;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_partials) != cudaSuccess || p == nullptr) return MUON_CUDA_ERROR;
+    g_noalloc_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return MUON_OK;
+}
+}  // namespace
+
 // ============================================================================
 // C ABI
 // ============================================================================
@@ -631,6 +657,34 @@ muon_status muon_momentum_norm(const muon_batch* batches, int nb, const muon_hpa
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   return launch_norm(batches, nb, hp, 0, reinterpret_cast<float*>(ws + L.partials),
                      reinterpret_cast<float*>(ws + L.sumsq), sms, stream);
+}
+
+muon_status muon_momentum_norm_noalloc(const muon_batch* batches, int nb, const muon_hparams* hp,
+                                       cudaStream_t stream) {
+  if (nb < 0 || (nb > 0 && !batches)) return MUON_INVALID_ARG;
+  muon_status st = check_hp(hp);
+  if (st != MUON_OK) return st;
+  bool any = false;
+  for (int i = 0; i < nb; ++i) {
+    const muon_batch& b = batches[i];
+    if ((st = check_shape(b)) != MUON_OK) return st;
+    if (batch_empty(b)) continue;
+    any = true;
+    if ((st = check_view(b, b.grad, {MUON_F32, MUON_BF16}, false)) != MUON_OK) return st;
+    if ((st = check_view(b, b.momentum, {MUON_F32, MUON_BF16}, false)) != MUON_OK) return st;
+    if ((st = check_view(b, b.ns_in, {MUON_BF16}, false)) != MUON_OK) return st;
+    if (!b.sumsq) return MUON_INVALID_ARG;
+  }
+  if (!any) return MUON_OK;
+  const Layout L = plan_layout(batches, nb, 0);
+  if (L.total_chunks > MUON_NOALLOC_SCRATCH_FLOATS) return MUON_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  if ((st = device_setup(&sms)) != MUON_OK) return st;
+  float* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != MUON_OK) return st;
+  // Every batch carries its own sumsq, so the finalize step never writes the
+  // fallback array; it is given the scratch only as a valid pointer.
+  return launch_norm(batches, nb, hp, 0, scratch, scratch, sms, stream);
 }
 
 muon_status muon_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
