@@ -226,7 +226,8 @@ struct Mat {                 // a strided batch of row-major [rows][cols] matric
   int f16;                   // element type: 1 fp16, 0 bf16
 };
 
-bool encode_map(CUtensorMap* map, const Mat& m, int box_x, int box_y) {
+bool encode_map(CUtensorMap* map, const Mat& m, int box_x, int box_y,
+                CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(m.cols), static_cast<cuuint64_t>(m.rows),
                         static_cast<cuuint64_t>(m.n)};
   const int64_t bs = m.n > 1 ? m.bs : m.ld * m.rows;
@@ -235,7 +236,7 @@ bool encode_map(CUtensorMap* map, const Mat& m, int box_x, int box_y) {
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = g_encode(map, m.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                               const_cast<void*>(m.ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -314,6 +315,10 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
       // A operand: K-major box 64 (K) x 128 rows; MN-major box 64 (M) x 64 (K rows).
       if (!encode_map(&P.mapA[np], s.a, 64, s.a_mn ? 64 : BM)) return MUON_CUDA_ERROR;
       if (!encode_map(&P.mapB[np], s.b, 64, s.b_mn ? 64 : BN)) return MUON_CUDA_ERROR;
+      // Output: 32 x 32 boxes, swizzled for the direct staging layout, plain for the transposed one.
+      const Mat c{s.out, s.M, s.N, s.out_ld, s.out_bs, s.slices, s.out_f16};
+      if (!encode_map(&P.mapC[np], c, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return MUON_CUDA_ERROR;
+      if (!encode_map(&P.mapCT[np], c, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) return MUON_CUDA_ERROR;
       const long long t = static_cast<long long>(g.tiles_per_slice) * s.slices;
       if (tiles + t > INT32_MAX) return MUON_BAD_SHAPE;
       tiles += static_cast<int>(t);

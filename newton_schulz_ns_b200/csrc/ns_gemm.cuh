@@ -13,9 +13,15 @@
 // s = 1 / (sqrt(sumsq[slice]) + eps) and p in {0, 1, 2}.
 //
 // Symmetric problems ("tri") compute only the 128x256 tiles that touch the
-// lower triangle and write each lower element and its mirror, so A = X X^T
-// and B = b*A + c*A^2 cost about half of a full product (the one-triangle
-// products of the Megatron-Core layer_sharded_muon docs, use_syrk).
+// lower triangle, so A = X X^T and B = b*A + c*A^2 cost about half of a full
+// product (the one-triangle products of the Megatron-Core
+// layer_sharded_muon docs, use_syrk).  The two tiles of each 256 x 256
+// diagonal block are written as computed; every tile below them is written
+// twice, as computed and transposed into the upper triangle.
+//
+// The epilogue stages each warp's 32 x 32 piece of the tile in shared
+// memory (double-buffered) and writes it, and its transpose for mirrored
+// tiles, with TMA bulk tensor stores, which clip at the slice's bounds.
 //
 // Roles (192 threads, one CTA per SM, persistent over a static tile stride):
 //   warp 0 lane 0 : TMA producer over a STAGES-deep shared-memory ring
@@ -46,7 +52,11 @@ constexpr int MN_BLOCK_BYTES = 64 * BK * 2;      // one [64 K rows][64 MN] swizz
 constexpr uint32_t TMEM_COLS = 2 * BN;           // two accumulators
 constexpr int GEMM_THREADS = 192;
 constexpr int MAX_PROBLEMS = 8;
-constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int EPI_WARPS = 4;
+constexpr int STG_BYTES = 32 * 32 * 2;                      // one 32 x 32 box of 16-bit values
+constexpr int STG_PER_WARP = 2 /*buffers*/ * 2 /*direct, mirror*/ * STG_BYTES;
+constexpr int GEMM_SMEM_BYTES =
+    STAGES * STAGE_BYTES + EPI_WARPS * STG_PER_WARP + 1024 /*align*/ + 256 /*barriers*/;
 
 enum GemmError : int { kErrNone = 0, kErrProducer = 1, kErrMma = 2, kErrEpilogue = 3 };
 
@@ -75,6 +85,8 @@ struct GemmProblem {
 struct __align__(64) GemmParams {
   CUtensorMap mapA[MAX_PROBLEMS];
   CUtensorMap mapB[MAX_PROBLEMS];
+  CUtensorMap mapC[MAX_PROBLEMS];     // output, 32 x 32 boxes, 64-byte swizzle (direct tiles)
+  CUtensorMap mapCT[MAX_PROBLEMS];    // output, 32 x 32 boxes, no swizzle (mirrored tiles)
   GemmProblem prob[MAX_PROBLEMS];
   int num_problems;
   int total_tiles;
@@ -120,25 +132,14 @@ __device__ __forceinline__ float load_elem(const void* base, long long off, int 
   return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[off]);
 }
 
-// Rounds v to the output type, stores it, and returns the rounded value.
-__device__ __forceinline__ float store_elem(void* base, long long off, float v, int f16) {
-  if (f16) {
-    __half h = __float2half_rn(v);
-    reinterpret_cast<__half*>(base)[off] = h;
-    return __half2float(h);
-  }
-  __nv_bfloat16 h = __float2bfloat16_rn(v);
-  reinterpret_cast<__nv_bfloat16*>(base)[off] = h;
-  return __bfloat162float(h);
-}
-
 __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_constant__ GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* sStg = smem + STAGES * STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + EPI_WARPS * STG_PER_WARP);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -168,6 +169,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
     for (int p = 0; p < P.num_problems; ++p) {
       tma_prefetch_desc(&P.mapA[p]);
       tma_prefetch_desc(&P.mapB[p]);
+      tma_prefetch_desc(&P.mapC[p]);
+      tma_prefetch_desc(&P.mapCT[p]);
     }
   }
   if (warp == 1) {
@@ -292,7 +295,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    uint8_t* stg = sStg + (warp - 2) * STG_PER_WARP;
     int iter = 0;
+    uint32_t stores = 0;     // bulk groups this warp has committed (selects the staging buffer)
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++iter) {
       const TileCoord tc = decode_tile(P, t);
       const GemmProblem& pr = P.prob[tc.p];
@@ -306,14 +311,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
       }
       tc_fence_after();
 
-      const int row = tc.tm * BM + q * 32 + lane;
+      const int row0 = tc.tm * BM + q * 32;
+      const int row = row0 + lane;
       const bool row_ok = row < pr.M;
+      // Mirrored tiles: strictly below the 256 x 256 diagonal blocks.
+      const bool mirror = pr.tri && tc.tm >= 2 * tc.tn + 2;
       float f = pr.f0;
       if (pr.s_pow > 0) {
         const float s = 1.0f / (sqrtf(pr.sumsq[tc.slice]) + pr.eps);
         f *= (pr.s_pow == 2) ? s * s : s;
       }
-      const long long out_slice = static_cast<long long>(tc.slice) * pr.out_bs;
       const long long add_slice = static_cast<long long>(tc.slice) * pr.add_bs;
       const bool use_add = pr.beta != 0.0f && pr.addend != nullptr;
       float rss = 0.0f;
@@ -325,12 +332,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
                            r);
         tmem_ld_wait();
         const int col0 = tc.tn * BN + c * 32;
-        if (col0 >= pr.N || !row_ok) continue;
+        if (col0 >= pr.N) continue;                       // warp-uniform
         const bool full_chunk = col0 + 32 <= pr.N;
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = pr.alpha * __uint_as_float(r[j]);
-        if (use_add) {
+        if (use_add && row_ok) {
           const long long aoff = add_slice + static_cast<long long>(row) * pr.add_ld + col0;
           if (full_chunk) {
             const uint4* src = reinterpret_cast<const uint4*>(
@@ -356,54 +363,77 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
               }
             }
           } else {
-            for (int j = 0; j < 32 && col0 + j < pr.N; ++j) v[j] += pr.beta * load_elem(pr.addend, aoff + j, pr.add_f16);
+            for (int j = 0; j < 32 && col0 + j < pr.N; ++j)
+              v[j] += pr.beta * load_elem(pr.addend, aoff + j, pr.add_f16);
           }
         }
+        // Round to the output type once; these are the values stored.
+        uint16_t h16[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] *= f;
-        if (pr.tri) {
-          for (int j = 0; j < 32; ++j) {
-            const int col = col0 + j;
-            if (col >= pr.N || col > row) break;
-            float x = v[j];
-            if (col == row) x += pr.gamma;
-            store_elem(pr.out, out_slice + static_cast<long long>(row) * pr.out_ld + col, x, pr.out_f16);
-            if (col < row) store_elem(pr.out, out_slice + static_cast<long long>(col) * pr.out_ld + row, x, pr.out_f16);
-          }
-        } else {
-          const long long ooff = out_slice + static_cast<long long>(row) * pr.out_ld + col0;
-          if (full_chunk) {
-            uint32_t packed[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              uint16_t lo, hi;
-              float rlo, rhi;
-              if (pr.out_f16) {
-                __half a = __float2half_rn(v[2 * j]), b = __float2half_rn(v[2 * j + 1]);
-                lo = __half_as_ushort(a);
-                hi = __half_as_ushort(b);
-                rlo = __half2float(a);
-                rhi = __half2float(b);
-              } else {
-                __nv_bfloat16 a = __float2bfloat16_rn(v[2 * j]), b = __float2bfloat16_rn(v[2 * j + 1]);
-                lo = __bfloat16_as_ushort(a);
-                hi = __bfloat16_as_ushort(b);
-                rlo = __bfloat162float(a);
-                rhi = __bfloat162float(b);
-              }
-              rss += rlo * rlo + rhi * rhi;
-              packed[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(pr.out) + ooff);
-#pragma unroll
-            for (int w = 0; w < 4; ++w)
-              dst[w] = make_uint4(packed[4 * w], packed[4 * w + 1], packed[4 * w + 2], packed[4 * w + 3]);
+        for (int j = 0; j < 32; ++j) {
+          float x = v[j] * f;
+          if (pr.gamma != 0.0f && row == col0 + j) x += pr.gamma;
+          float xr;
+          if (pr.out_f16) {
+            const __half hv = __float2half_rn(x);
+            h16[j] = __half_as_ushort(hv);
+            xr = __half2float(hv);
           } else {
-            for (int j = 0; j < 32 && col0 + j < pr.N; ++j) {
-              const float x = store_elem(pr.out, ooff + j, v[j], pr.out_f16);
-              rss += x * x;
+            const __nv_bfloat16 hv = __float2bfloat16_rn(x);
+            h16[j] = __bfloat16_as_ushort(hv);
+            xr = __bfloat162float(hv);
+          }
+          if (row_ok && col0 + j < pr.N) rss += xr * xr;
+        }
+        // Boxes whose innermost extent lies fully inside the slice go out by
+        // TMA; the ragged last chunk of a row (and of a mirrored column) is
+        // written element by element, so nothing past the slice's last column
+        // is ever touched.
+        const bool st_d = full_chunk;
+        const bool st_m = mirror && row0 + 32 <= pr.M;
+        const long long out_slice = static_cast<long long>(tc.slice) * pr.out_bs;
+        uint16_t* out16 = reinterpret_cast<uint16_t*>(pr.out);
+        if (st_d || st_m) {
+          // The staging buffer used two stores ago must have been read out.
+          const uint32_t buf = stores & 1u;
+          uint8_t* sd = stg + buf * (2 * STG_BYTES);
+          uint8_t* sm = sd + STG_BYTES;
+          if (lane == 0 && stores >= 2) bulk_wait_group_read<1>();
+          __syncwarp();
+          if (st_d) {
+            // Row `lane`, 64 bytes, 16-byte chunks placed by the 64-byte swizzle.
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const uint4 val = make_uint4(
+                  static_cast<uint32_t>(h16[8 * w + 0]) | (static_cast<uint32_t>(h16[8 * w + 1]) << 16),
+                  static_cast<uint32_t>(h16[8 * w + 2]) | (static_cast<uint32_t>(h16[8 * w + 3]) << 16),
+                  static_cast<uint32_t>(h16[8 * w + 4]) | (static_cast<uint32_t>(h16[8 * w + 5]) << 16),
+                  static_cast<uint32_t>(h16[8 * w + 6]) | (static_cast<uint32_t>(h16[8 * w + 7]) << 16));
+              *reinterpret_cast<uint4*>(sd + lane * 64 + ((w ^ ((lane >> 1) & 3)) << 4)) = val;
             }
           }
+          if (st_m) {
+            // Transposed box: row j holds column j of this warp's 32 rows.
+            uint16_t* mt = reinterpret_cast<uint16_t*>(sm);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) mt[j * 32 + lane] = h16[j];
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (st_d) tma_store_3d(&P.mapC[tc.p], sd, col0, row0, tc.slice);
+            if (st_m) tma_store_3d(&P.mapCT[tc.p], sm, row0, col0, tc.slice);
+            bulk_commit_group();
+          }
+          ++stores;
+        }
+        if (!st_d && row_ok) {
+          for (int j = 0; j < 32 && col0 + j < pr.N; ++j)
+            out16[out_slice + static_cast<long long>(row) * pr.out_ld + col0 + j] = h16[j];
+        }
+        if (mirror && !st_m && row_ok) {
+          for (int j = 0; j < 32 && col0 + j < pr.N; ++j)
+            out16[out_slice + static_cast<long long>(col0 + j) * pr.out_ld + row] = h16[j];
         }
       }
       if (pr.row_ss != nullptr && row_ok)
@@ -411,6 +441,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
+    // Every store has landed before the kernel (and its shared memory) ends.
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
 
   tc_fence_before();
