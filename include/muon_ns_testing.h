@@ -16,6 +16,10 @@
  * when beta == 0.  All pointers are device memory; ld/bs are in elements.
  * row_ss (device, may be NULL; non-tri only) receives, per slice, per
  * 256-column block and per row, the sum of squares of the stored C values.
+ * cta_pair: 0 lets the library choose the tile kernel, 1 forces single-CTA
+ * 128 x 256 tiles, 2 forces 2-CTA (cta_group::2) 256 x 256 tiles.
+ * raster_group: row tiles per raster band of a non-symmetric problem
+ * (0: the library's default).
  * The workspace (>= 256 bytes, 256-byte aligned) receives the error word.
  */
 #ifndef MUON_NS_TESTING_H_
@@ -34,7 +38,8 @@ MUON_API muon_status muon_testing_gemm(int M, int N, int K, int slices, int tri,
                               void* C, int64_t ldc, int64_t bsc, int out_dtype,
                               float alpha, float beta, float gamma, float f0,
                               int s_pow, const float* sumsq, float eps, float* row_ss,
-                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+                              int cta_pair, int raster_group, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

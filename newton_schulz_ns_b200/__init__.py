@@ -233,13 +233,14 @@ def workspace_error(workspace: torch.Tensor, stream=None) -> int:
 def testing_gemm(A: torch.Tensor, a_mn: bool, B: torch.Tensor, b_mn: bool, C: torch.Tensor, *, K: int,
                  tri: bool = False, D: Optional[torch.Tensor] = None, alpha: float = 1.0, beta: float = 0.0,
                  gamma: float = 0.0, f0: float = 1.0, s_pow: int = 0, sumsq: Optional[torch.Tensor] = None,
-                 eps: float = 0.0, row_ss: Optional[torch.Tensor] = None, workspace: torch.Tensor = None,
-                 stream=None) -> None:
+                 eps: float = 0.0, row_ss: Optional[torch.Tensor] = None, cta_pair: int = 0,
+                 raster_group: int = 0, workspace: torch.Tensor = None, stream=None) -> None:
     """Runs one tensor-core GEMM problem of the library (include/muon_ns_testing.h).
 
     A, B, C, D are 3-D [slices, rows, cols] with contiguous rows.  C is
     [slices, M, N]; A is [slices, M, K] (a_mn False) or [slices, K, M];
-    B is [slices, N, K] (b_mn False) or [slices, K, N].
+    B is [slices, N, K] (b_mn False) or [slices, K, N].  cta_pair: 0 the
+    library's choice, 1 single-CTA tiles, 2 CTA-pair tiles.
     """
     S, M, N = C.shape
     if A.dtype != B.dtype:
@@ -259,5 +260,6 @@ def testing_gemm(A: torch.Tensor, a_mn: bool, B: torch.Tensor, b_mn: bool, C: to
         D.data_ptr() if D is not None else None, ldd, bsd, _DT[D.dtype] if D is not None else MUON_BF16,
         C.data_ptr(), ldc, bsc, _DT[C.dtype], alpha, beta, gamma, f0, s_pow,
         sumsq.data_ptr() if sumsq is not None else None, eps,
-        row_ss.data_ptr() if row_ss is not None else None, p, nbytes, _stream_ptr(stream))
+        row_ss.data_ptr() if row_ss is not None else None, int(cta_pair), int(raster_group), p, nbytes,
+        _stream_ptr(stream))
     _capi.check(st, "muon_testing_gemm")

@@ -84,7 +84,7 @@ def _load() -> ctypes.CDLL:
     i64, i32, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_float
     lib.muon_testing_gemm.argtypes = [i32, i32, i32, i32, i32, i32,
                                       P, i64, i64, i32, P, i64, i64, i32, P, i64, i64, i32,
-                                      P, i64, i64, i32, f32, f32, f32, f32, i32, P, f32, P,
+                                      P, i64, i64, i32, f32, f32, f32, f32, i32, P, f32, P, i32, i32,
                                       P, ctypes.c_size_t, P]
     lib.muon_testing_gemm.restype = ctypes.c_int
     return lib

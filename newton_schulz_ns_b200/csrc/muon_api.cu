@@ -41,6 +41,7 @@ struct DeviceInfo {
   bool ready = false;
   bool ok = false;
   int sms = 0;
+  int pair_units = 0;   // 2-CTA clusters of the pair GEMM that fit on the device at once
 };
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
@@ -54,7 +55,7 @@ inline bool launched() {
   return true;
 }
 
-muon_status device_setup(int* sms_out) {
+muon_status device_setup(int* sms_out, int* pair_units_out = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MUON_CUDA_ERROR;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -71,11 +72,23 @@ muon_status device_setup(int* sms_out) {
     d.sms = sms;
     d.ok = (major == 10 && minor == 0);
     if (d.ok) {
-      if (cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) !=
-          cudaSuccess) {
+      if (cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               GemmCfg<1>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(ns_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               GemmCfg<2>::SMEM_BYTES) != cudaSuccess) {
         d.ready = false;
         return MUON_CUDA_ERROR;
       }
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+      cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+      cfg.dynamicSmemBytes = GemmCfg<2>::SMEM_BYTES;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, ns_gemm_pair_kernel, &cfg) != cudaSuccess || clusters <= 0) {
+        (void)cudaGetLastError();
+        clusters = sms / 2;
+      }
+      d.pair_units = std::min(clusters, sms / 2);
     }
     if (!g_encode) {
       void* fn = nullptr;
@@ -90,6 +103,7 @@ muon_status device_setup(int* sms_out) {
   }
   if (!d.ok) return MUON_UNSUPPORTED_DEVICE;
   *sms_out = d.sms;
+  if (pair_units_out) *pair_units_out = d.pair_units;
   return MUON_OK;
 }
 
@@ -263,39 +277,76 @@ struct ProblemSpec {
   float* row_ss;
 };
 
-muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* err, cudaStream_t stream) {
+// Builds every launch of `specs` (at most MAX_PROBLEMS problems each) and
+// then enqueues them, so that an encoding error enqueues nothing.
+// cta_pair: 0 chooses per launch (pairs when every problem has at least 256
+// rows), 1 forces single-CTA tiles, 2 forces CTA pairs.
+muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* err, cudaStream_t stream,
+                         int cta_pair = 0, int raster_group = 0) {
+  int pair_units = 0;
+  {
+    int s2 = 0;
+    muon_status st = device_setup(&s2, &pair_units);
+    if (st != MUON_OK) return st;
+  }
+  struct Launch {
+    GemmParams P;
+    int cg;
+  };
+  std::vector<Launch> launches;
   size_t i = 0;
   while (i < specs.size()) {
-    GemmParams P;
+    // The next group of non-empty problems.
+    std::vector<const ProblemSpec*> group;
+    for (; i < specs.size() && static_cast<int>(group.size()) < MAX_PROBLEMS; ++i) {
+      const ProblemSpec& s = specs[i];
+      if (s.slices == 0 || s.M == 0 || s.N == 0) continue;
+      group.push_back(&s);
+    }
+    if (group.empty()) continue;
+    int cg = 1;
+    if (cta_pair == 2) {
+      cg = 2;
+    } else if (cta_pair == 0 && pair_units > 0) {
+      cg = 2;
+      for (const ProblemSpec* s : group)
+        if (s->M < 256) cg = 1;
+    }
+    const int tile_m = BM * cg, b_rows = BN / cg, step = BN / tile_m;
+    launches.emplace_back();
+    Launch& L = launches.back();
+    L.cg = cg;
+    GemmParams& P = L.P;
     std::memset(&P, 0, sizeof(P));
     P.err = err;
     P.timeout_ns = kWaitLimitNs;
-    int tiles = 0;
+    long long tiles = 0;
     int np = 0;
-    for (; i < specs.size() && np < MAX_PROBLEMS; ++i) {
-      const ProblemSpec& s = specs[i];
-      if (s.slices == 0 || s.M == 0 || s.N == 0) continue;
+    for (const ProblemSpec* sp : group) {
+      const ProblemSpec& s = *sp;
       GemmProblem& g = P.prob[np];
       g.M = s.M;
       g.N = s.N;
       g.K = s.K;
       g.slices = s.slices;
-      g.mt = static_cast<int>(cdiv(s.M, BM));
+      g.mt = static_cast<int>(cdiv(s.M, tile_m));
       g.nt = static_cast<int>(cdiv(s.N, BN));
-      g.kt = static_cast<int>(cdiv(s.K, BK));
+      g.kt = static_cast<int>(cdiv(s.K, cg == 2 ? GemmCfg<2>::KB : GemmCfg<1>::KB));
       g.tri = s.tri;
       if (s.tri) {
         int cnt = 0;
-        for (int j = 0; j < g.nt; ++j) cnt += std::max(0, g.mt - 2 * j);
+        for (int j = 0; j < g.nt; ++j) cnt += std::max(0, g.mt - step * j);
         g.tiles_per_slice = cnt;
       } else {
         g.tiles_per_slice = g.mt * g.nt;
       }
-      g.tile_begin = tiles;
+      g.tile_begin = static_cast<int>(tiles);
+      // Raster bands: about sqrt(units * 256 / tile_m) row tiles (16 single, 8 paired).
+      g.group_m = std::max(1, std::min(g.mt, raster_group > 0 ? raster_group : (cg == 2 ? 8 : 16)));
       g.a_mn = s.a_mn;
       g.b_mn = s.b_mn;
-      g.idesc = mma_idesc_f16(s.in_f16 ? 0u : 1u, static_cast<uint32_t>(s.a_mn), static_cast<uint32_t>(s.b_mn), BM,
-                              BN);
+      g.idesc = mma_idesc_f16(s.in_f16 ? 0u : 1u, static_cast<uint32_t>(s.a_mn), static_cast<uint32_t>(s.b_mn),
+                              static_cast<uint32_t>(tile_m), BN);
       g.alpha = s.alpha;
       g.beta = s.beta;
       g.gamma = s.gamma;
@@ -312,23 +363,30 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
       g.out_bs = s.out_bs;
       g.out_f16 = s.out_f16;
       g.row_ss = s.row_ss;
-      // A operand: K-major box 64 (K) x 128 rows; MN-major box 64 (M) x 64 (K rows).
-      if (!encode_map(&P.mapA[np], s.a, 64, s.a_mn ? 64 : BM)) return MUON_CUDA_ERROR;
-      if (!encode_map(&P.mapB[np], s.b, 64, s.b_mn ? 64 : BN)) return MUON_CUDA_ERROR;
+      // A: K-major box 64 (K) x 128 rows; MN-major box 64 (M) x (K per stage) rows.
+      // B: K-major box 64 x (256 / CTAs) rows; MN-major as A.
+      const int kb_rows = cg == 2 ? GemmCfg<2>::KB : GemmCfg<1>::KB;
+      if (!encode_map(&P.mapA[np], s.a, 64, s.a_mn ? kb_rows : BM)) return MUON_CUDA_ERROR;
+      if (!encode_map(&P.mapB[np], s.b, 64, s.b_mn ? kb_rows : b_rows)) return MUON_CUDA_ERROR;
       // Output: 32 x 32 boxes, swizzled for the direct staging layout, plain for the transposed one.
       const Mat c{s.out, s.M, s.N, s.out_ld, s.out_bs, s.slices, s.out_f16};
       if (!encode_map(&P.mapC[np], c, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return MUON_CUDA_ERROR;
       if (!encode_map(&P.mapCT[np], c, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) return MUON_CUDA_ERROR;
-      const long long t = static_cast<long long>(g.tiles_per_slice) * s.slices;
-      if (tiles + t > INT32_MAX) return MUON_BAD_SHAPE;
-      tiles += static_cast<int>(t);
+      tiles += static_cast<long long>(g.tiles_per_slice) * s.slices;
+      if (tiles > INT32_MAX) return MUON_BAD_SHAPE;
       ++np;
     }
-    if (np == 0) continue;
     P.num_problems = np;
-    P.total_tiles = tiles;
-    const int grid = std::min(tiles, sms);
-    ns_gemm_kernel<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(P);
+    P.total_tiles = static_cast<int>(tiles);
+  }
+  for (const Launch& L : launches) {
+    if (L.cg == 2) {
+      const int units = std::max(1, std::min(L.P.total_tiles, pair_units));
+      ns_gemm_pair_kernel<<<2 * units, GEMM_THREADS, GemmCfg<2>::SMEM_BYTES, stream>>>(L.P);
+    } else {
+      const int grid = std::min(L.P.total_tiles, sms);
+      ns_gemm_kernel<<<grid, GEMM_THREADS, GemmCfg<1>::SMEM_BYTES, stream>>>(L.P);
+    }
     if (!launched()) return MUON_CUDA_ERROR;
   }
   return MUON_OK;
@@ -905,9 +963,10 @@ muon_status muon_testing_gemm(int M, int N, int K, int slices, int tri, int in_d
                               int64_t bsa, int a_mn, const void* B, int64_t ldb, int64_t bsb, int b_mn,
                               const void* D, int64_t ldd, int64_t bsd, int add_dtype, void* C, int64_t ldc,
                               int64_t bsc, int out_dtype, float alpha, float beta, float gamma, float f0, int s_pow,
-                              const float* sumsq, float eps, float* row_ss, void* workspace,
-                              size_t workspace_bytes, cudaStream_t stream) {
+                              const float* sumsq, float eps, float* row_ss, int cta_pair, int raster_group,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (M < 0 || N < 0 || K < 1 || slices < 0) return MUON_BAD_SHAPE;
+  if (cta_pair < 0 || cta_pair > 2 || raster_group < 0) return MUON_INVALID_ARG;
   if (tri && M != N) return MUON_BAD_SHAPE;
   if (!A || !B || !C) return MUON_INVALID_ARG;
   if (beta != 0.0f && !D) return MUON_INVALID_ARG;
@@ -954,7 +1013,7 @@ muon_status muon_testing_gemm(int M, int N, int K, int slices, int tri, int in_d
   s.out_f16 = out_dtype == MUON_F16;
   s.row_ss = tri ? nullptr : row_ss;
   std::vector<ProblemSpec> v{s};
-  return launch_gemms(v, sms, reinterpret_cast<int*>(workspace), stream);
+  return launch_gemms(v, sms, reinterpret_cast<int*>(workspace), stream, cta_pair, raster_group);
 }
 
 }  // extern "C"

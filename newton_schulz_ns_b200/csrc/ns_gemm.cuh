@@ -4,28 +4,35 @@
 // same-shape slices C[s] = epilogue(opA(A[s]) * opB(B[s])) with
 //   opA: M x K, stored K-major ([M][K] row-major) or MN-major ([K][M]);
 //   opB: K x N, stored K-major ([N][K], i.e. C = A B^T) or MN-major ([K][N]).
-// Tiles are 128 x 256 (BM x BN) with 64-wide K blocks.  Operands are
-// brought into shared memory by TMA (128-byte swizzle, zero fill outside the
-// slice), multiplied by tcgen05.mma (bf16 or fp16 in, fp32 accumulate in
-// TMEM), and the epilogue applies
+// Output tiles are TILE_M x 256 with 64-wide K blocks.  Two variants share
+// the code: CG = 1 runs one CTA per 128 x 256 tile; CG = 2 runs a 2-CTA
+// cluster per 256 x 256 tile with the pair MMA (cta_group::2), each CTA
+// holding half of A and half of B in its shared memory, which halves the
+// operand bytes each SM moves per flop.  Operands are brought into shared
+// memory by TMA (128-byte swizzle, zero fill outside the slice), multiplied
+// by tcgen05.mma (bf16 or fp16 in, fp32 accumulate in TMEM), and the
+// epilogue applies
 //   C = f * (alpha * acc + beta * D) + gamma * [row == col]
 // where D is an addend with C's shape and f = f0 * s^p per slice, with
 // s = 1 / (sqrt(sumsq[slice]) + eps) and p in {0, 1, 2}.
 //
-// Symmetric problems ("tri") compute only the 128x256 tiles that touch the
-// lower triangle, so A = X X^T and B = b*A + c*A^2 cost about half of a full
+// Symmetric problems ("tri") compute only the tiles that touch the lower
+// triangle, so A = X X^T and B = b*A + c*A^2 cost about half of a full
 // product (the one-triangle products of the Megatron-Core
-// layer_sharded_muon docs, use_syrk).  The two tiles of each 256 x 256
-// diagonal block are written as computed; every tile below them is written
-// twice, as computed and transposed into the upper triangle.
+// layer_sharded_muon docs, use_syrk).  The tiles of each 256 x 256 diagonal
+// block are written as computed; every tile below them is written twice, as
+// computed and transposed into the upper triangle.
 //
 // The epilogue stages each warp's 32 x 32 piece of the tile in shared
 // memory (double-buffered) and writes it, and its transpose for mirrored
 // tiles, with TMA bulk tensor stores, which clip at the slice's bounds.
 //
 // Roles (192 threads, one CTA per SM, persistent over a static tile stride):
-//   warp 0 lane 0 : TMA producer over a STAGES-deep shared-memory ring
-//   warp 1        : TMEM allocation; lane 0 issues the MMAs
+//   warp 0 lane 0 : TMA producer over a STAGES-deep shared-memory ring (in a
+//                   pair, both CTAs load their halves; the leader's barrier
+//                   counts the bytes of both)
+//   warp 1        : TMEM allocation; lane 0 issues the MMAs (the leader only
+//                   in a pair; its commits reach both CTAs' barriers)
 //   warps 2..5    : epilogue, one TMEM lane (= output row) per thread;
 //                   two 256-column accumulators let the epilogue of one
 //                   tile overlap the main loop of the next.
@@ -41,22 +48,36 @@
 
 namespace muon {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_STAGE_BYTES = BM * BK * 2;
-constexpr int B_STAGE_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-constexpr int MN_BLOCK_BYTES = 64 * BK * 2;      // one [64 K rows][64 MN] swizzled block
+constexpr int BM = 128;                          // rows of A (and of the accumulator) per CTA
+constexpr int BN = 256;                          // columns of a tile
+constexpr int BK = 64;                           // K of one TMA box (one 128-byte swizzled row of bf16)
 constexpr uint32_t TMEM_COLS = 2 * BN;           // two accumulators
 constexpr int GEMM_THREADS = 192;
 constexpr int MAX_PROBLEMS = 8;
 constexpr int EPI_WARPS = 4;
 constexpr int STG_BYTES = 32 * 32 * 2;                      // one 32 x 32 box of 16-bit values
 constexpr int STG_PER_WARP = 2 /*buffers*/ * 2 /*direct, mirror*/ * STG_BYTES;
-constexpr int GEMM_SMEM_BYTES =
-    STAGES * STAGE_BYTES + EPI_WARPS * STG_PER_WARP + 1024 /*align*/ + 256 /*barriers*/;
+
+// A stage holds KB = 64 * KSUB elements of K.  K-major operands are KSUB
+// boxes of [rows][64] (one 128-byte swizzled row each); MN-major operands are
+// blocks of [KB rows][64 MN].  Several MMAs per stage amortize the stage's
+// barrier wait and commit: the pair kernel takes 128-wide K stages.
+template <int CG>
+struct GemmCfg {
+  static constexpr int TILE_M = BM * CG;                    // rows of a tile
+  static constexpr int B_ROWS = BN / CG;                    // rows of B this CTA loads
+  static constexpr int KSUB = CG == 1 ? 1 : 2;
+  static constexpr int KB = BK * KSUB;                      // K per stage
+  static constexpr int A_STAGE_BYTES = BM * KB * 2;
+  static constexpr int B_STAGE_BYTES = B_ROWS * KB * 2;
+  static constexpr int MN_BLOCK_BYTES = 64 * KB * 2;        // one [KB K rows][64 MN] swizzled block
+  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+  static constexpr int STAGES = CG == 1 ? 4 : 3;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_WARPS * STG_PER_WARP + 1024 /*align*/ +
+                                    256 /*barriers*/;
+  // Bytes the leader's full barrier counts per stage (both CTAs' loads in a pair).
+  static constexpr uint32_t TX_BYTES = static_cast<uint32_t>(STAGE_BYTES * CG);
+};
 
 enum GemmError : int { kErrNone = 0, kErrProducer = 1, kErrMma = 2, kErrEpilogue = 3 };
 
@@ -66,6 +87,7 @@ struct GemmProblem {
   int mt, nt, kt;           // tile counts along M, N, K
   int tiles_per_slice;
   int tile_begin;           // first linear tile of this problem in the launch
+  int group_m;              // non-symmetric problems: row tiles per raster band
   int tri;                  // symmetric output: lower-triangle tiles + mirror
   int a_mn, b_mn;           // operand majors (1 = MN-major)
   uint32_t idesc;           // tcgen05 instruction descriptor
@@ -98,7 +120,14 @@ struct TileCoord {
   int p, slice, tm, tn;
 };
 
+// Column j (256 output columns) of a symmetric problem needs the row tiles
+// from j * (256 / TILE_M) on.  Other problems are walked in bands of group_m
+// row tiles, M fastest within a band, so that the tiles in flight at once
+// cover a near-square block of the output and share operand rows and
+// columns in L2.
+template <int CG>
 __device__ __forceinline__ TileCoord decode_tile(const GemmParams& P, int t) {
+  constexpr int STEP = BN / GemmCfg<CG>::TILE_M;
   int p = 0;
   while (p + 1 < P.num_problems && t >= P.prob[p + 1].tile_begin) ++p;
   const GemmProblem& pr = P.prob[p];
@@ -107,17 +136,19 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& P, int t) {
   int r = local - slice * pr.tiles_per_slice;
   int tm, tn;
   if (pr.tri) {
-    // Column j of 256 output columns needs row tiles 2j .. mt-1.
     int j = 0;
-    while (r >= pr.mt - 2 * j) {
-      r -= pr.mt - 2 * j;
+    while (r >= pr.mt - STEP * j) {
+      r -= pr.mt - STEP * j;
       ++j;
     }
     tn = j;
-    tm = 2 * j + r;
+    tm = STEP * j + r;
   } else {
-    tm = r % pr.mt;
-    tn = r / pr.mt;
+    const int band = r / (pr.group_m * pr.nt);
+    const int rem = r - band * pr.group_m * pr.nt;
+    const int rows = min(pr.group_m, pr.mt - band * pr.group_m);
+    tn = rem / rows;
+    tm = band * pr.group_m + (rem - tn * rows);
   }
   return TileCoord{p, slice, tm, tn};
 }
@@ -132,13 +163,16 @@ __device__ __forceinline__ float load_elem(const void* base, long long off, int 
   return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[off]);
 }
 
-__global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_constant__ GemmParams P) {
+template <int CG>
+__device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
+  using Cfg = GemmCfg<CG>;
+  constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
-  uint8_t* sStg = smem + STAGES * STAGE_BYTES;
+  uint8_t* sB = smem + STAGES * Cfg::A_STAGE_BYTES;
+  uint8_t* sStg = smem + STAGES * Cfg::STAGE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + EPI_WARPS * STG_PER_WARP);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
@@ -151,6 +185,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint64_t limit = P.timeout_ns;
+  // In a pair, rank 0 is the leader (issues the MMAs); tiles are per pair.
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit = CG == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = CG == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -159,7 +198,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 128 * CG);     // every epilogue thread of the pair
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -174,11 +213,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc_pair(tmem_slot, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();   // the peer signals the leader's barriers only once they exist
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -194,34 +239,41 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
         last_par[s] = 0;
       }
       bool ok = true;
-      for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x) {
-        const TileCoord tc = decode_tile(P, t);
+      for (int t = unit; t < P.total_tiles && ok; t += units) {
+        const TileCoord tc = decode_tile<CG>(P, t);
         const GemmProblem& pr = P.prob[tc.p];
+        const int arow = tc.tm * Cfg::TILE_M + static_cast<int>(rank) * BM;      // this CTA's A rows
+        const int brow = tc.tn * BN + static_cast<int>(rank) * Cfg::B_ROWS;      // this CTA's B rows
         for (int kb = 0; kb < pr.kt; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit)) {
             record_error(P.err, abort_flag, kErrProducer);
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          uint8_t* a_dst = sA + stage * A_STAGE_BYTES;
-          uint8_t* b_dst = sB + stage * B_STAGE_BYTES;
-          const int k0 = kb * BK;
-          if (!pr.a_mn) {
-            tma_load_3d(a_dst, &P.mapA[tc.p], &full[stage], k0, tc.tm * BM, tc.slice);
-          } else {
+          if (leader) mbar_arrive_expect_tx(&full[stage], Cfg::TX_BYTES);
+          uint8_t* a_dst = sA + stage * Cfg::A_STAGE_BYTES;
+          uint8_t* b_dst = sB + stage * Cfg::B_STAGE_BYTES;
+          const int k0 = kb * Cfg::KB;
+          // K-major: KSUB boxes [rows][64]; MN-major: blocks [KB][64] along M (or N).
 #pragma unroll
-            for (int c = 0; c < BM / 64; ++c)
-              tma_load_3d(a_dst + c * MN_BLOCK_BYTES, &P.mapA[tc.p], &full[stage], tc.tm * BM + 64 * c, k0,
-                          tc.slice);
+          for (int j = 0; j < (pr.a_mn ? BM / 64 : Cfg::KSUB); ++j) {
+            const int x = pr.a_mn ? arow + 64 * j : k0 + 64 * j;
+            const int y = pr.a_mn ? k0 : arow;
+            uint8_t* dst = a_dst + j * (pr.a_mn ? Cfg::MN_BLOCK_BYTES : BM * BK * 2);
+            if (CG == 2)
+              tma_load_3d_pair(dst, &P.mapA[tc.p], &full[stage], x, y, tc.slice);
+            else
+              tma_load_3d(dst, &P.mapA[tc.p], &full[stage], x, y, tc.slice);
           }
-          if (!pr.b_mn) {
-            tma_load_3d(b_dst, &P.mapB[tc.p], &full[stage], k0, tc.tn * BN, tc.slice);
-          } else {
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              tma_load_3d(b_dst + c * MN_BLOCK_BYTES, &P.mapB[tc.p], &full[stage], tc.tn * BN + 64 * c, k0,
-                          tc.slice);
+          for (int j = 0; j < (pr.b_mn ? Cfg::B_ROWS / 64 : Cfg::KSUB); ++j) {
+            const int x = pr.b_mn ? brow + 64 * j : k0 + 64 * j;
+            const int y = pr.b_mn ? k0 : brow;
+            uint8_t* dst = b_dst + j * (pr.b_mn ? Cfg::MN_BLOCK_BYTES : Cfg::B_ROWS * BK * 2);
+            if (CG == 2)
+              tma_load_3d_pair(dst, &P.mapB[tc.p], &full[stage], x, y, tc.slice);
+            else
+              tma_load_3d(dst, &P.mapB[tc.p], &full[stage], x, y, tc.slice);
           }
           used[stage] = true;
           last_par[stage] = phase;
@@ -231,8 +283,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
           }
         }
       }
-      if (!ok) {
-        // Leave no bulk copy in flight into shared memory.
+      if (!ok && leader) {
+        // Leave no bulk copy in flight into shared memory (the leader's full
+        // barriers count the peer's copies too).
         for (int s = 0; s < STAGES; ++s)
           if (used[s]) {
             volatile int never = 0;
@@ -241,14 +294,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ------------------------------------------------------------ MMA issuer
       int stage = 0;
       uint32_t phase = 0;
       int iter = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x, ++iter) {
-        const TileCoord tc = decode_tile(P, t);
+      for (int t = unit; t < P.total_tiles && ok; t += units, ++iter) {
+        const TileCoord tc = decode_tile<CG>(P, t);
         const GemmProblem& pr = P.prob[tc.p];
         const int acc = iter & 1;
         const uint32_t acc_par = (iter >> 1) & 1;
@@ -259,36 +312,59 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < pr.kt; ++kb) {
+        // Descriptors of stage 0, advanced by adding to the start-address
+        // field (bits 0-13, in 16-byte units; shared memory stays below 256 KB).
+        // K-major: the next 16 K elements are 32 bytes along the swizzled row,
+        // and every 64 K the next box; MN-major: the next 16 K rows are two
+        // 8-row groups, 2048 bytes.
+        const uint64_t a_desc0 = pr.a_mn ? smem_desc_sw128(smem_u32(sA), Cfg::MN_BLOCK_BYTES, 1024)
+                                         : smem_desc_sw128(smem_u32(sA), 16, 1024);
+        const uint64_t b_desc0 = pr.b_mn ? smem_desc_sw128(smem_u32(sB), Cfg::MN_BLOCK_BYTES, 1024)
+                                         : smem_desc_sw128(smem_u32(sB), 16, 1024);
+        const bool a_mn = pr.a_mn != 0, b_mn = pr.b_mn != 0;
+        const uint32_t idesc = pr.idesc;
+        const int kt = pr.kt;
+        for (int kb = 0; kb < kt; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, limit)) {
             record_error(P.err, abort_flag, kErrMma);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + stage * A_STAGE_BYTES);
-          const uint32_t b_base = smem_u32(sB + stage * B_STAGE_BYTES);
+          const uint64_t ad = a_desc0 + static_cast<uint64_t>((stage * Cfg::A_STAGE_BYTES) >> 4);
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>((stage * Cfg::B_STAGE_BYTES) >> 4);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            // K-major: 16 elements = 32 bytes along the swizzled row.
-            // MN-major: 16 K rows = two 8-row groups of 1024 bytes.
-            const uint64_t ad = pr.a_mn ? smem_desc_sw128(a_base + k * 2048, MN_BLOCK_BYTES, 1024)
-                                        : smem_desc_sw128(a_base + k * 32, 16, 1024);
-            const uint64_t bd = pr.b_mn ? smem_desc_sw128(b_base + k * 2048, MN_BLOCK_BYTES, 1024)
-                                        : smem_desc_sw128(b_base + k * 32, 16, 1024);
-            tc_mma_f16(d_tmem, ad, bd, pr.idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < Cfg::KB / 16; ++k) {
+            const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
+            const uint64_t ak = a_mn ? static_cast<uint64_t>(k * (2048 >> 4))
+                                     : static_cast<uint64_t>((k >> 2) * (BM * BK * 2 >> 4) + (k & 3) * 2);
+            const uint64_t bk = b_mn ? static_cast<uint64_t>(k * (2048 >> 4))
+                                     : static_cast<uint64_t>((k >> 2) * (Cfg::B_ROWS * BK * 2 >> 4) + (k & 3) * 2);
+            if (CG == 2)
+              tc_mma_f16_pair(d_tmem, ad + ak, bd + bk, idesc, accum);
+            else
+              tc_mma_f16(d_tmem, ad + ak, bd + bk, idesc, accum);
           }
-          tc_commit(&empty[stage]);
+          if (CG == 2)
+            tc_commit_pair_mc(&empty[stage], 0x3);
+          else
+            tc_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(&tfull[acc]);
+        if (CG == 2)
+          tc_commit_pair_mc(&tfull[acc], 0x3);
+        else
+          tc_commit(&tfull[acc]);
       }
       // Every MMA this thread issued has finished before TMEM can be freed.
-      tc_commit(drain);
+      if (CG == 2)
+        tc_commit_pair_mc(drain, 0x1);
+      else
+        tc_commit(drain);
       volatile int never = 0;
       if (!mbar_wait_bounded(drain, 0, &never, limit)) record_error(P.err, abort_flag, kErrMma);
     }
@@ -298,8 +374,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
     uint8_t* stg = sStg + (warp - 2) * STG_PER_WARP;
     int iter = 0;
     uint32_t stores = 0;     // bulk groups this warp has committed (selects the staging buffer)
-    for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++iter) {
-      const TileCoord tc = decode_tile(P, t);
+    for (int t = unit; t < P.total_tiles; t += units, ++iter) {
+      const TileCoord tc = decode_tile<CG>(P, t);
       const GemmProblem& pr = P.prob[tc.p];
       const int acc = iter & 1;
       const uint32_t acc_par = (iter >> 1) & 1;
@@ -311,11 +387,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
       }
       tc_fence_after();
 
-      const int row0 = tc.tm * BM + q * 32;
+      const int row0 = tc.tm * Cfg::TILE_M + static_cast<int>(rank) * BM + q * 32;
       const int row = row0 + lane;
       const bool row_ok = row < pr.M;
       // Mirrored tiles: strictly below the 256 x 256 diagonal blocks.
-      const bool mirror = pr.tri && tc.tm >= 2 * tc.tn + 2;
+      const bool mirror = pr.tri && tc.tm * Cfg::TILE_M >= (tc.tn + 1) * BN;
       float f = pr.f0;
       if (pr.s_pow > 0) {
         const float s = 1.0f / (sqrtf(pr.sumsq[tc.slice]) + pr.eps);
@@ -439,7 +515,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
       if (pr.row_ss != nullptr && row_ok)
         pr.row_ss[(static_cast<long long>(tc.slice) * pr.nt + tc.tn) * pr.M + row] = rss;
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      if (CG == 2)
+        mbar_arrive_leader(&tempty[acc]);
+      else
+        mbar_arrive(&tempty[acc]);
     }
     // Every store has landed before the kernel (and its shared memory) ends.
     if (lane == 0) bulk_wait_group_all();
@@ -448,10 +527,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_c
 
   tc_fence_before();
   __syncthreads();
+  // Neither CTA of a pair leaves while the other may still signal its barriers.
+  if (CG == 2) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (CG == 2)
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
   }
+}
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_constant__ GemmParams P) {
+  ns_gemm_body<1>(P);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+    ns_gemm_pair_kernel(const __grid_constant__ GemmParams P) {
+  ns_gemm_body<2>(P);
 }
 
 }  // namespace muon

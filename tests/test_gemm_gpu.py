@@ -51,15 +51,19 @@ def _check(C, ref, rel_tol=4e-3):
     assert np.max(np.abs(C - ref)) <= 2e-2 * np.max(np.abs(ref)) + 1e-6
 
 
+PAIRS = [1, 2]      # single-CTA 128x256 tiles, 2-CTA (cta_group::2) 256x256 tiles
+
+
+@pytest.mark.parametrize("cta_pair", PAIRS)
 @pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("M,N,K,S", [(300, 520, 200, 2), (128, 256, 64, 1), (77, 40, 33, 3), (513, 300, 520, 1)])
-def test_gemm_majors(mn, a_mn, b_mn, dtype, M, N, K, S):
+def test_gemm_majors(mn, a_mn, b_mn, dtype, M, N, K, S, cta_pair):
     A = _rnd((S, K, M) if a_mn else (S, M, K), dtype, 1)
     B = _rnd((S, K, N) if b_mn else (S, N, K), dtype, 2)
     C = _empty((S, M, N), torch.bfloat16)
     ws = _ws()
-    mn.testing_gemm(A, bool(a_mn), B, bool(b_mn), C, K=K, alpha=0.5, workspace=ws)
+    mn.testing_gemm(A, bool(a_mn), B, bool(b_mn), C, K=K, alpha=0.5, cta_pair=cta_pair, workspace=ws)
     torch.cuda.synchronize()
     assert mn.workspace_error(ws) == 0
     a = _f64(A)
@@ -69,7 +73,8 @@ def test_gemm_majors(mn, a_mn, b_mn, dtype, M, N, K, S):
     _check(C, 0.5 * a @ b)
 
 
-def test_gemm_strided_slices_and_padding(mn):
+@pytest.mark.parametrize("cta_pair", PAIRS)
+def test_gemm_strided_slices_and_padding(mn, cta_pair):
     # Slices with ld > cols and batch stride > rows*ld; padding must stay untouched.
     S, M, N, K = 3, 200, 260, 136
     Abig = _rnd((S, M + 8, K + 24), torch.bfloat16, 3)
@@ -79,7 +84,7 @@ def test_gemm_strided_slices_and_padding(mn):
     Cbig = torch.full((S, M + 5, N + 60), 7.0, dtype=torch.bfloat16, device=DEV)
     C = Cbig[:, :M, :N]
     ws = _ws()
-    mn.testing_gemm(A, False, B, True, C, K=K, workspace=ws)
+    mn.testing_gemm(A, False, B, True, C, K=K, cta_pair=cta_pair, workspace=ws)
     torch.cuda.synchronize()
     _check(C, _f64(A) @ _f64(B))
     rest = _f64(Cbig)
@@ -87,16 +92,17 @@ def test_gemm_strided_slices_and_padding(mn):
     assert np.all(rest == 7.0)
 
 
+@pytest.mark.parametrize("cta_pair", PAIRS)
 @pytest.mark.parametrize("mnmaj", [0, 1])
-@pytest.mark.parametrize("m,n", [(384, 500), (200, 1000), (64, 576), (513, 130)])
-def test_syrk_triangle_mirror(mn, mnmaj, m, n):
+@pytest.mark.parametrize("m,n", [(384, 500), (200, 1000), (64, 576), (513, 130), (1024, 600)])
+def test_syrk_triangle_mirror(mn, mnmaj, m, n, cta_pair):
     S = 2
     X = _rnd((S, n, m) if mnmaj else (S, m, n), torch.bfloat16, 5)
     C = _empty((S, m, m), torch.bfloat16)
     ss = torch.tensor([4.0, 9.0], device=DEV)
     ws = _ws()
     mn.testing_gemm(X, bool(mnmaj), X, bool(mnmaj), C, K=n, tri=True, s_pow=2, sumsq=ss, eps=0.0, f0=3.0,
-                    workspace=ws)
+                    cta_pair=cta_pair, workspace=ws)
     torch.cuda.synchronize()
     x = _f64(X)
     x = np.swapaxes(x, 1, 2) if mnmaj else x
@@ -106,7 +112,8 @@ def test_syrk_triangle_mirror(mn, mnmaj, m, n):
     _check(C, ref)
 
 
-def test_symmetric_epilogue_addend_identity_fp16(mn):
+@pytest.mark.parametrize("cta_pair", PAIRS)
+def test_symmetric_epilogue_addend_identity_fp16(mn, cta_pair):
     # P = a I + (b/k) A + (c/k^2) A A with fp16 A, as the Gram iteration forms it.
     S, m = 2, 300
     X = _rnd((S, m, 2 * m), torch.float32, 6)
@@ -117,14 +124,15 @@ def test_symmetric_epilogue_addend_identity_fp16(mn):
     a, b, c, k = 3.4445, -4.7750, 2.0315, 4.0
     ws = _ws()
     mn.testing_gemm(A, False, A, False, P, K=m, tri=True, D=A, alpha=c / k ** 2, beta=b / k, gamma=a,
-                    workspace=ws)
+                    cta_pair=cta_pair, workspace=ws)
     torch.cuda.synchronize()
     an = _f64(A)
     ref = a * np.eye(m)[None] + (b / k) * an + (c / k ** 2) * an @ an
     _check(P, ref, rel_tol=2e-3)
 
 
-def test_row_sums_of_squares(mn):
+@pytest.mark.parametrize("cta_pair", PAIRS)
+def test_row_sums_of_squares(mn, cta_pair):
     S, M, N, K = 2, 260, 600, 100
     A = _rnd((S, M, K), torch.bfloat16, 7)
     B = _rnd((S, K, N), torch.bfloat16, 8)
@@ -132,7 +140,7 @@ def test_row_sums_of_squares(mn):
     nt = (N + 255) // 256
     rss = torch.full((S, nt, M), float("nan"), device=DEV)
     ws = _ws()
-    mn.testing_gemm(A, False, B, True, C, K=K, row_ss=rss, workspace=ws)
+    mn.testing_gemm(A, False, B, True, C, K=K, row_ss=rss, cta_pair=cta_pair, workspace=ws)
     torch.cuda.synchronize()
     c = _f64(C)
     for t in range(nt):
@@ -140,17 +148,35 @@ def test_row_sums_of_squares(mn):
         assert np.allclose(_f64(rss)[:, t], ref, rtol=1e-5)
 
 
-def test_gemm_deterministic_and_batch_invariant(mn):
+@pytest.mark.parametrize("cta_pair", PAIRS)
+def test_gemm_deterministic_and_batch_invariant(mn, cta_pair):
     M, N, K = 384, 512, 640
     A = _rnd((4, M, K), torch.bfloat16, 9)
     B = _rnd((4, K, N), torch.bfloat16, 10)
     ws = _ws()
     C1 = torch.empty((4, M, N), dtype=torch.bfloat16, device=DEV)
     C2 = torch.empty_like(C1)
-    mn.testing_gemm(A, False, B, True, C1, K=K, workspace=ws)
-    mn.testing_gemm(A, False, B, True, C2, K=K, workspace=ws)
+    mn.testing_gemm(A, False, B, True, C1, K=K, cta_pair=cta_pair, workspace=ws)
+    mn.testing_gemm(A, False, B, True, C2, K=K, cta_pair=cta_pair, workspace=ws)
     C3 = torch.empty((1, M, N), dtype=torch.bfloat16, device=DEV)
-    mn.testing_gemm(A[2:3], False, B[2:3], True, C3, K=K, workspace=ws)
+    mn.testing_gemm(A[2:3], False, B[2:3], True, C3, K=K, cta_pair=cta_pair, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(C1, C2)
     assert torch.equal(C1[2:3], C3)
+
+
+def test_pair_and_single_cta_agree(mn):
+    # Same products, different tile shapes: the accumulation order over K is
+    # the same, so the two kernels produce the same bits.
+    M, N, K = 640, 768, 512
+    A = _rnd((2, M, K), torch.bfloat16, 11)
+    B = _rnd((2, K, N), torch.bfloat16, 12)
+    ws = _ws()
+    C1 = _empty((2, M, N), torch.bfloat16)
+    C2 = _empty((2, M, N), torch.bfloat16)
+    mn.testing_gemm(A, False, B, True, C1, K=K, cta_pair=1, workspace=ws)
+    mn.testing_gemm(A, False, B, True, C2, K=K, cta_pair=2, workspace=ws)
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0
+    _check(C2, _f64(A) @ _f64(B))
+    assert float((C1.float() - C2.float()).abs().max()) <= 2e-2 * float(C1.float().abs().max())
