@@ -93,6 +93,37 @@ def ns_flops(rows, cols, variant, steps):
     return float(3 * m * m * n + prods * m ** 3)
 
 
+TRAFFIC_SOURCES = ("newton_schulz_ns_b200/csrc/ns_gemm.cuh", "newton_schulz_ns_b200/csrc/ptx_sm100.cuh",
+                   "newton_schulz_ns_b200/csrc/muon_api.cu")
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(key, variant):
+    """DRAM bytes of one Newton-Schulz call from the committed ncu summary, or None.
+
+    The summary records the hash of the kernel sources it was captured with;
+    a different hash (the kernel changed since) gives None.
+    """
+    import re
+    path = os.path.join(ROOT, "profiles", f"ns_gemm_{key}_{variant}_traffic.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_ns_call:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
 def default_variant(wl):
     return "gram" if wl.key == "moe" else "standard"
 
@@ -342,7 +373,8 @@ def run_ours(args, wl, variant, rank, world, local_rank):
                      "achieved": round(achieved, 2), "peak": peak_s, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_s, 4), "frac_of_burst": round(achieved / peak_b, 4),
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a long step)",
-                     "traffic": None},
+                     "traffic": measured_traffic(wl.key, variant),
+                     "traffic_unit": "bytes per Newton-Schulz call (ncu dram__bytes_read.sum + write.sum)"},
         "gpu_launches": int(launches),
         "clocks": clk,
     }

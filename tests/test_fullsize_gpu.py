@@ -1,0 +1,100 @@
+"""Full-size parity: the bench's workloads, in the bench's launch configuration.
+
+The whole Llama-8B-shaped step (224 matrices, standard Newton-Schulz) and
+the whole MoE step (128 expert matrices, Gram Newton-Schulz) run exactly as
+bench.py runs them -- one call per stage over every batch -- and a sample of
+matrices is checked against the fp64 oracle one by one: the Newton-Schulz
+output (3e-2 relative Frobenius), the momentum (one bf16 ulp), and NorMuon
+plus the update fed the device's own Newton-Schulz output (1e-5 relative on
+the fp32 variance and the fp32 weight change).  The samples cover every
+orientation (wide, square, tall iterated transposed) and both variants.
+"""
+import numpy as np
+import pytest
+import torch
+
+import bench
+import oracle
+import workloads
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+DEV = "cuda"
+
+
+def f64(t):
+    return t.detach().float().cpu().double().numpy()
+
+
+def h32(x):
+    return float(np.float32(x))
+
+
+def rel(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def _bf16_within_one_ulp(got, want):
+    ulp = np.abs(oracle.bf16_round(np.abs(want) * (1 + 2.0 ** -7)) - oracle.bf16_round(np.abs(want)))
+    ulp = np.maximum(ulp, 2.0 ** -133)
+    assert np.all(np.abs(got - want) <= ulp * 1.0001)
+    assert np.mean(got == want) >= 0.999
+
+
+def _run_full_step(key, variant, samples):
+    import newton_schulz_ns_b200 as mn
+    wl = workloads.WORKLOADS[key]
+    groups, hp, ws = bench.build_state(wl, variant, DEV)
+    # Inputs of the sampled slices, read back before the step mutates them.
+    before = {}
+    for gi, si in samples:
+        b = groups[gi]
+        before[(gi, si)] = dict(G=f64(b.grad[si]), M=f64(b.momentum[si]), W=f64(b.weight[si]),
+                                v=f64(b.variance.view(b.n, b.rows)[si]) if b.variance is not None else None)
+    mn.muon_momentum_norm(groups, hp, ws)
+    (mn.muon_ns_batched if variant == "standard" else mn.muon_gram_ns_batched)(groups, hp, ws)
+    mn.normuon_update(groups, hp, wl.normuon, ws)
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0
+    mstore = "bf16" if wl.mom_dtype == torch.bfloat16 else "f32"
+    for (gi, si), st in before.items():
+        b = groups[gi]
+        g = wl.groups[gi]
+        O = f64(b.ns_out[si])[None]
+        ref = oracle.muon_step_slices(st["G"][None], st["M"][None], st["W"][None],
+                                      st["v"][None] if st["v"] is not None else None,
+                                      mu=h32(wl.momentum), nesterov=wl.nesterov, variant=variant,
+                                      normuon=wl.normuon, beta2=h32(wl.beta2), nor_eps=h32(wl.nor_eps),
+                                      lr=h32(wl.lr), weight_decay=h32(wl.weight_decay),
+                                      lr_scale=h32(b.lr_scale), mom_store=mstore, w_store="f64")
+        err = rel(O[0], ref["O"][0])
+        assert err < 3e-2, (g.name, si, err)
+        _bf16_within_one_ulp(f64(b.momentum[si]), ref["M"][0])
+        # Later stages fed the device's own Newton-Schulz output.
+        ref2 = oracle.muon_step_slices(st["G"][None], st["M"][None], st["W"][None],
+                                       st["v"][None] if st["v"] is not None else None,
+                                       mu=h32(wl.momentum), nesterov=wl.nesterov, normuon=wl.normuon,
+                                       beta2=h32(wl.beta2), nor_eps=h32(wl.nor_eps), lr=h32(wl.lr),
+                                       weight_decay=h32(wl.weight_decay), lr_scale=h32(b.lr_scale),
+                                       mom_store=mstore, w_store="f64", O_override=O)
+        if wl.normuon:
+            assert rel(f64(b.variance.view(b.n, b.rows)[si]), ref2["v"][0]) < 1e-5
+        if wl.weight_dtype == torch.float32:
+            dW = f64(b.weight[si]) - st["W"]
+            assert rel(dW, ref2["W"][0] - st["W"]) < 1e-5
+            if b.weight_copy is not None:
+                _bf16_within_one_ulp(f64(b.weight_copy[si]), oracle.bf16_round(oracle.fp32_round(ref2["W"][0])))
+        else:
+            _bf16_within_one_ulp(f64(b.weight[si]), oracle.bf16_round(ref2["W"][0]))
+    del groups, ws
+    torch.cuda.empty_cache()
+
+
+def test_llama8b_full_step_standard_sampled():
+    # (group, slice): k_proj layer 0 (wide), q_proj layer 5 (square),
+    # gate_proj layer 17 (tall, iterated transposed), down_proj layer 31 (wide).
+    _run_full_step("llama8b", "standard", [(1, 0), (0, 5), (4, 17), (6, 31)])
+
+
+def test_moe_full_step_gram_sampled():
+    # w1 of experts 0 and 37 (wide), w2 of experts 5 and 63 (tall).
+    _run_full_step("moe", "gram", [(0, 0), (0, 37), (1, 5), (1, 63)])
