@@ -247,6 +247,23 @@ class Clocks:
                 "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
 
 
+# ----------------------------------------------------------------------------- replicas
+
+def max_over_ranks(values, device):
+    """Element-wise maximum of a list of floats over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def replica_throughput(work_per_rank, world, seconds_max, scale=1e12):
+    """Whole-job rate of `world` independent replicas timed by the slowest one."""
+    return world * work_per_rank / seconds_max / scale
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args, wl, variant, rank, world, local_rank):
@@ -343,17 +360,13 @@ def run_ours(args, wl, variant, rank, world, local_rank):
         e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
 
     # ---- max over ranks
-    vals = torch.tensor([ms_total, statistics.mean(ns_ms), e2e["ms"] if e2e else 0.0], device=dev,
-                        dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms_total, ns_mean, e2e_ms = (float(x) for x in vals.tolist())
+    ms_total, ns_mean, e2e_ms = max_over_ranks([ms_total, statistics.mean(ns_ms), e2e["ms"] if e2e else 0.0], dev)
     if rank != 0:
         return None
 
     peaks, src = load_peaks()
     sec = ms_total / 1e3
-    value = world * ns_flop * args.steps / sec / 1e12
+    value = replica_throughput(ns_flop * args.steps, world, sec)
     ms_step = ms_total / args.steps
     achieved = ns_flop / (ns_mean / 1e3) / 1e12          # per NS call, averaged over the timed steps
     peak_s = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
@@ -381,7 +394,8 @@ def run_ours(args, wl, variant, rank, world, local_rank):
     if e2e_skip:
         out["e2e"] = {"value": None, "unit": "TFLOP/s", "skipped": e2e_skip}
     if e2e:
-        out["e2e"] = {"value": round(world * ns_flop * args.steps / (e2e_ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
+        out["e2e"] = {"value": round(replica_throughput(ns_flop * args.steps, world, e2e_ms / 1e3), 3),
+                      "unit": "TFLOP/s",
                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                       "ms_per_step": round(e2e_ms / args.steps, 3),
                       "path": "public C-ABI calls; gradients copied H2D from pinned host memory and the per-slice "
