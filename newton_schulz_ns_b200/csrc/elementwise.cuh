@@ -148,24 +148,47 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_chunks_kernel(const __gri
     const long long e1 = min(e0 + CHUNK, total);
     float acc = 0.0f;
     if (S.vec8) {
-      for (long long e = e0 + threadIdx.x * 8; e < e1; e += EW_THREADS * 8) {
-        const long long r = e / S.cols, col = e - r * S.cols;
+      // Every load of this thread's part of the chunk is issued before any
+      // store, so a chunk keeps VPT 16-byte loads per operand in flight.
+      constexpr int VPT = CHUNK / (EW_THREADS * 8);
+      long long off_g[VPT], off_m[VPT], off_u[VPT];
+      bool live[VPT];
+      float g[VPT][8], m[VPT][8];
+#pragma unroll
+      for (int it = 0; it < VPT; ++it) {
+        const long long e = e0 + (static_cast<long long>(it) * EW_THREADS + threadIdx.x) * 8;
+        live[it] = e < e1;
+        const long long r = live[it] ? e / S.cols : 0, col = live[it] ? e - r * S.cols : 0;
+        off_g[it] = slice * S.g_bs + r * S.g_ld + col;
+        off_m[it] = slice * S.m_bs + r * S.m_ld + col;
+        off_u[it] = slice * S.u_bs + r * S.u_ld + col;
+        if (live[it]) {
+          if (MODE == 0) {
+            ld8(S.g, off_g[it], S.g_dt, g[it]);
+            ld8(S.m, off_m[it], S.m_dt, m[it]);
+          } else {
+            ld8(S.u, off_u[it], 1, g[it]);
+          }
+        }
+      }
+#pragma unroll
+      for (int it = 0; it < VPT; ++it) {
+        if (!live[it]) continue;
         float u[8];
         if (MODE == 0) {
-          float g[8], m[8];
-          ld8(S.g, slice * S.g_bs + r * S.g_ld + col, S.g_dt, g);
-          ld8(S.m, slice * S.m_bs + r * S.m_ld + col, S.m_dt, m);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) m[i] = P.mu * m[i] + g[i];
           float mn[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mn[i] = m[i];
-          st8(S.m, slice * S.m_bs + r * S.m_ld + col, S.m_dt, m);   // m now holds the stored values
+          for (int i = 0; i < 8; ++i) {
+            mn[i] = P.mu * m[it][i] + g[it][i];
+            m[it][i] = mn[i];
+          }
+          st8(S.m, off_m[it], S.m_dt, m[it]);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) u[i] = P.nesterov ? g[i] + P.mu * mn[i] : mn[i];
-          st8(S.u, slice * S.u_bs + r * S.u_ld + col, 1, u);         // u now holds bf16(U)
+          for (int i = 0; i < 8; ++i) u[i] = P.nesterov ? g[it][i] + P.mu * mn[i] : mn[i];
+          st8(S.u, off_u[it], 1, u);                 // u now holds bf16(U)
         } else {
-          ld8(S.u, slice * S.u_bs + r * S.u_ld + col, 1, u);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) u[i] = g[it][i];
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc += u[i] * u[i];

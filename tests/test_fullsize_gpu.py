@@ -33,10 +33,22 @@ def rel(a, b):
     return float(np.linalg.norm(a - b) / np.linalg.norm(b))
 
 
-def _bf16_within_one_ulp(got, want):
+def _bf16_within_one_ulp(got, want, terms=None):
+    """At most one bf16 ulp from the oracle, >= 99.9% identical.
+
+    ``terms``: magnitude of the quantities the device adds in float32 to form
+    the value; where they nearly cancel, their float32 rounding (a few 2^-24
+    of each) may exceed the bf16 ulp of the small result, and that much more
+    is allowed.
+    """
     ulp = np.abs(oracle.bf16_round(np.abs(want) * (1 + 2.0 ** -7)) - oracle.bf16_round(np.abs(want)))
     ulp = np.maximum(ulp, 2.0 ** -133)
-    assert np.all(np.abs(got - want) <= ulp * 1.0001)
+    slack = 0.0 if terms is None else 4 * 2.0 ** -24 * terms
+    bad = np.abs(got - want) > ulp * 1.0001 + slack
+    if np.any(bad):
+        i = np.flatnonzero(bad)[:5]
+        raise AssertionError(f"{int(bad.sum())} elements beyond one ulp: got {got.flat[i]}, want {want.flat[i]}, "
+                             f"ulp {ulp.flat[i]}, terms {None if terms is None else terms.flat[i]}")
     assert np.mean(got == want) >= 0.999
 
 
@@ -81,10 +93,13 @@ def _run_full_step(key, variant, samples):
         if wl.weight_dtype == torch.float32:
             dW = f64(b.weight[si]) - st["W"]
             assert rel(dW, ref2["W"][0] - st["W"]) < 1e-5
+            terms = np.abs(st["W"]) + np.abs(ref2["W"][0] - st["W"])
             if b.weight_copy is not None:
-                _bf16_within_one_ulp(f64(b.weight_copy[si]), oracle.bf16_round(oracle.fp32_round(ref2["W"][0])))
+                _bf16_within_one_ulp(f64(b.weight_copy[si]), oracle.bf16_round(oracle.fp32_round(ref2["W"][0])),
+                                     terms)
         else:
-            _bf16_within_one_ulp(f64(b.weight[si]), oracle.bf16_round(ref2["W"][0]))
+            terms = np.abs(st["W"]) + np.abs(ref2["W"][0] - st["W"])
+            _bf16_within_one_ulp(f64(b.weight[si]), oracle.bf16_round(ref2["W"][0]), terms)
     del groups, ws
     torch.cuda.empty_cache()
 

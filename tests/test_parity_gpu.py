@@ -246,7 +246,7 @@ def test_momentum_norm(mn, gdt, mdt, shape, nesterov):
         assert abs(float(ss[i]) / np.sum(Ug[i] ** 2) - 1) < 1e-5
 
 
-def _bf16_close(got, want, exact_frac=0.9999):
+def _bf16_close(got, want, exact_frac=0.9999, terms=None):
     """<= 1 bf16 ulp everywhere and >= exact_frac identical (at least 2 differing elements allowed).
 
     fp32 arithmetic on the device and fp64 in the oracle round the same
@@ -255,8 +255,11 @@ def _bf16_close(got, want, exact_frac=0.9999):
     """
     ulp = np.abs(oracle.bf16_round(np.abs(want) * (1 + 2.0 ** -7)) - oracle.bf16_round(np.abs(want)))
     ulp = np.maximum(ulp, 2.0 ** -133)                      # smallest bf16 subnormal
+    # terms: magnitude of the float32 quantities summed to form the value;
+    # where they cancel, their float32 rounding may exceed a bf16 ulp.
+    slack = 0.0 if terms is None else 4 * 2.0 ** -24 * terms
     diff = np.abs(got - want)
-    assert np.all(diff <= ulp * 1.0001), float(np.max(diff / ulp))
+    assert np.all(diff <= ulp * 1.0001 + slack), float(np.max(diff / ulp))
     flips = int(np.sum(diff != 0))
     assert flips <= max(2, int((1 - exact_frac) * diff.size)), (flips, diff.size)
 
@@ -292,9 +295,10 @@ def test_update_fed_same_ns_output(mn, wdt, copy, normuon, shape):
         dW = f64(W) - f64(W0)
         assert rel(dW, ref["W"] - f64(W0)) < 1e-5
         if copy:
-            _bf16_close(f64(Wc), oracle.bf16_round(oracle.fp32_round(ref["W"])))
+            _bf16_close(f64(Wc), oracle.bf16_round(oracle.fp32_round(ref["W"])),
+                        terms=np.abs(f64(W0)) + np.abs(ref["W"] - f64(W0)))
     else:
-        _bf16_close(f64(W), oracle.bf16_round(ref["W"]))
+        _bf16_close(f64(W), oracle.bf16_round(ref["W"]), terms=np.abs(f64(W0)) + np.abs(ref["W"] - f64(W0)))
 
 
 # ----------------------------------------------------------------- whole step
