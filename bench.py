@@ -61,7 +61,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama8b", choices=sorted(DESCRIPTIONS))
-    ap.add_argument("--variant", choices=["standard", "gram"], default=None)
+    ap.add_argument("--variant", choices=["standard", "gram", "auto"], default=None,
+                    help="auto: Gram form for slices with n >= 1.25 m, standard otherwise")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scale-down", type=int, default=1, help="divide every parameter count (smoke runs only)")
@@ -77,6 +78,16 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+AUTO_GRAM_RATIO = 1.25
+
+
+def slice_variant(rows, cols, variant):
+    if variant != "auto":
+        return variant
+    m, n = min(rows, cols), max(rows, cols)
+    return "gram" if n > m and n >= AUTO_GRAM_RATIO * m else "standard"
+
+
 def ns_flops(rows, cols, variant, steps):
     """Work of one slice's orthogonalization, as the metric counts it (m = short side, n = long side).
 
@@ -87,6 +98,7 @@ def ns_flops(rows, cols, variant, steps):
     Both arms of the benchmark count the same work for the same variant.
     """
     m, n = min(rows, cols), max(rows, cols)
+    variant = slice_variant(rows, cols, variant)
     if variant == "standard":
         return float(steps * (3 * m * m * n + m ** 3))
     prods = sum(1 + (k > 0) + 2 * (k < steps - 1) for k in range(steps))
@@ -154,7 +166,8 @@ def oracle_sample(wl, variant, budget_s=30.0):
                 M = np.zeros_like(G)
                 v = np.zeros(G.shape[:2]) if wl.normuon else None
                 oracle.muon_step_slices(G, M, W, v, mu=wl.momentum, nesterov=wl.nesterov, ns_eps=wl.ns_eps,
-                                        ns_steps=wl.ns_steps, variant=variant, normuon=wl.normuon,
+                                        ns_steps=wl.ns_steps, variant=slice_variant(g.slice_rows, g.cols, variant),
+                                        normuon=wl.normuon,
                                         beta2=wl.beta2, nor_eps=wl.nor_eps, lr=wl.lr,
                                         weight_decay=wl.weight_decay,
                                         lr_scale=math.sqrt(max(1.0, g.rows / g.cols)))
@@ -247,6 +260,24 @@ class Clocks:
                 "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
 
 
+def momentum_bytes(groups):
+    """Algorithmic bytes of muon_momentum_norm: read G, M; write M, U (bf16)."""
+    tot = 0
+    for b in groups:
+        e = b.n * b.rows * b.cols
+        tot += e * (b.grad.element_size() + 2 * b.momentum.element_size() + 2)
+    return tot
+
+
+def update_bytes(groups, normuon):
+    """Algorithmic bytes of normuon_update: read O (twice with NorMuon: row sums, update), W; write W, copy."""
+    tot = 0
+    for b in groups:
+        e = b.n * b.rows * b.cols
+        tot += e * ((4 if normuon else 2) + 2 * b.weight.element_size() + (2 if b.weight_copy is not None else 0))
+    return tot
+
+
 # ----------------------------------------------------------------------------- replicas
 
 def max_over_ranks(values, device):
@@ -274,20 +305,28 @@ def run_ours(args, wl, variant, rank, world, local_rank):
     dev = f"cuda:{local_rank}"
     torch.cuda.set_device(dev)
     groups, hp, ws = build_state(wl, variant, dev)
-    ns_fn = mn.muon_ns_batched if variant == "standard" else mn.muon_gram_ns_batched
+    if variant == "auto":
+        def ns_fn(g, h, w, s):
+            mn.muon_ns_auto_batched(g, h, w, AUTO_GRAM_RATIO, s)
+    else:
+        ns_fn = mn.muon_ns_batched if variant == "standard" else mn.muon_gram_ns_batched
     stream = torch.cuda.current_stream()
 
     ns_flop = sum(b.n * ns_flops(b.rows, b.cols, variant, wl.ns_steps) for b in groups)
     slices = sum(b.n for b in groups)
 
     def step(ev=None):
-        mn.muon_momentum_norm(groups, hp, ws, stream)
         if ev is not None:
             ev[0].record(stream)
-        ns_fn(groups, hp, ws, stream)
+        mn.muon_momentum_norm(groups, hp, ws, stream)
         if ev is not None:
             ev[1].record(stream)
+        ns_fn(groups, hp, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
         mn.normuon_update(groups, hp, wl.normuon, ws, stream)
+        if ev is not None:
+            ev[3].record(stream)
 
     def barrier():
         if world > 1:
@@ -301,8 +340,7 @@ def run_ours(args, wl, variant, rank, world, local_rank):
     # ---- device-resident timing
     gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[local_rank] \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else str(local_rank)
-    ns_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in range(args.steps)]
+    ns_events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
@@ -317,7 +355,9 @@ def run_ours(args, wl, variant, rank, world, local_rank):
     clk = clocks.stop()
     barrier()
     ms_total = start.elapsed_time(end)
-    ns_ms = [a.elapsed_time(b) for a, b in ns_events]
+    ns_ms = [e[1].elapsed_time(e[2]) for e in ns_events]
+    mom_ms = [e[0].elapsed_time(e[1]) for e in ns_events]
+    upd_ms = [e[2].elapsed_time(e[3]) for e in ns_events]
     assert mn.workspace_error(ws) == 0, "device-side wait timed out"
 
     # ---- end to end: gradients H2D from pinned host memory, step, result D2H
@@ -360,7 +400,9 @@ def run_ours(args, wl, variant, rank, world, local_rank):
         e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
 
     # ---- max over ranks
-    ms_total, ns_mean, e2e_ms = max_over_ranks([ms_total, statistics.mean(ns_ms), e2e["ms"] if e2e else 0.0], dev)
+    ms_total, ns_mean, mom_mean, upd_mean, e2e_ms = max_over_ranks(
+        [ms_total, statistics.mean(ns_ms), statistics.mean(mom_ms), statistics.mean(upd_ms),
+         e2e["ms"] if e2e else 0.0], dev)
     if rank != 0:
         return None
 
@@ -381,7 +423,11 @@ def run_ours(args, wl, variant, rank, world, local_rank):
         "pct_bf16_peak": round(100 * value / world / peak_s, 2),
         "pct_bf16_peak_burst": round(100 * value / world / peak_b, 2),
         "matrices_per_s": round(world * slices * args.steps / sec, 2),
-        "ms_breakdown": {"ns": round(ns_mean, 3), "momentum_and_update": round(ms_step - ns_mean, 3)},
+        "ms_breakdown": {"momentum_norm": round(mom_mean, 3), "ns": round(ns_mean, 3),
+                         "normuon_update": round(upd_mean, 3)},
+        "hbm_kernels": {"momentum_gbs": round(momentum_bytes(groups) / (mom_mean / 1e3) / 1e9, 1),
+                        "update_gbs": round(update_bytes(groups, wl.normuon) / (upd_mean / 1e3) / 1e9, 1),
+                        "peak_gbs": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])},
         "roofline": {"bound": "tensor", "kernel": "ns_gemm_kernel (all launches of one Newton-Schulz call)",
                      "achieved": round(achieved, 2), "peak": peak_s, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_s, 4), "frac_of_burst": round(achieved / peak_b, 4),

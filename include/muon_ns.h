@@ -169,6 +169,21 @@ MUON_API muon_status muon_gram_ns_batched(const muon_batch* batches, int nb, con
                                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Newton-Schulz with the form chosen per batch: the Gram form for slices whose
+ * long side exceeds the short side by at least `gram_min_ratio` (n >= ratio*m),
+ * the standard form otherwise.  By operation count the Gram form
+ * (3m^2 n + 17m^3 with one-triangle products) is cheaper than the standard
+ * form (5(3m^2 n + m^3)) exactly when n > m; square slices stay standard, the
+ * form that keeps rank-deficient inputs in band.  gram_min_ratio <= 1 picks
+ * the Gram form for every non-square slice; both forms compute the same map
+ * ([ds-8437] "Measurement": the Gram and standard kernels agree).
+ * Workspace: max of muon_workspace_size for which = 1 and 2.
+ */
+MUON_API muon_status muon_ns_auto_batched(const muon_batch* batches, int nb, const muon_hparams* hp,
+                                          float gram_min_ratio, void* workspace, size_t workspace_bytes,
+                                          cudaStream_t stream);
+
+/*
  * NorMuon normalization and the weight update.
  * [dion-121] follow-on "What it does": one variance per output channel,
  * over the last dim of the flattened [N, out, prod(rest)] view;

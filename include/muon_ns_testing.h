@@ -41,6 +41,17 @@ MUON_API muon_status muon_testing_gemm(int M, int N, int K, int slices, int tri,
                               int cta_pair, int raster_group, void* workspace,
                               size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Failure-path hook: one thread waits, with the GEMM kernel's bounded wait,
+ * on an mbarrier that nothing ever arrives on.  After `limit_ns` of global
+ * time the wait gives up, the kernel writes MUON_TESTING_WAIT_TIMEOUT at
+ * workspace offset 0 and returns; the context stays usable.  Workspace:
+ * >= 256 bytes, 256-byte aligned, device memory.
+ */
+#define MUON_TESTING_WAIT_TIMEOUT 4
+MUON_API muon_status muon_testing_bounded_wait(uint64_t limit_ns, void* workspace, size_t workspace_bytes,
+                                               cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,7 +20,7 @@ from ._capi import MUON_BF16, MUON_F16, MUON_F32, MuonError  # noqa: F401
 
 __all__ = ["Batch", "Hparams", "muon_workspace_size", "muon_momentum_norm", "muon_ns_batched",
            "muon_gram_ns_batched", "normuon_update", "workspace_error", "testing_gemm", "spectral_scale",
-           "ns_flops", "version", "kernel_launches", "muon_momentum_norm_noalloc", "allocate_workspace", "MuonError", "LIB_PATH"]
+           "ns_flops", "version", "kernel_launches", "muon_momentum_norm_noalloc", "muon_ns_auto_batched", "allocate_workspace", "MuonError", "LIB_PATH"]
 
 LIB_PATH = _capi.LIB_PATH
 
@@ -212,6 +212,16 @@ def muon_gram_ns_batched(batches: Sequence[Batch], hp: Hparams, workspace: torch
     p, nbytes = _ws(workspace)
     _capi.check(_capi.lib.muon_gram_ns_batched(arr, nb, ctypes.byref(h), p, nbytes, _stream_ptr(stream)),
                 "muon_gram_ns_batched")
+
+
+def muon_ns_auto_batched(batches: Sequence[Batch], hp: Hparams, workspace: torch.Tensor, gram_min_ratio: float = 1.25,
+                         stream=None) -> None:
+    """Newton-Schulz with the Gram form for slices with n >= gram_min_ratio * m, standard otherwise."""
+    arr, nb = _batches(batches)
+    h, _keep = hp.to_c()
+    p, nbytes = _ws(workspace)
+    _capi.check(_capi.lib.muon_ns_auto_batched(arr, nb, ctypes.byref(h), float(gram_min_ratio), p, nbytes,
+                                               _stream_ptr(stream)), "muon_ns_auto_batched")
 
 
 def normuon_update(batches: Sequence[Batch], hp: Hparams, use_normuon: bool, workspace: torch.Tensor,

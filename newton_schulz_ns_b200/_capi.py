@@ -49,7 +49,8 @@ class MuonHparams(ctypes.Structure):
 
 EXPORTS = ("muon_workspace_size", "muon_momentum_norm", "muon_ns_batched", "muon_gram_ns_batched",
            "normuon_update", "muon_workspace_error", "muon_status_string", "muon_version",
-           "muon_testing_gemm", "muon_kernel_launches", "muon_momentum_norm_noalloc")
+           "muon_testing_gemm", "muon_kernel_launches", "muon_momentum_norm_noalloc",
+           "muon_testing_bounded_wait", "muon_ns_auto_batched")
 
 
 def _load() -> ctypes.CDLL:
@@ -71,6 +72,8 @@ def _load() -> ctypes.CDLL:
         fn.restype = ctypes.c_int
     lib.muon_momentum_norm_noalloc.argtypes = [B, ctypes.c_int, H, P]
     lib.muon_momentum_norm_noalloc.restype = ctypes.c_int
+    lib.muon_ns_auto_batched.argtypes = [B, ctypes.c_int, H, ctypes.c_float, P, ctypes.c_size_t, P]
+    lib.muon_ns_auto_batched.restype = ctypes.c_int
     lib.normuon_update.argtypes = [B, ctypes.c_int, H, ctypes.c_int, P, ctypes.c_size_t, P]
     lib.normuon_update.restype = ctypes.c_int
     lib.muon_workspace_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
@@ -87,6 +90,8 @@ def _load() -> ctypes.CDLL:
                                       P, i64, i64, i32, f32, f32, f32, f32, i32, P, f32, P, i32, i32,
                                       P, ctypes.c_size_t, P]
     lib.muon_testing_gemm.restype = ctypes.c_int
+    lib.muon_testing_bounded_wait.argtypes = [ctypes.c_uint64, P, ctypes.c_size_t, P]
+    lib.muon_testing_bounded_wait.restype = ctypes.c_int
     return lib
 
 

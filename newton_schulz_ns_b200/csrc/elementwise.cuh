@@ -27,6 +27,7 @@ struct EwSeg {
   long long slice_begin;          // first global slice of this segment (for per-slice arrays)
   long long row_begin;            // first global row of this segment (for per-row arrays)
   int vec8;                       // 1: cols, strides and pointers allow 8-wide vectors
+  int flat;                       // 1: every tensor the kernel touches is one dense [n*rows*cols] array
   // tensors: (ptr, ld, batch stride, dtype: 0 f32, 1 bf16)
   const void* g; long long g_ld, g_bs; int g_dt;
   void* m; long long m_ld, m_bs; int m_dt;
@@ -87,8 +88,9 @@ __device__ __forceinline__ void ld8(const void* p, long long off, int dt, float 
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __bfloat162float(__ushort_as_bfloat16(static_cast<uint16_t>(w[i] & 0xFFFFu)));
-      v[2 * i + 1] = __bfloat162float(__ushort_as_bfloat16(static_cast<uint16_t>(w[i] >> 16)));
+      // bf16 -> f32 is a 16-bit shift of the bit pattern.
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
   }
 }
@@ -103,10 +105,10 @@ __device__ __forceinline__ void st8(void* p, long long off, int dt, float (&v)[8
     uint32_t w[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      __nv_bfloat16 lo = __float2bfloat16_rn(v[2 * i]), hi = __float2bfloat16_rn(v[2 * i + 1]);
-      v[2 * i] = __bfloat162float(lo);
-      v[2 * i + 1] = __bfloat162float(hi);
-      w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);   // .x = low half
+      w[i] = *reinterpret_cast<const uint32_t*>(&h);
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
     *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p) + off) = make_uint4(w[0], w[1], w[2], w[3]);
   }
@@ -148,47 +150,34 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_chunks_kernel(const __gri
     const long long e1 = min(e0 + CHUNK, total);
     float acc = 0.0f;
     if (S.vec8) {
-      // Every load of this thread's part of the chunk is issued before any
-      // store, so a chunk keeps VPT 16-byte loads per operand in flight.
-      constexpr int VPT = CHUNK / (EW_THREADS * 8);
-      long long off_g[VPT], off_m[VPT], off_u[VPT];
-      bool live[VPT];
-      float g[VPT][8], m[VPT][8];
-#pragma unroll
-      for (int it = 0; it < VPT; ++it) {
-        const long long e = e0 + (static_cast<long long>(it) * EW_THREADS + threadIdx.x) * 8;
-        live[it] = e < e1;
-        const long long r = live[it] ? e / S.cols : 0, col = live[it] ? e - r * S.cols : 0;
-        off_g[it] = slice * S.g_bs + r * S.g_ld + col;
-        off_m[it] = slice * S.m_bs + r * S.m_ld + col;
-        off_u[it] = slice * S.u_bs + r * S.u_ld + col;
-        if (live[it]) {
-          if (MODE == 0) {
-            ld8(S.g, off_g[it], S.g_dt, g[it]);
-            ld8(S.m, off_m[it], S.m_dt, m[it]);
-          } else {
-            ld8(S.u, off_u[it], 1, g[it]);
-          }
+      const long long flat0 = slice * S.rows * S.cols;
+      for (long long e = e0 + threadIdx.x * 8; e < e1; e += EW_THREADS * 8) {
+        // Dense slices need no row/column split (a 64-bit division per vector).
+        long long og, om, ou;
+        if (S.flat) {
+          og = om = ou = flat0 + e;
+        } else {
+          const long long r = e / S.cols, col = e - r * S.cols;
+          og = slice * S.g_bs + r * S.g_ld + col;
+          om = slice * S.m_bs + r * S.m_ld + col;
+          ou = slice * S.u_bs + r * S.u_ld + col;
         }
-      }
-#pragma unroll
-      for (int it = 0; it < VPT; ++it) {
-        if (!live[it]) continue;
         float u[8];
         if (MODE == 0) {
+          float g[8], m[8];
+          ld8(S.g, og, S.g_dt, g);
+          ld8(S.m, om, S.m_dt, m);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m[i] = P.mu * m[i] + g[i];
           float mn[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            mn[i] = P.mu * m[it][i] + g[it][i];
-            m[it][i] = mn[i];
-          }
-          st8(S.m, off_m[it], S.m_dt, m[it]);
+          for (int i = 0; i < 8; ++i) mn[i] = m[i];
+          st8(S.m, om, S.m_dt, m);                                  // m now holds the stored values
 #pragma unroll
-          for (int i = 0; i < 8; ++i) u[i] = P.nesterov ? g[it][i] + P.mu * mn[i] : mn[i];
-          st8(S.u, off_u[it], 1, u);                 // u now holds bf16(U)
+          for (int i = 0; i < 8; ++i) u[i] = P.nesterov ? g[i] + P.mu * mn[i] : mn[i];
+          st8(S.u, ou, 1, u);                                       // u now holds bf16(U)
         } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) u[i] = g[it][i];
+          ld8(S.u, ou, 1, u);
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc += u[i] * u[i];
@@ -316,16 +305,33 @@ __global__ void __launch_bounds__(EW_THREADS) update_kernel(const __grid_constan
     const float base = P.lr * S.lr_scale * (P.use_normuon ? P.slice_factor[S.slice_begin + slice] : 1.0f);
     const float* rowd = P.use_normuon ? P.row_d + S.row_begin + slice * S.rows : nullptr;
     if (S.vec8) {
+      const long long flat0 = slice * S.rows * S.cols;
+      // The row of element e changes at most once per 8 consecutive elements
+      // (cols is a multiple of 8), so track it instead of dividing.
+      long long r = (e0 + threadIdx.x * 8) / S.cols;
+      long long rstart = r * S.cols;
       for (long long e = e0 + threadIdx.x * 8; e < e1; e += EW_THREADS * 8) {
-        const long long r = e / S.cols, col = e - r * S.cols;
+        while (e >= rstart + S.cols) {
+          rstart += S.cols;
+          ++r;
+        }
+        const long long col = e - rstart;
         const float coef = rowd ? base * rowd[r] : base;
+        long long oo, ow, oc;
+        if (S.flat) {
+          oo = ow = oc = flat0 + e;
+        } else {
+          oo = slice * S.o_bs + r * S.o_ld + col;
+          ow = slice * S.w_bs + r * S.w_ld + col;
+          oc = slice * S.wc_bs + r * S.wc_ld + col;
+        }
         float o[8], w[8];
-        ld8(S.o, slice * S.o_bs + r * S.o_ld + col, 1, o);
-        ld8(S.w, slice * S.w_bs + r * S.w_ld + col, S.w_dt, w);
+        ld8(S.o, oo, 1, o);
+        ld8(S.w, ow, S.w_dt, w);
 #pragma unroll
         for (int i = 0; i < 8; ++i) w[i] = fmaf(-coef, o[i], w[i] * keep);
-        st8(S.w, slice * S.w_bs + r * S.w_ld + col, S.w_dt, w);
-        if (S.wc) st8(S.wc, slice * S.wc_bs + r * S.wc_ld + col, 1, w);
+        st8(S.w, ow, S.w_dt, w);
+        if (S.wc) st8(S.wc, oc, 1, w);
       }
     } else {
       for (long long e = e0 + threadIdx.x; e < e1; e += EW_THREADS) {

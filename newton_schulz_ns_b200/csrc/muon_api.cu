@@ -140,6 +140,15 @@ muon_status check_view(const muon_batch& b, const muon_view& v, std::initializer
   return MUON_OK;
 }
 
+// Every given view is one dense [n][rows][cols] array (rows ld = cols apart, slices rows*cols apart).
+bool flat_ok(const muon_batch& b, std::initializer_list<const muon_view*> views) {
+  for (const muon_view* v : views) {
+    if (v->ptr == nullptr) continue;
+    if (v->ld != b.cols || (b.n > 1 && v->batch_stride != b.rows * b.cols)) return false;
+  }
+  return true;
+}
+
 bool vec8_ok(const muon_batch& b, std::initializer_list<const muon_view*> views) {
   if (b.cols % 8) return false;
   for (const muon_view* v : views) {
@@ -483,6 +492,7 @@ muon_status launch_norm(const muon_batch* bs, int nb, const muon_hparams* hp, in
       S.u_ld = b.ns_in.ld;
       S.u_bs = b.ns_in.batch_stride;
       S.vec8 = mode == 0 ? vec8_ok(b, {&b.grad, &b.momentum, &b.ns_in}) : vec8_ok(b, {&b.ns_in});
+      S.flat = mode == 0 ? flat_ok(b, {&b.grad, &b.momentum, &b.ns_in}) : flat_ok(b, {&b.ns_in});
       P.sumsq_out[ns] = b.sumsq;
       ++ns;
     }
@@ -645,8 +655,8 @@ muon_status validate_ns(const muon_batch* bs, int nb, const muon_hparams* hp) {
 // Clears the error word and makes sure every batch has a per-slice sum of squares.
 // Returns the per-batch sumsq pointers to use.
 muon_status prepare_norms(const muon_batch* bs, int nb, const Layout& L, uint8_t* ws, int sms, cudaStream_t stream,
-                          std::vector<const float*>& sumsq) {
-  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), stream) != cudaSuccess) return MUON_CUDA_ERROR;
+                          std::vector<const float*>& sumsq, bool clear_err = true) {
+  if (clear_err && cudaMemsetAsync(ws, 0, sizeof(int32_t), stream) != cudaSuccess) return MUON_CUDA_ERROR;
   sumsq.assign(nb, nullptr);
   std::vector<muon_batch> missing;
   float* base = reinterpret_cast<float*>(ws + L.sumsq);
@@ -794,8 +804,25 @@ muon_status muon_momentum_norm_noalloc(const muon_batch* batches, int nb, const 
   return launch_norm(batches, nb, hp, 0, scratch, scratch, sms, stream);
 }
 
+muon_status ns_standard_impl(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream, bool clear_err);
+muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream, bool clear_err);
+
 muon_status muon_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
                             size_t workspace_bytes, cudaStream_t stream) {
+  return ns_standard_impl(batches, nb, hp, workspace, workspace_bytes, stream, true);
+}
+
+muon_status muon_gram_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+  return ns_gram_impl(batches, nb, hp, workspace, workspace_bytes, stream, true);
+}
+
+}  // extern "C"
+
+muon_status ns_standard_impl(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream, bool clear_err) {
   muon_status st = validate_ns(batches, nb, hp);
   if (st != MUON_OK) return st;
   bool any = false;
@@ -807,7 +834,7 @@ muon_status muon_ns_batched(const muon_batch* batches, int nb, const muon_hparam
   if ((st = device_setup(&sms)) != MUON_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   std::vector<const float*> sumsq;
-  if ((st = prepare_norms(batches, nb, L, ws, sms, stream, sumsq)) != MUON_OK) return st;
+  if ((st = prepare_norms(batches, nb, L, ws, sms, stream, sumsq, clear_err)) != MUON_OK) return st;
   int* err = reinterpret_cast<int*>(ws);
 
   const int S = hp->ns_steps;
@@ -843,8 +870,8 @@ muon_status muon_ns_batched(const muon_batch* batches, int nb, const muon_hparam
   return MUON_OK;
 }
 
-muon_status muon_gram_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
-                                 size_t workspace_bytes, cudaStream_t stream) {
+muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream, bool clear_err) {
   muon_status st = validate_ns(batches, nb, hp);
   if (st != MUON_OK) return st;
   bool any = false;
@@ -856,7 +883,7 @@ muon_status muon_gram_ns_batched(const muon_batch* batches, int nb, const muon_h
   if ((st = device_setup(&sms)) != MUON_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   std::vector<const float*> sumsq;
-  if ((st = prepare_norms(batches, nb, L, ws, sms, stream, sumsq)) != MUON_OK) return st;
+  if ((st = prepare_norms(batches, nb, L, ws, sms, stream, sumsq, clear_err)) != MUON_OK) return st;
   int* err = reinterpret_cast<int*>(ws);
   const int S = hp->ns_steps;
   const float kap = kGramScale;
@@ -926,6 +953,36 @@ muon_status muon_gram_ns_batched(const muon_batch* batches, int nb, const muon_h
   return MUON_OK;
 }
 
+extern "C" {
+
+muon_status muon_ns_auto_batched(const muon_batch* batches, int nb, const muon_hparams* hp, float gram_min_ratio,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  muon_status st = validate_ns(batches, nb, hp);
+  if (st != MUON_OK) return st;
+  if (!std::isfinite(gram_min_ratio)) return MUON_INVALID_ARG;
+  std::vector<muon_batch> std_b, gram_b;
+  for (int i = 0; i < nb; ++i) {
+    const muon_batch& b = batches[i];
+    if (batch_empty(b)) continue;
+    const int64_t m = std::min(b.rows, b.cols), n = std::max(b.rows, b.cols);
+    const bool gram = n > m && static_cast<double>(n) >= static_cast<double>(gram_min_ratio) * static_cast<double>(m);
+    (gram ? gram_b : std_b).push_back(b);
+  }
+  const size_t need = std::max(plan_layout(std_b.data(), static_cast<int>(std_b.size()), 1).total,
+                               plan_layout(gram_b.data(), static_cast<int>(gram_b.size()), 2).total);
+  if (!std_b.empty() || !gram_b.empty())
+    if ((st = check_ws(workspace, workspace_bytes, need)) != MUON_OK) return st;
+  // One error word for the whole call: cleared once, kept across both forms.
+  if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), stream) != cudaSuccess) return MUON_CUDA_ERROR;
+  if (!std_b.empty() && (st = ns_standard_impl(std_b.data(), static_cast<int>(std_b.size()), hp, workspace,
+                                               workspace_bytes, stream, false)) != MUON_OK)
+    return st;
+  if (!gram_b.empty())
+    return ns_gram_impl(gram_b.data(), static_cast<int>(gram_b.size()), hp, workspace, workspace_bytes, stream,
+                        false);
+  return MUON_OK;
+}
+
 muon_status normuon_update(const muon_batch* batches, int nb, const muon_hparams* hp, int use_normuon,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (nb < 0 || (nb > 0 && !batches)) return MUON_INVALID_ARG;
@@ -976,6 +1033,7 @@ muon_status normuon_update(const muon_batch* batches, int nb, const muon_hparams
       S.variance = b.variance;
       S.lr_scale = b.lr_scale;
       S.vec8 = vec8_ok(b, {&b.ns_out, &b.weight, &b.weight_copy});
+      S.flat = flat_ok(b, {&b.ns_out, &b.weight, &b.weight_copy});
       ++ns;
     }
     if (ns == 0) continue;
@@ -1058,6 +1116,19 @@ muon_status muon_testing_gemm(int M, int N, int K, int slices, int tri, int in_d
   s.row_ss = tri ? nullptr : row_ss;
   std::vector<ProblemSpec> v{s};
   return launch_gemms(v, sms, reinterpret_cast<int*>(workspace), stream, cta_pair, raster_group);
+}
+
+muon_status muon_testing_bounded_wait(uint64_t limit_ns, void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream) {
+  muon_status st = check_ws(workspace, workspace_bytes, kErrBytes);
+  if (st != MUON_OK) return st;
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return MUON_INVALID_ARG;
+  int sms = 0;
+  if ((st = device_setup(&sms)) != MUON_OK) return st;
+  if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), stream) != cudaSuccess) return MUON_CUDA_ERROR;
+  bounded_wait_probe_kernel<<<1, 32, 0, stream>>>(reinterpret_cast<int*>(workspace), limit_ns,
+                                                  MUON_TESTING_WAIT_TIMEOUT);
+  return launched() ? MUON_OK : MUON_CUDA_ERROR;
 }
 
 }  // extern "C"

@@ -538,6 +538,20 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
   }
 }
 
+// Failure-path probe: waits with the same bounded wait on a barrier that no
+// one arrives on, and records the timeout like the GEMM roles do.
+__global__ void bounded_wait_probe_kernel(int* err, unsigned long long limit_ns, int code) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, &abort_flag, limit_ns)) record_error(err, &abort_flag, code);
+}
+
 __global__ void __launch_bounds__(GEMM_THREADS, 1) ns_gemm_kernel(const __grid_constant__ GemmParams P) {
   ns_gemm_body<1>(P);
 }

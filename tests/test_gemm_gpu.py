@@ -180,3 +180,20 @@ def test_pair_and_single_cta_agree(mn):
     assert mn.workspace_error(ws) == 0
     _check(C2, _f64(A) @ _f64(B))
     assert float((C1.float() - C2.float()).abs().max()) <= 2e-2 * float(C1.float().abs().max())
+
+
+def test_bounded_wait_times_out_and_context_survives(mn):
+    # A device wait that nothing satisfies gives up after its limit, reports
+    # through the workspace word, and leaves the context usable.
+    from newton_schulz_ns_b200 import _capi
+    ws = _ws()
+    st = _capi.lib.muon_testing_bounded_wait(2_000_000, ws.data_ptr(), 256, torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    assert mn.workspace_error(ws) == 4                      # MUON_TESTING_WAIT_TIMEOUT
+    A = _rnd((1, 128, 64), torch.bfloat16, 13)
+    B = _rnd((1, 256, 64), torch.bfloat16, 14)
+    C = _empty((1, 128, 256), torch.bfloat16)
+    mn.testing_gemm(A, False, B, False, C, K=64, workspace=ws)
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0
+    _check(C, _f64(A) @ np.swapaxes(_f64(B), 1, 2))

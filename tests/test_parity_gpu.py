@@ -374,3 +374,24 @@ def test_full_step_matches_oracle(mn, key, variant):
             st["M"] = f64(b.momentum)
             st["W"] = f64(b.weight)
             st["v"] = f64(b.variance).reshape(b.n, b.rows) if w.normuon else None
+
+
+def test_auto_dispatch_routes_by_shape(mn):
+    # n >= 1.25 m goes through the Gram form, square and near-square through
+    # the standard form; each batch must come out exactly as its own form's
+    # call produces it.
+    shapes = [(64, 576, 3), (256, 256, 2), (300, 340, 2), (1000, 200, 1)]
+    Us = [_seeded(n, r, c, 500 + k, torch.bfloat16) for k, (r, c, n) in enumerate(shapes)]
+    auto = [_ns_batch(mn, U) for U in Us]
+    ws = mn.allocate_workspace(auto, -1)
+    mn.muon_ns_auto_batched(auto, mn.Hparams(), ws, gram_min_ratio=1.25)
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0
+    for (r, c, n), U, b in zip(shapes, Us, auto):
+        variant = "gram" if max(r, c) >= 1.25 * min(r, c) else "standard"
+        one = _ns_batch(mn, U)
+        _run_ns(mn, [one], variant, mn.Hparams())
+        assert torch.equal(one.ns_out, b.ns_out), (r, c, variant)
+        ref = _oracle_ns(U, variant)
+        for i in range(n):
+            assert rel(f64(b.ns_out)[i], ref[i]) < NS_TOL
