@@ -342,7 +342,23 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
     const long long per = std::max<long long>(1, tiles_per_slice(s, cg));
     const long long units = cg == 2 ? std::max(1, pair_units) : std::max(1, sms);
     int step_slices = s.slices;
-    if (max_waves > 0) step_slices = static_cast<int>(std::max<long long>(1, (units * max_waves) / per));
+    if (max_waves > 0) {
+      // Among chunk sizes that fit the wave budget, take the one whose launches
+      // leave the fewest idle tile slots in their last waves (largest on ties).
+      const int kmax = static_cast<int>(std::max<long long>(1, std::min<long long>(s.slices, (units * max_waves) / per)));
+      double best = 1e30;
+      for (int k = kmax; k >= 1; --k) {
+        double idle = 0.0;
+        for (int s0 = 0; s0 < s.slices; s0 += k) {
+          const long long t = per * std::min(k, s.slices - s0);
+          idle += static_cast<double>(cdiv(t, units) * units - t);
+        }
+        if (idle < best - 0.5) {
+          best = idle;
+          step_slices = k;
+        }
+      }
+    }
     for (int s0 = 0; s0 < s.slices; s0 += step_slices) {
       ProblemSpec c = s;
       const int n = std::min(step_slices, s.slices - s0);

@@ -395,3 +395,47 @@ def test_auto_dispatch_routes_by_shape(mn):
         ref = _oracle_ns(U, variant)
         for i in range(n):
             assert rel(f64(b.ns_out)[i], ref[i]) < NS_TOL
+
+
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+def test_step_captured_in_cuda_graph_matches_eager(mn, variant):
+    # The calls enqueue only kernels and memsets on the given stream, so a
+    # whole step can be captured once and replayed.  Per-device set-up runs
+    # on the first call, which therefore happens eagerly before capture.
+    w = workloads.WORKLOADS["conv_megabatch"]
+
+    def fresh():
+        gb = _workload_batches(mn, w)
+        return [b for _, b in gb]
+
+    hp = mn.Hparams(lr=w.lr, weight_decay=w.weight_decay)
+    ns_fn = mn.muon_ns_batched if variant == "standard" else mn.muon_gram_ns_batched
+    eager = fresh()
+    ws_e = mn.allocate_workspace(eager, -1)
+    for _ in range(2):
+        mn.muon_momentum_norm(eager, hp, ws_e)
+        ns_fn(eager, hp, ws_e)
+        mn.normuon_update(eager, hp, True, ws_e)
+    torch.cuda.synchronize()
+
+    graphed = fresh()
+    ws_g = mn.allocate_workspace(graphed, -1)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        # warm-up outside capture would change the state; set-up is per device
+        # and already done by the eager calls above.
+        with torch.cuda.graph(graph, stream=side):
+            mn.muon_momentum_norm(graphed, hp, ws_g, side)
+            ns_fn(graphed, hp, ws_g, side)
+            mn.normuon_update(graphed, hp, True, ws_g, side)
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws_g) == 0
+    for a, b in zip(eager, graphed):
+        assert torch.equal(a.momentum, b.momentum)
+        assert torch.equal(a.ns_out, b.ns_out)
+        assert torch.equal(a.weight, b.weight)
+        assert torch.equal(a.variance, b.variance)
