@@ -439,3 +439,55 @@ def test_step_captured_in_cuda_graph_matches_eager(mn, variant):
         assert torch.equal(a.ns_out, b.ns_out)
         assert torch.equal(a.weight, b.weight)
         assert torch.equal(a.variance, b.variance)
+
+
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+@pytest.mark.parametrize("shape", [(1, 1), (1, 16), (16, 1), (3, 5), (5, 3), (2, 2), (1, 1000), (700, 1)])
+def test_ns_degenerate_tiny_shapes(mn, variant, shape):
+    r, c = shape
+    U = _seeded(2, r, c, 40 + r * 7 + c, torch.bfloat16)
+    b = _ns_batch(mn, U)
+    _run_ns(mn, [b], variant, mn.Hparams())
+    ref = _oracle_ns(U, variant)
+    got = f64(b.ns_out)
+    for i in range(2):
+        assert rel(got[i], ref[i]) < NS_TOL, (shape, variant, rel(got[i], ref[i]))
+
+
+def _p5(s, abc=oracle.QUINTIC_ABC, steps=5):
+    a, b, c = abc
+    for _ in range(steps):
+        s = a * s + b * s ** 3 + c * s ** 5
+    return s
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("tall", [False, True])
+def test_ns_maximum_size_closed_form(mn, tall):
+    # Near the library's size limit (rows*cols < 2^31): a signed, permuted
+    # partial identity Q (orthonormal rows) scaled by 3 has every singular
+    # value equal, so Newton-Schulz maps it to p^5(1/sqrt(m)) * Q exactly.
+    # The check needs no oracle and holds at any size; the scattered +-1
+    # entries exercise every tile's indexing.
+    m, n = 32768, 65472
+    r, c = (n, m) if tall else (m, n)
+    g = torch.Generator(device=DEV).manual_seed(50)
+    cols = torch.randperm(n, generator=g, device=DEV)[:m]
+    rows = torch.randperm(m, generator=g, device=DEV)
+    signs = torch.where(torch.rand(m, generator=g, device=DEV) < 0.5, -3.0, 3.0).to(torch.bfloat16)
+    U = torch.zeros((1, r, c), dtype=torch.bfloat16, device=DEV)
+    if tall:
+        U[0, cols, rows] = signs
+    else:
+        U[0, rows, cols] = signs
+    b = _ns_batch(mn, U)
+    ws = mn.allocate_workspace([b], 1)
+    mn.muon_ns_batched([b], mn.Hparams(), ws)
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0
+    scale = _p5(3.0 / (3.0 * m ** 0.5 + 1e-7))
+    want = U.float() * (scale / 3.0)
+    err = float((b.ns_out.float() - want).norm() / want.norm())
+    assert err < 1e-2, err
+    del ws
+    torch.cuda.empty_cache()
