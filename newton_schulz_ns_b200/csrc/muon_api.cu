@@ -22,6 +22,7 @@
 #include "../../include/muon_ns_testing.h"
 #include "elementwise.cuh"
 #include "ns_gemm.cuh"
+#include "ns_small.cuh"
 
 using namespace muon;
 
@@ -76,7 +77,9 @@ muon_status device_setup(int* sms_out, int* pair_units_out = nullptr) {
       if (cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                GemmCfg<1>::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(ns_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               GemmCfg<2>::SMEM_BYTES) != cudaSuccess) {
+                               GemmCfg<2>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SMALL_SMEM_BYTES) != cudaSuccess) {
         d.ready = false;
         return MUON_CUDA_ERROR;
       }
@@ -375,12 +378,21 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
       chunk_cg.push_back(cg);
     }
   }
+  // Consecutive chunks share a launch up to max_problems; beyond that only
+  // while the whole launch stays within one wave of tiles (small problems,
+  // where a launch costs more than its tiles and nothing drifts apart).
   size_t i = 0;
   while (i < chunks.size()) {
     std::vector<const ProblemSpec*> group;
     const int cg = chunk_cg[i];
-    for (; i < chunks.size() && static_cast<int>(group.size()) < max_problems && chunk_cg[i] == cg; ++i)
+    const long long units = cg == 2 ? std::max(1, pair_units) : std::max(1, sms);
+    long long group_tiles = 0;
+    for (; i < chunks.size() && static_cast<int>(group.size()) < MAX_PROBLEMS && chunk_cg[i] == cg; ++i) {
+      const long long t = tiles_per_slice(chunks[i], cg) * chunks[i].slices;
+      if (static_cast<int>(group.size()) >= max_problems && group_tiles + t > units) break;
       group.push_back(&chunks[i]);
+      group_tiles += t;
+    }
     const int tile_m = BM * cg, b_rows = BN / cg, step = BN / tile_m;
     launches.emplace_back();
     Launch& L = launches.back();
@@ -546,6 +558,91 @@ Coefs coefs_at(const muon_hparams* hp, int it) {
 
 Mat view_mat(const muon_batch& b, const muon_view& v) {
   return Mat{v.ptr, b.rows, b.cols, v.ld, v.batch_stride, b.n, 0};
+}
+
+// ---------------------------------------------------------------- fused small-side Newton-Schulz
+// Column split of an m x n slice over a cluster: C CTAs of w columns each
+// (w a multiple of 64, at most SMALL_MAX_W; C at most SMALL_MAX_CLUSTER).
+struct SmallSplit {
+  int C, w;
+};
+
+// C is a power of two (so it divides every multiple of 8 rows of A): the
+// smallest that keeps w <= SMALL_MAX_W, raised to 4 where the slice has that
+// many 64-column blocks.  Clusters of 4 tile the device's SMs well (clusters
+// of 8 leave a fifth of the B200's SMs idle); the split depends on the shape
+// only, so a slice's sums never depend on the rest of the batch.
+SmallSplit small_split(int64_t n) {
+  const int blocks = static_cast<int>(cdiv(n, 64));
+  auto pow2_at_least = [](int x) {
+    int p = 1;
+    while (p < x) p *= 2;
+    return p;
+  };
+  int C = pow2_at_least(static_cast<int>(cdiv(blocks, SMALL_MAX_W / 64)));
+  C = std::max(C, std::min(4, pow2_at_least(blocks)));
+  return SmallSplit{C, 64 * static_cast<int>(cdiv(blocks, C))};
+}
+
+// Slices with rows <= cols, rows <= 128 and cols <= 8 * 512 run the whole
+// iteration in one clustered launch (ns_small.cuh).  The choice depends on the shape only,
+// so a slice's result never depends on the rest of the batch.  Setting
+// MUON_NS_FUSED_SMALL=0 sends them through the GEMM path instead.
+bool small_eligible(const muon_batch& b) {
+  const char* e = std::getenv("MUON_NS_FUSED_SMALL");
+  if (e && std::atoi(e) == 0) return false;
+  if (b.rows > b.cols || b.rows > SMALL_MAX_M) return false;
+  const SmallSplit sp = small_split(b.cols);
+  return sp.C <= SMALL_MAX_CLUSTER && sp.w <= SMALL_MAX_W;
+}
+
+muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const float* sumsq, int* err,
+                         cudaStream_t stream) {
+  const SmallSplit sp = small_split(b.cols);
+  SmallParams P;
+  std::memset(&P, 0, sizeof(P));
+  if (!encode_map(&P.map_in, view_mat(b, b.ns_in), 64, 128)) return MUON_CUDA_ERROR;
+  if (!encode_map(&P.map_out, view_mat(b, b.ns_out), 64, 128)) return MUON_CUDA_ERROR;
+  P.tma_store = (b.cols % 8 == 0) ? 1 : 0;
+  P.out = static_cast<__nv_bfloat16*>(const_cast<void*>(b.ns_out.ptr));
+  P.out_ld = b.ns_out.ld;
+  P.out_bs = b.ns_out.batch_stride;
+  P.sumsq = sumsq;
+  P.eps = hp->ns_eps;
+  P.m = static_cast<int>(b.rows);
+  P.n = static_cast<int>(b.cols);
+  P.w = sp.w;
+  P.steps = hp->ns_steps;
+  for (int k = 0; k < hp->ns_steps; ++k) {
+    const Coefs cf = coefs_at(hp, k);
+    P.a[k] = cf.a;
+    P.b[k] = cf.b;
+    P.c[k] = cf.c;
+  }
+  P.err = err;
+  P.timeout_ns = kWaitLimitNs;
+  constexpr int64_t kMaxGridY = 65535;
+  for (int64_t s0 = 0; s0 < b.n; s0 += kMaxGridY) {
+    P.slice0 = static_cast<int>(s0);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(sp.C), static_cast<unsigned>(std::min(kMaxGridY, b.n - s0)), 1);
+    cfg.blockDim = dim3(SMALL_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMALL_SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(sp.C);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, ns_small_kernel, P) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return MUON_CUDA_ERROR;
+    }
+    if (!launched()) return MUON_CUDA_ERROR;
+  }
+  return MUON_OK;
 }
 
 // SYRK of the slice storage X ([rows][cols]) on the short side: out = f * X X^T (rows <= cols)
@@ -853,13 +950,19 @@ muon_status ns_standard_impl(const muon_batch* batches, int nb, const muon_hpara
   if ((st = prepare_norms(batches, nb, L, ws, sms, stream, sumsq, clear_err)) != MUON_OK) return st;
   int* err = reinterpret_cast<int*>(ws);
 
+  std::vector<char> fused(nb, 0);
+  for (int i = 0; i < nb; ++i) {
+    if (batch_empty(batches[i]) || !small_eligible(batches[i])) continue;
+    fused[i] = 1;
+    if ((st = launch_small(batches[i], hp, sumsq[i], err, stream)) != MUON_OK) return st;
+  }
   const int S = hp->ns_steps;
   for (int it = 0; it < S; ++it) {
     const Coefs cf = coefs_at(hp, it);
     std::vector<ProblemSpec> syrk, poly, apply;
     for (int i = 0; i < nb; ++i) {
       const muon_batch& b = batches[i];
-      if (batch_empty(b)) continue;
+      if (batch_empty(b) || fused[i]) continue;
       const NsBatchWs& w = L.nsb[i];
       const int m = static_cast<int>(std::min(b.rows, b.cols));
       void* Abuf = ws + w.off[0];

@@ -1,0 +1,412 @@
+// Fused Newton-Schulz for slices whose short side is at most 128 (sm_100a).
+//
+// For a slice X (m x n, stored row-major, m = rows <= cols, m <= 128) every
+// quintic step is
+//   A = X X^T,  B = b A + c A^2,  X <- a X + B X
+// (Newton-Schulz iteration as the Megatron-Core layer_sharded_muon docs and
+// DeepSpeed issue #8437 describe it; the first step works on the Frobenius-
+// normalized X0 = s U, s = 1 / (||U||_F + eps), folded into the epilogues as
+// on the GEMM path).  With m this small each product is a few MFLOP, so the
+// GEMM path spends its time in launches and pipeline fill.  Here one
+// thread-block cluster of C CTAs (C = 1, 2, 4 or 8) runs all steps of one
+// slice in one launch:
+//
+//   * CTA r keeps columns [r w, (r+1) w) of X resident in shared memory for
+//     the whole iteration (w <= 512, 128 rows: rows past m are zero and stay
+//     zero, since A, B and X vanish there);
+//   * A = sum_r X_r X_r^T: each CTA multiplies its own columns on the tensor
+//     core (fp32 in TMEM) and pushes each row of its partial to the CTA that
+//     owns the row (R = m8 / C rows each, m8 = m rounded up to 8) with
+//     distributed-shared-memory stores; after a cluster barrier each owner
+//     sums its rows over the C partials in rank order (deterministic),
+//     scales and rounds them to bf16 and pushes them into every CTA's copy
+//     of A; a second barrier completes A everywhere;
+//   * each CTA forms B = b A + c A^2 over its copy of A (128^3, redundantly;
+//     cheaper than another exchange) and its own columns of a X + B X, which
+//     need no other CTA's data, and writes them back over X;
+//   * after the last step the resident columns go to ns_out by TMA.
+//
+// Precision follows the GEMM path: bf16 operands, fp32 accumulation, A, B
+// and X rounded to bf16 between products.  Operand layouts are the 128-byte
+// swizzled tiles TMA writes (64 columns x 128 rows per 16 KB block): X is
+// read K-major for X X^T and MN-major for B X without any copy.
+//
+// 256 threads, one CTA per SM (the shared-memory request reserves the SM):
+// thread 0 issues TMA and MMAs; in the epilogues warp w reads TMEM lanes
+// 32 (w % 4) .. + 31 (one row per thread) and half w / 4 of the columns.
+// Every mbarrier wait is bounded; a CTA that gives up records an error,
+// stops issuing work and still takes every cluster barrier, so its peers
+// finish too.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "ptx_sm100.cuh"
+
+namespace muon {
+
+constexpr int SMALL_THREADS = 256;
+constexpr int SMALL_MAX_STEPS = 16;
+constexpr int SMALL_MAX_CLUSTER = 8;
+constexpr int SMALL_MAX_M = 128;
+constexpr int SMALL_MAX_W = 512;                       // resident columns per CTA
+constexpr int SMALL_BLK = 128 * 128;                   // one 64-column block of 128 bf16 rows
+constexpr int SMALL_X_BYTES = SMALL_MAX_W / 64 * SMALL_BLK;   // 128 KB
+constexpr int SMALL_A_BYTES = 2 * SMALL_BLK;                  // A (then B in place): 128 x 128 bf16
+constexpr int SMALL_RECV_BYTES = 128 * 512;                   // C slots x R rows of fp32 partials
+constexpr int SMALL_SMEM_BYTES = 1024 + SMALL_X_BYTES + SMALL_A_BYTES + SMALL_RECV_BYTES + 64;
+
+enum SmallError : int { kSmallErrLoad = 5, kSmallErrMma = 6 };
+
+struct __align__(64) SmallParams {
+  CUtensorMap map_in;        // ns_in  [slices][m][n] bf16, box {64, 128, 1}, 128-B swizzle
+  CUtensorMap map_out;       // ns_out, same geometry (used when tma_store)
+  __nv_bfloat16* out;        // ns_out, for element stores
+  long long out_ld, out_bs;
+  const float* sumsq;        // [slices] sum of squares of each input slice
+  float eps;
+  int m, n;                  // short side (rows) and long side (cols)
+  int w;                     // columns per CTA, a multiple of 64, <= SMALL_MAX_W
+  int slice0;                // first slice of this launch
+  int steps;
+  int tma_store;             // n is a multiple of 8: whole 16-byte chunks, TMA clips exactly
+  float a[SMALL_MAX_STEPS], b[SMALL_MAX_STEPS], c[SMALL_MAX_STEPS];
+  int* err;
+  unsigned long long timeout_ns;
+};
+
+// Byte offset of the 16-byte chunk holding columns [8 ch, 8 ch + 8) of row r
+// in a stack of 64-column SW128 blocks of 128 rows.
+__device__ __forceinline__ uint32_t sw128_chunk(int r, int ch) {
+  return static_cast<uint32_t>((ch >> 3) * SMALL_BLK + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+}
+
+// Byte offset of the 16-byte chunk holding columns [4 j, 4 j + 4) of row t
+// of the partial-sum receive buffer (512-byte rows; chunks XOR-swizzled by
+// the row so that the rows pushed by one warp land in distinct banks).
+__device__ __forceinline__ uint32_t recv_chunk(int t, int j) {
+  return static_cast<uint32_t>(t * 512 + ((j ^ (t & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    f[2 * h] = __uint_as_float(w[h] << 16);
+    f[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float (&o)[8]) {
+  return make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                    pack_bf16x2(o[6], o[7]));
+}
+
+__device__ __forceinline__ void small_record_error(int* err, volatile int* abort_flag, int code) {
+  *abort_flag = 1;
+  if (err) atomicCAS(err, 0, code);
+}
+
+// Two 32-column TMEM loads (64 columns of this thread's row) and one wait.
+__device__ __forceinline__ void tmem_ld_64(uint32_t taddr, uint32_t (&v)[64]) {
+  tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(v));
+  tmem_ld_32x32b_x32(taddr + 32u, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+  tmem_ld_wait();
+}
+
+__global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid_constant__ SmallParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* Xs = smem;
+  uint8_t* As = Xs + SMALL_X_BYTES;   // A, overwritten in place by B = b A + c A^2
+  uint8_t* Rv = As + SMALL_A_BYTES;   // partial rows pushed here by every CTA of the cluster
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Rv + SMALL_RECV_BYTES);   // [0] load, [1] MMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int quarter = warp & 3;                     // TMEM lanes 32 quarter .. + 31
+  const int half = warp >> 2;                       // column half handled in the epilogues
+  const int row = quarter * 32 + (tid & 31);        // TMEM lane = row of the 128-row tiles
+  const uint32_t tlane = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t rank = cluster_ctarank();
+  const int C = static_cast<int>(gridDim.x);        // the cluster spans gridDim.x
+  const int slice = P.slice0 + static_cast<int>(blockIdx.y);
+  const int w = P.w;
+  const int nblk = w >> 6;
+  const int m8 = (P.m + 7) & ~7;                    // rows / columns of A that can be nonzero
+  const int R = m8 / C;                             // rows of A each CTA reduces (C divides m8)
+  const uint32_t ncols = w > 256 ? 512u : 256u;     // P and A^2 take 256 columns; a X + B X takes w
+
+  if (tid == 0) {
+    *abort_flag = 0;
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&P.map_in);
+    tma_prefetch_desc(&P.map_out);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, ncols);
+    tmem_relinquish();
+  }
+  // A outside its m8 x m8 corner is never written by the exchange: zero it once.
+  for (int i = tid; i < SMALL_A_BYTES / 16; i += SMALL_THREADS)
+    reinterpret_cast<uint4*>(As)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // ---- resident columns of the slice (zero outside it)
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], static_cast<uint32_t>(nblk * SMALL_BLK));
+    for (int j = 0; j < nblk; ++j)
+      tma_load_3d(Xs + j * SMALL_BLK, &P.map_in, &bars[0], static_cast<int>(rank) * w + 64 * j, 0, slice);
+  }
+  bool ok = __syncthreads_and(mbar_wait_bounded(&bars[0], 0, abort_flag, P.timeout_ns)) != 0;
+  if (!ok && tid == 0) small_record_error(P.err, abort_flag, kSmallErrLoad);
+  cluster_sync();             // every CTA of the cluster runs before its shared memory is addressed remotely
+
+  const float s = 1.0f / (sqrtf(P.sumsq[slice]) + P.eps);
+  uint32_t mph = 0;          // completed phases of the MMA barrier
+  bool pending = false;      // an MMA commit whose wait gave up
+  auto wait_mma = [&]() {
+    const bool got = mbar_wait_bounded(&bars[1], mph & 1u, abort_flag, P.timeout_ns);
+    const bool all = __syncthreads_and(got) != 0;
+    if (!all) {
+      pending = true;
+      if (tid == 0) small_record_error(P.err, abort_flag, kSmallErrMma);
+    }
+    ++mph;
+    return all;
+  };
+
+  const uint32_t idesc_sq = mma_idesc_f16(1, 0, 0, 128, 128);
+  const uint32_t rv0 = smem_u32(Rv);
+  const uint32_t a0 = smem_u32(As);
+
+  for (int k = 0; k < P.steps; ++k) {
+    const float ca = P.a[k], cb = P.b[k], cc = P.c[k];
+    // ---- partial X_r X_r^T -> TMEM columns [0, 128)
+    if (ok) {
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t x0 = smem_u32(Xs);
+        for (int kk = 0; kk < w / 16; ++kk) {
+          const uint64_t d = smem_desc_sw128(x0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+          tc_mma_f16(tmem, d, d, idesc_sq, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars[1]);
+      }
+      ok = wait_mma();
+    }
+    // ---- push row `row` of the partial, columns [64 half, 64 half + 64) below m8, to the row's owner
+    if (ok && half * 64 < m8) {
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld_64(tmem + tlane + static_cast<uint32_t>(half * 64), v);
+      if (row < m8) {
+        const int owner = row / R;
+        const int t = static_cast<int>(rank) * R + (row - owner * R);   // slot `rank`, row within it
+        const int jn = min(16, (m8 - half * 64) >> 2);                  // 4-column chunks to send
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if (j < jn) {
+            const uint32_t dst = mapa_shared(rv0 + recv_chunk(t, half * 16 + j), static_cast<uint32_t>(owner));
+            st_cluster_v4(dst, make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+          }
+        }
+      }
+    }
+    tc_fence_before();
+    cluster_sync();           // every partial row has reached its owner
+
+    // ---- owner: A rows [rank R, rank R + R) = f * sum over the slots, pushed to every CTA
+    if (ok) {
+      const float fA = (k == 0) ? s * s : 1.0f;
+      const int groups = m8 >> 3;                   // 8-column groups per row
+      for (int it = tid; it < R * groups; it += SMALL_THREADS) {
+        const int i = it / groups;
+        const int g = it - i * groups;
+        float4 lo[SMALL_MAX_CLUSTER], hi[SMALL_MAX_CLUSTER];
+#pragma unroll
+        for (int q = 0; q < SMALL_MAX_CLUSTER; ++q) {
+          if (q < C) {
+            const int t = q * R + i;
+            lo[q] = *reinterpret_cast<const float4*>(Rv + recv_chunk(t, 2 * g));
+            hi[q] = *reinterpret_cast<const float4*>(Rv + recv_chunk(t, 2 * g + 1));
+          }
+        }
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+#pragma unroll
+        for (int q = 0; q < SMALL_MAX_CLUSTER; ++q) {
+          if (q < C) {
+            acc[0] += lo[q].x; acc[1] += lo[q].y; acc[2] += lo[q].z; acc[3] += lo[q].w;
+            acc[4] += hi[q].x; acc[5] += hi[q].y; acc[6] += hi[q].z; acc[7] += hi[q].w;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= fA;
+        const uint4 pk = pack_bf16x8(acc);
+        const uint32_t dst = a0 + sw128_chunk(static_cast<int>(rank) * R + i, g);
+        for (int q = 0; q < C; ++q) st_cluster_v4(mapa_shared(dst, static_cast<uint32_t>(q)), pk);
+      }
+      fence_proxy_async_cluster();
+    }
+    cluster_sync();           // every CTA holds the whole A; the receive slots are free again
+
+    // ---- A^2 -> TMEM columns [128, 256)
+    if (ok) {
+      if (tid == 0) {
+        fence_proxy_async_smem();
+        tc_fence_after();
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t d = smem_desc_sw128(a0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+          tc_mma_f16(tmem + 128, d, d, idesc_sq, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars[1]);
+      }
+      ok = wait_mma();
+    }
+    // ---- B = c A^2 + b A, in place over A (row `row`, columns [64 half, 64 half + 64))
+    if (ok) {
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld_64(tmem + tlane + 128u + static_cast<uint32_t>(half * 64), v);
+      if (row < m8) {
+        uint4 av[8];
+#pragma unroll
+        for (int h = 0; h < 8; ++h) av[h] = *reinterpret_cast<const uint4*>(As + sw128_chunk(row, half * 8 + h));
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          float af[8], o[8];
+          unpack_bf16x8(av[h], af);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float x = cc * __uint_as_float(v[h * 8 + e]);
+            x += cb * af[e];
+            o[e] = x;
+          }
+          *reinterpret_cast<uint4*>(As + sw128_chunk(row, half * 8 + h)) = pack_bf16x8(o);
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- B X_r -> TMEM columns [0, w)
+    if (ok) {
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t x0 = smem_u32(Xs);
+        for (int nc = 0; nc < w; nc += 256) {
+          const int N = min(256, w - nc);
+          const uint32_t idesc = mma_idesc_f16(1, 0, 1, 128, static_cast<uint32_t>(N));
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ad = smem_desc_sw128(a0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(x0 + (nc >> 6) * SMALL_BLK + kk * 16 * 128, SMALL_BLK, 1024);
+            tc_mma_f16(tmem + static_cast<uint32_t>(nc), ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+        }
+        tc_commit(&bars[1]);
+      }
+      ok = wait_mma();
+    }
+    // ---- X <- f * (B X + a X), in place (row `row`, columns [half w/2, half w/2 + w/2))
+    if (ok) {
+      tc_fence_after();
+      const float fX = (k == 0) ? s : 1.0f;
+      const int hw = w >> 1;
+      const int cend = half * hw + hw;
+#pragma unroll 1
+      for (int c0 = half * hw; c0 < cend; c0 += 64) {
+        const bool two = c0 + 64 <= cend;           // warp-uniform: 64 or 32 columns
+        uint32_t v[64];
+        if (two) {
+          tmem_ld_64(tmem + tlane + static_cast<uint32_t>(c0), v);
+        } else {
+          tmem_ld_32x32b_x32(tmem + tlane + static_cast<uint32_t>(c0), *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld_wait();
+        }
+        if (row < m8) {
+          const int nch = two ? 8 : 4;
+          uint4 xv[8];
+#pragma unroll
+          for (int h = 0; h < 8; ++h)
+            if (h < nch) xv[h] = *reinterpret_cast<const uint4*>(Xs + sw128_chunk(row, (c0 >> 3) + h));
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            if (h < nch) {
+              float xf[8], o[8];
+              unpack_bf16x8(xv[h], xf);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                float x = __uint_as_float(v[h * 8 + e]);
+                x += ca * xf[e];
+                o[e] = x * fX;
+              }
+              *reinterpret_cast<uint4*>(Xs + sw128_chunk(row, (c0 >> 3) + h)) = pack_bf16x8(o);
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  // ---- resident columns -> ns_out (rows < m, columns < n)
+  if (ok) {
+    const int col_base = static_cast<int>(rank) * w;
+    if (P.tma_store) {
+      if (tid == 0) {
+        for (int j = 0; j < nblk && col_base + 64 * j < P.n; ++j)
+          tma_store_3d(&P.map_out, Xs + j * SMALL_BLK, col_base + 64 * j, 0, slice);
+        bulk_commit_group();
+        bulk_wait_group_all();
+      }
+    } else {
+      const int chunks = w >> 3;
+      __nv_bfloat16* out = P.out + static_cast<long long>(slice) * P.out_bs;
+      for (int it = tid; it < P.m * chunks; it += SMALL_THREADS) {
+        const int r = it / chunks;
+        const int ch = it - r * chunks;
+        const int col = col_base + ch * 8;
+        if (col >= P.n) continue;
+        const uint4 v = *reinterpret_cast<const uint4*>(Xs + sw128_chunk(r, ch));
+        __nv_bfloat16* dst = out + static_cast<long long>(r) * P.out_ld + col;
+        if (col + 8 <= P.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+          *reinterpret_cast<uint4*>(dst) = v;
+        } else {
+          const uint16_t* e16 = reinterpret_cast<const uint16_t*>(&v);
+          for (int e = 0; e < 8 && col + e < P.n; ++e) reinterpret_cast<uint16_t*>(dst)[e] = e16[e];
+        }
+      }
+    }
+  }
+
+  // A commit whose wait gave up may still be running: give it one more
+  // bounded wait before its TMEM is released.
+  if (pending && tid == 0) {
+    volatile int never = 0;
+    (void)mbar_wait_bounded(&bars[1], (mph - 1u) & 1u, &never, P.timeout_ns);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();             // no CTA leaves while a peer may still address its shared memory
+  if (warp == 0) tmem_dealloc(tmem, ncols);
+}
+
+}  // namespace muon

@@ -1,0 +1,186 @@
+"""Parity of the fused small-side Newton-Schulz kernel with the fp64 oracle.
+
+Slices with rows <= cols, rows <= 128 and cols <= 4096 (the per-head
+[32, 128, 4096] batch, the conv megabatch [16, 64, 576]) run the whole
+iteration in one clustered launch: each CTA keeps a column block of X in
+shared memory and the cluster sums X X^T over distributed shared memory.
+The shapes below cover every cluster split the planner picks (1 to 8 CTAs,
+64 to 512 columns each), ragged last blocks, CTAs that hold only padding,
+and short sides from 1 to 128.  Bars: 3e-2 relative Frobenius error against
+the oracle per slice; bitwise batch invariance and run-to-run determinism;
+nothing written outside the slice.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+NS_TOL = 3e-2
+
+
+@pytest.fixture(scope="module")
+def mn():
+    import newton_schulz_ns_b200 as m
+    return m
+
+
+def f64(t):
+    return t.detach().float().cpu().double().numpy()
+
+
+def rel(a, b):
+    nb = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / nb) if nb > 0 else float(np.linalg.norm(a))
+
+
+def _padded(n, r, c, dtype, fill, pad=8):
+    ld = (c + 7) // 8 * 8 + pad
+    base = torch.full((n, r, ld), fill, dtype=dtype, device=DEV)
+    return base, base[:, :, :c]
+
+
+def _seeded(n, r, c, seed, std=1.0):
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn((n, r, c), generator=g) * std).to(torch.bfloat16)
+    _, t = _padded(n, r, c, torch.bfloat16, 0.0)
+    t.copy_(x.to(DEV))
+    return t
+
+
+def _ns(mn, U, hp=None, fused=True):
+    n, r, c = U.shape
+    base, out = _padded(n, r, c, torch.bfloat16, float("nan"))
+    b = mn.Batch(n, r, c, ns_in=U, ns_out=out)
+    ws = mn.allocate_workspace([b], 1)
+    old = os.environ.get("MUON_NS_FUSED_SMALL")
+    os.environ["MUON_NS_FUSED_SMALL"] = "1" if fused else "0"
+    try:
+        before = mn.kernel_launches()
+        mn.muon_ns_batched([b], hp or mn.Hparams(), ws)
+        launches = mn.kernel_launches() - before
+        torch.cuda.synchronize()
+    finally:
+        if old is None:
+            del os.environ["MUON_NS_FUSED_SMALL"]
+        else:
+            os.environ["MUON_NS_FUSED_SMALL"] = old
+    assert mn.workspace_error(ws) == 0
+    return base, out, launches
+
+
+# (rows, cols): cluster split (CTAs x columns each) the planner picks
+SHAPES = [
+    (64, 576),     # conv megabatch slice: 4 x 192, the last CTA partly padding
+    (128, 4096),   # attention head: 8 x 512
+    (128, 2000),   # 4 x 512, ragged last block
+    (100, 1000),   # 4 x 256, ragged
+    (128, 128),    # 2 x 64
+    (3, 5),        # 1 x 64, element stores (cols not a multiple of 8)
+    (1, 4096),     # one row: each CTA owns one row of A
+    (128, 4040),   # 8 x 512, last CTA mostly padding
+    (65, 3000),    # 8 x 384, 9 rows of A per CTA
+    (33, 200),     # 4 x 64, 10 rows of A per CTA, one CTA only padding
+    (50, 1001),    # 4 x 256, 14 rows of A per CTA, element stores
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_fused_small_matches_oracle(mn, shape):
+    r, c = shape
+    U = _seeded(3, r, c, 500 + r + c)
+    base, out, launches = _ns(mn, U)
+    assert launches <= 3      # norms (2) + one fused launch
+    ref = oracle.ns_batched(f64(U), "standard")
+    got = f64(out)
+    for i in range(3):
+        assert rel(got[i], ref[i]) < NS_TOL, (shape, i, rel(got[i], ref[i]))
+    # Nothing outside the slice was written.
+    pad = base[:, :, c:]
+    assert torch.isnan(pad.float()).all()
+
+
+@pytest.mark.parametrize("shape", [(64, 576), (128, 4096), (100, 1000)])
+def test_fused_small_agrees_with_gemm_path(mn, shape):
+    r, c = shape
+    U = _seeded(2, r, c, 900 + r)
+    _, fused, nf = _ns(mn, U, fused=True)
+    _, gemm, ng = _ns(mn, U, fused=False)
+    assert nf < ng
+    ref = oracle.ns_batched(f64(U), "standard")
+    for i in range(2):
+        assert rel(f64(fused)[i], ref[i]) < NS_TOL
+        assert rel(f64(gemm)[i], ref[i]) < NS_TOL
+        # Same arithmetic up to the order of fp32 sums: far below the bar.
+        assert rel(f64(fused)[i], f64(gemm)[i]) < 1e-2
+
+
+def test_fused_small_batch_invariance_and_determinism(mn):
+    U = _seeded(40, 128, 1024, 77)
+    _, all_out, _ = _ns(mn, U)
+    _, again, _ = _ns(mn, U)
+    assert torch.equal(all_out, again)
+    for i in (0, 17, 39):
+        _, one, _ = _ns(mn, U[i:i + 1].clone())
+        assert torch.equal(one[0], all_out[i])
+    rev = U.flip(0).contiguous()
+    _, rout, _ = _ns(mn, rev)
+    assert torch.equal(rout.flip(0), all_out)
+
+
+def test_fused_small_many_slices(mn):
+    # Many more clusters than fit on the device at once: 300 slices of 8 CTAs.
+    U = _seeded(300, 128, 4096, 31)
+    _, out, launches = _ns(mn, U)
+    assert launches <= 3
+    ref = oracle.ns_batched(f64(U[::37]), "standard")
+    got = f64(out[::37])
+    for i in range(ref.shape[0]):
+        assert rel(got[i], ref[i]) < NS_TOL
+
+
+@pytest.mark.parametrize("steps", [1, 3, 16])
+def test_fused_small_steps_and_schedule(mn, steps):
+    sched = [(3.4445 - 0.05 * k, -4.7750 + 0.1 * k, 2.0315 - 0.05 * k) for k in range(steps)]
+    U = _seeded(2, 96, 700, 8)
+    _, out, _ = _ns(mn, U, mn.Hparams(ns_steps=steps, abc_schedule=sched))
+    X = f64(U)
+    for i in range(2):
+        x = oracle.frobenius_normalize(X[i], 1e-7)
+        for (a, bb, cc) in sched:
+            A = x @ x.T
+            x = a * x + (bb * A + cc * A @ A) @ x
+        assert rel(f64(out)[i], x) < NS_TOL
+
+
+def test_fused_small_head_view_of_projection(mn):
+    # q_proj 4096 x 4096 viewed as 32 heads of 128 rows: no copy, the batch
+    # stride is 128 rows of the projection.
+    g = torch.Generator().manual_seed(3)
+    W = torch.randn((4096, 4096), generator=g).to(torch.bfloat16).to(DEV)
+    heads = W.view(32, 128, 4096)
+    out = torch.empty_like(heads)
+    b = mn.Batch(32, 128, 4096, ns_in=heads, ns_out=out)
+    ws = mn.allocate_workspace([b], 1)
+    mn.muon_ns_batched([b], mn.Hparams(), ws)
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0
+    ref = oracle.per_head_ns(f64(W), 32, "standard")
+    got = f64(out.view(4096, 4096))
+    for h in (0, 13, 31):
+        blk = slice(128 * h, 128 * h + 128)
+        assert rel(got[blk], ref[blk]) < NS_TOL
+
+
+def test_fused_small_zero_slice(mn):
+    U = _seeded(3, 64, 576, 5)
+    U[1].zero_()
+    _, out, _ = _ns(mn, U)
+    assert torch.count_nonzero(out[1]) == 0
+    ref = oracle.ns_batched(f64(U), "standard")
+    for i in (0, 2):
+        assert rel(f64(out)[i], ref[i]) < NS_TOL
