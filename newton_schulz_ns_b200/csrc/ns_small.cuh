@@ -15,12 +15,13 @@
 //     the whole iteration (w <= 512, 128 rows: rows past m are zero and stay
 //     zero, since A, B and X vanish there);
 //   * A = sum_r X_r X_r^T: each CTA multiplies its own columns on the tensor
-//     core (fp32 in TMEM) and pushes each row of its partial to the CTA that
-//     owns the row (R = m8 / C rows each, m8 = m rounded up to 8) with
-//     distributed-shared-memory stores; after a cluster barrier each owner
-//     sums its rows over the C partials in rank order (deterministic),
-//     scales and rounds them to bf16 and pushes them into every CTA's copy
-//     of A; a second barrier completes A everywhere;
+//     core (fp32 in TMEM) and pushes the lower triangle of each row of its
+//     partial to the CTA that owns the row's 8-row block, with distributed-
+//     shared-memory stores; after a cluster barrier each owner sums its rows
+//     over the C partials in rank order (deterministic), scales and rounds
+//     them to bf16 and pushes them into every CTA's copy of A; after a
+//     second barrier each CTA fills A's upper triangle from the lower one
+//     (A is exactly symmetric, as on the GEMM path);
 //   * each CTA forms B = b A + c A^2 over its copy of A (128^3, redundantly;
 //     cheaper than another exchange) and its own columns of a X + B X, which
 //     need no other CTA's data, and writes them back over X;
@@ -52,7 +53,7 @@ constexpr int SMALL_MAX_W = 512;                       // resident columns per C
 constexpr int SMALL_BLK = 128 * 128;                   // one 64-column block of 128 bf16 rows
 constexpr int SMALL_X_BYTES = SMALL_MAX_W / 64 * SMALL_BLK;   // 128 KB
 constexpr int SMALL_A_BYTES = 2 * SMALL_BLK;                  // A (then B in place): 128 x 128 bf16
-constexpr int SMALL_RECV_BYTES = 128 * 512;                   // C slots x R rows of fp32 partials
+constexpr int SMALL_RECV_BYTES = 128 * 512;                   // C slots of fp32 partial rows
 constexpr int SMALL_SMEM_BYTES = 1024 + SMALL_X_BYTES + SMALL_A_BYTES + SMALL_RECV_BYTES + 64;
 
 enum SmallError : int { kSmallErrLoad = 5, kSmallErrMma = 6 };
@@ -101,6 +102,12 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& u, float (&f)[8]) {
   }
 }
 
+// 16-bit element e (0..7, a compile-time constant after unrolling) of 8 packed values.
+__device__ __forceinline__ uint32_t bf16_at(const uint4& u, int e) {
+  const uint32_t word = (e >> 1) == 0 ? u.x : (e >> 1) == 1 ? u.y : (e >> 1) == 2 ? u.z : u.w;
+  return (e & 1) ? (word >> 16) : (word & 0xFFFFu);
+}
+
 __device__ __forceinline__ uint4 pack_bf16x8(const float (&o)[8]) {
   return make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
                     pack_bf16x2(o[6], o[7]));
@@ -141,7 +148,17 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
   const int w = P.w;
   const int nblk = w >> 6;
   const int m8 = (P.m + 7) & ~7;                    // rows / columns of A that can be nonzero
-  const int R = m8 / C;                             // rows of A each CTA reduces (C divides m8)
+  // Row blocks of 8 are dealt to the C CTAs in the order 0, G-1, 1, G-2, ...
+  // in runs of kb, so that every CTA reduces about the same share of the
+  // lower triangle; a receive slot holds the kb blocks of one owner.
+  const int G = m8 >> 3;
+  const int kb = (G + C - 1) / C;
+  const int Rm = kb * 8;                            // rows per receive slot (C * Rm <= 128)
+  auto fold = [G](int b) {
+    const int lo = min(b, G - 1 - b);
+    return 2 * lo + (b > G - 1 - b ? 1 : 0);
+  };
+  auto unfold = [G](int p) { return (p & 1) ? G - 1 - (p >> 1) : (p >> 1); };
   const uint32_t ncols = w > 256 ? 512u : 256u;     // P and A^2 take 256 columns; a X + B X takes w
 
   if (tid == 0) {
@@ -208,15 +225,18 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
       }
       ok = wait_mma();
     }
-    // ---- push row `row` of the partial, columns [64 half, 64 half + 64) below m8, to the row's owner
+    // ---- push row `row` of the partial, its lower triangle (4-column chunks
+    //      up to the diagonal) within columns [64 half, 64 half + 64), to the
+    //      CTA that owns the row's 8-row block
     if (ok && half * 64 < m8) {
       tc_fence_after();
       uint32_t v[64];
       tmem_ld_64(tmem + tlane + static_cast<uint32_t>(half * 64), v);
       if (row < m8) {
-        const int owner = row / R;
-        const int t = static_cast<int>(rank) * R + (row - owner * R);   // slot `rank`, row within it
-        const int jn = min(16, (m8 - half * 64) >> 2);                  // 4-column chunks to send
+        const int p = fold(row >> 3);
+        const int owner = p / kb;
+        const int t = static_cast<int>(rank) * Rm + (p - owner * kb) * 8 + (row & 7);   // slot `rank`
+        const int jn = min(16, (row >> 2) + 1 - half * 16);                             // chunks to send
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           if (j < jn) {
@@ -229,20 +249,29 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
     tc_fence_before();
     cluster_sync();           // every partial row has reached its owner
 
-    // ---- owner: A rows [rank R, rank R + R) = f * sum over the slots, pushed to every CTA
+    // ---- owner: for its row blocks b, A[8b .. 8b+7][0 .. 8b+7] = f * sum over
+    //      the slots in rank order, pushed to every CTA (the diagonal block's
+    //      upper half carries unsent entries; the mirror below replaces it)
     if (ok) {
       const float fA = (k == 0) ? s * s : 1.0f;
-      const int groups = m8 >> 3;                   // 8-column groups per row
-      for (int it = tid; it < R * groups; it += SMALL_THREADS) {
-        const int i = it / groups;
-        const int g = it - i * groups;
+      int items = 0;
+      for (int lb = 0; lb < kb && rank * kb + lb < G; ++lb) items += 8 * (unfold(rank * kb + lb) + 1);
+      for (int it = tid; it < items; it += SMALL_THREADS) {
+        int lb = 0, rest = it, b = unfold(rank * kb);
+        while (rest >= 8 * (b + 1)) {
+          rest -= 8 * (b + 1);
+          ++lb;
+          b = unfold(rank * kb + lb);
+        }
+        const int r8 = rest / (b + 1);
+        const int g = rest - r8 * (b + 1);
+        const int tl = lb * 8 + r8;                 // row within each slot
         float4 lo[SMALL_MAX_CLUSTER], hi[SMALL_MAX_CLUSTER];
 #pragma unroll
         for (int q = 0; q < SMALL_MAX_CLUSTER; ++q) {
           if (q < C) {
-            const int t = q * R + i;
-            lo[q] = *reinterpret_cast<const float4*>(Rv + recv_chunk(t, 2 * g));
-            hi[q] = *reinterpret_cast<const float4*>(Rv + recv_chunk(t, 2 * g + 1));
+            lo[q] = *reinterpret_cast<const float4*>(Rv + recv_chunk(q * Rm + tl, 2 * g));
+            hi[q] = *reinterpret_cast<const float4*>(Rv + recv_chunk(q * Rm + tl, 2 * g + 1));
           }
         }
         float acc[8];
@@ -258,12 +287,49 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] *= fA;
         const uint4 pk = pack_bf16x8(acc);
-        const uint32_t dst = a0 + sw128_chunk(static_cast<int>(rank) * R + i, g);
+        const uint32_t dst = a0 + sw128_chunk(8 * b + r8, g);
         for (int q = 0; q < C; ++q) st_cluster_v4(mapa_shared(dst, static_cast<uint32_t>(q)), pk);
       }
       fence_proxy_async_cluster();
     }
-    cluster_sync();           // every CTA holds the whole A; the receive slots are free again
+    cluster_sync();           // every CTA holds the lower triangle of A; the receive slots are free again
+
+    // ---- upper triangle of A from the lower one, in 8 x 8 blocks (local)
+    if (ok) {
+      for (int it = tid; it < G * (G + 1) / 2; it += SMALL_THREADS) {
+        int bi = 0, rest = it;
+        while (rest >= G - bi) {
+          rest -= G - bi;
+          ++bi;
+        }
+        const int bj = bi + rest;                   // block (bi, bj) on or above the diagonal
+        uint4 src[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) src[r] = *reinterpret_cast<const uint4*>(As + sw128_chunk(8 * bj + r, bi));
+        // src[r] holds A[8 bj + r][8 bi .. 8 bi + 7]; row r' of the result is
+        // column r' of that block (above the diagonal of a diagonal block, the
+        // row's own entries below it are kept).
+#pragma unroll
+        for (int rp = 0; rp < 8; ++rp) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            uint32_t e2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int cp = 2 * h + u;             // column of the result row
+              const uint32_t mine = bf16_at(src[rp], cp);     // A[8 bi + rp][8 bi + cp] (diagonal block)
+              const uint32_t mirr = bf16_at(src[cp], rp);     // A[8 bj + cp][8 bi + rp]
+              e2[u] = (bi == bj && cp <= rp) ? mine : mirr;
+            }
+            w4[h] = e2[0] | (e2[1] << 16);
+          }
+          *reinterpret_cast<uint4*>(As + sw128_chunk(8 * bi + rp, bj)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    __syncthreads();
 
     // ---- A^2 -> TMEM columns [128, 256)
     if (ok) {
