@@ -200,9 +200,6 @@ MUON_API muon_status normuon_update(const muon_batch* batches, int nb, const muo
                            int use_normuon, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream);
 
-/* Reads the error word at workspace offset 0 after synchronizing the stream:
- * 0 = no device-side wait timed out since the word was last cleared (each
- * Newton-Schulz call clears it when it starts). */
 /*
  * muon_momentum_norm without a workspace argument.  The pages have no
  * counterpart: this entry point exists for callers that cannot allocate
@@ -233,7 +230,37 @@ MUON_API muon_status normuon_update(const muon_batch* batches, int nb, const muo
 MUON_API muon_status muon_momentum_norm_noalloc(const muon_batch* batches, int nb, const muon_hparams* hp,
                                                 cudaStream_t stream);
 
+/* Reads the error word at workspace offset 0 after synchronizing the stream:
+ * 0 = no device-side wait timed out since the word was last cleared (each
+ * Newton-Schulz call clears it when it starts). */
 MUON_API muon_status muon_workspace_error(const void* workspace, cudaStream_t stream, int32_t* error_word);
+
+/*
+ * Per-step coefficients for muon_hparams.abc_schedule: the Polar Express
+ * schedule.  The pages name a "production Polar Express" schedule but give
+ * no coefficients; this computes them by the greedy minimax construction of
+ * Amsel, Persson, Musco and Gower, "The Polar Express: Optimal Matrix Sign
+ * Methods and Their Application to the Muon Algorithm" (2025).  Step t
+ * applies the odd quintic p_t(x) = a x + b x^3 + c x^5 minimizing
+ * max |1 - p_t(x)| over the interval [lo_t, hi_t] that holds the singular
+ * values of the normalized input after t steps: [lower, 1] for t = 0, then
+ * the image of the previous interval under the polynomial applied.  With
+ * safety s > 1 the polynomial applied is p_t(x / s) (coefficients a/s,
+ * b/s^3, c/s^5).
+ *
+ *   lower   : bound on the smallest normalized singular value, 0 < lower < 1
+ *   steps   : 1 .. 16
+ *   safety  : 1 <= safety <= 2
+ *   abc_out : host array of 3 * steps floats, (a, b, c) per step
+ *   err_out : optional host array of `steps` doubles: max |1 - p_t| over
+ *             [lo_t, hi_t] of the polynomial applied at step t
+ *
+ * Host computation only (no device work, no GPU needed).  Returns
+ * MUON_INVALID_ARG for arguments out of range and MUON_BAD_SHAPE if the
+ * minimax solve fails; nothing is written then.
+ */
+MUON_API muon_status muon_polar_express_schedule(double lower, int steps, double safety, float* abc_out,
+                                                 double* err_out);
 
 MUON_API const char* muon_status_string(muon_status status);
 

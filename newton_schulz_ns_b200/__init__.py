@@ -20,7 +20,7 @@ from ._capi import MUON_BF16, MUON_F16, MUON_F32, MuonError  # noqa: F401
 
 __all__ = ["Batch", "Hparams", "muon_workspace_size", "muon_momentum_norm", "muon_ns_batched",
            "muon_gram_ns_batched", "normuon_update", "workspace_error", "testing_gemm", "spectral_scale",
-           "ns_flops", "version", "kernel_launches", "muon_momentum_norm_noalloc", "muon_ns_auto_batched", "allocate_workspace", "MuonError", "LIB_PATH"]
+           "ns_flops", "version", "kernel_launches", "muon_momentum_norm_noalloc", "muon_ns_auto_batched", "polar_express_schedule", "allocate_workspace", "MuonError", "LIB_PATH"]
 
 LIB_PATH = _capi.LIB_PATH
 
@@ -36,6 +36,21 @@ def version() -> str:
 def kernel_launches() -> int:
     """Kernels the library has enqueued in this process so far."""
     return int(_capi.lib.muon_kernel_launches())
+
+
+def polar_express_schedule(lower: float = 1e-3, steps: int = 5, safety: float = 1.0):
+    """Per-step (a, b, c) of the Polar Express schedule and each step's max |1 - p| (include/muon_ns.h).
+
+    Host computation in the library; pass the coefficients as
+    ``Hparams(ns_steps=steps, abc_schedule=coeffs)``.
+    """
+    abc = (ctypes.c_float * (3 * steps))()
+    err = (ctypes.c_double * steps)()
+    st = _capi.lib.muon_polar_express_schedule(float(lower), int(steps), float(safety), abc, err)
+    if st != 0:
+        raise MuonError(st, "muon_polar_express_schedule")
+    coeffs = [(abc[3 * t], abc[3 * t + 1], abc[3 * t + 2]) for t in range(steps)]
+    return coeffs, [err[t] for t in range(steps)]
 
 
 def spectral_scale(fan_out: int, fan_in: int, extra: float = 1.0) -> float:

@@ -50,7 +50,7 @@ class MuonHparams(ctypes.Structure):
 EXPORTS = ("muon_workspace_size", "muon_momentum_norm", "muon_ns_batched", "muon_gram_ns_batched",
            "normuon_update", "muon_workspace_error", "muon_status_string", "muon_version",
            "muon_testing_gemm", "muon_kernel_launches", "muon_momentum_norm_noalloc",
-           "muon_testing_bounded_wait", "muon_ns_auto_batched")
+           "muon_testing_bounded_wait", "muon_ns_auto_batched", "muon_polar_express_schedule")
 
 
 def _load() -> ctypes.CDLL:
@@ -84,6 +84,9 @@ def _load() -> ctypes.CDLL:
     lib.muon_kernel_launches.restype = ctypes.c_uint64
     lib.muon_version.argtypes = []
     lib.muon_version.restype = ctypes.c_char_p
+    lib.muon_polar_express_schedule.argtypes = [ctypes.c_double, ctypes.c_int, ctypes.c_double,
+                                                ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_double)]
+    lib.muon_polar_express_schedule.restype = ctypes.c_int
     i64, i32, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_float
     lib.muon_testing_gemm.argtypes = [i32, i32, i32, i32, i32, i32,
                                       P, i64, i64, i32, P, i64, i64, i32, P, i64, i64, i32,

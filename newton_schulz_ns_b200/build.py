@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libmuon_ns.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = [os.path.join(CSRC, "muon_api.cu")]
-DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("ns_gemm.cuh", "ns_small.cuh", "elementwise.cuh", "ptx_sm100.cuh")] + [
+DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("ns_gemm.cuh", "ns_small.cuh", "elementwise.cuh", "ptx_sm100.cuh", "polar_express.hpp")] + [
     os.path.join(INCLUDE, f) for f in ("muon_ns.h", "muon_ns_testing.h")]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

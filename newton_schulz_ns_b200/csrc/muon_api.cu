@@ -23,6 +23,7 @@
 #include "elementwise.cuh"
 #include "ns_gemm.cuh"
 #include "ns_small.cuh"
+#include "polar_express.hpp"
 
 using namespace muon;
 
@@ -826,6 +827,35 @@ muon_status noalloc_scratch(float** out) {
 extern "C" {
 
 const char* muon_version(void) { return "0.1.0"; }
+
+muon_status muon_polar_express_schedule(double lower, int steps, double safety, float* abc_out, double* err_out) {
+  namespace pe = muon::polar_express;
+  if (abc_out == nullptr || !(lower > 0.0 && lower < 1.0) || steps < 1 || steps > 16 || !(safety >= 1.0) ||
+      !(safety <= 2.0))
+    return MUON_INVALID_ARG;
+  float abc[3 * 16];
+  double errs[16];
+  double lo = lower, hi = 1.0;
+  for (int t = 0; t < steps; ++t) {
+    pe::Quintic p;
+    double E = 0.0;
+    if (!pe::minimax_quintic(lo, hi, &p, &E)) return MUON_BAD_SHAPE;
+    const double s = safety;
+    const pe::Quintic q{p.a / s, p.b / (s * s * s), p.c / (s * s * s * s * s)};
+    double mn = 0.0, mx = 0.0;
+    pe::image(q, lo, hi, &mn, &mx);
+    if (!(mn > 0.0) || !std::isfinite(mx)) return MUON_BAD_SHAPE;
+    abc[3 * t] = static_cast<float>(q.a);
+    abc[3 * t + 1] = static_cast<float>(q.b);
+    abc[3 * t + 2] = static_cast<float>(q.c);
+    errs[t] = std::max(std::fabs(1.0 - mn), std::fabs(mx - 1.0));
+    lo = mn;
+    hi = mx;
+  }
+  std::memcpy(abc_out, abc, sizeof(float) * 3 * steps);
+  if (err_out) std::memcpy(err_out, errs, sizeof(double) * steps);
+  return MUON_OK;
+}
 
 uint64_t muon_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 

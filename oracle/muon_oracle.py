@@ -131,6 +131,21 @@ def _orient(U: np.ndarray) -> Tuple[np.ndarray, bool]:
     return U, False
 
 
+def _step_coefs(abc, steps: int):
+    """Per-step (a, b, c): one triple for every step, or one triple per step.
+
+    A per-step schedule is what the Polar Express iteration uses (named in
+    [dion-121] "Validation"); the quintic of the Megatron-Core docs is the
+    same triple at every step.
+    """
+    abc = list(abc)
+    if len(abc) == 3 and not hasattr(abc[0], "__len__"):
+        return [tuple(float(v) for v in abc)] * steps
+    if len(abc) < steps:
+        raise ValueError("schedule shorter than the step count")
+    return [tuple(float(v) for v in t) for t in abc[:steps]]
+
+
 def newton_schulz(U: np.ndarray, steps: int = 5, eps: float = 1e-7,
                   abc: Sequence[float] = QUINTIC_ABC) -> np.ndarray:
     """Standard quintic Newton-Schulz of one slice, result in the slice's orientation.
@@ -138,12 +153,12 @@ def newton_schulz(U: np.ndarray, steps: int = 5, eps: float = 1e-7,
     [ds-8437] "Why it happens": normalize, then iterate on ``X @ X.mT``.
     [mcore-lsm] ``use_syrk``: the two symmetric products are ``A = X X^T`` and
     ``B = b*A + c*A^2``; ``coefficient_type='quintic'``, ``num_ns_steps=5``.
-    Each step then forms ``X <- a*X + B @ X``.
+    Each step then forms ``X <- a*X + B @ X``.  ``abc`` is one (a, b, c) for
+    every step or a per-step schedule.
     """
-    a, b, c = (float(v) for v in abc)
     X, transposed = _orient(U)
     X = frobenius_normalize(X, eps)
-    for _ in range(steps):
+    for a, b, c in _step_coefs(abc, steps):
         A = X @ X.T
         B = b * A + c * (A @ A)
         X = a * X + B @ X
@@ -161,16 +176,16 @@ def gram_newton_schulz(U: np.ndarray, steps: int = 5, eps: float = 1e-7,
     and repeat ``P = a*I + b*A + c*A^2``, ``Q <- P Q``, ``A <- P A P``; the
     result is ``Q X0``.  Because every matrix here is a polynomial in ``G``
     they commute, ``X_k = Q_k X0`` and ``X_k X_k^T = Q_k G Q_k``, so this equals
-    the standard iteration in exact arithmetic.
+    the standard iteration in exact arithmetic (also with a per-step
+    schedule of (a, b, c)).
     """
-    a, b, c = (float(v) for v in abc)
     X0, transposed = _orient(U)
     X0 = frobenius_normalize(X0, eps)
     m = X0.shape[0]
     I = np.eye(m)
     A = X0 @ X0.T
     Q = I.copy()
-    for _ in range(steps):
+    for a, b, c in _step_coefs(abc, steps):
         P = a * I + b * A + c * (A @ A)
         Q = P @ Q
         A = P @ A @ P

@@ -146,3 +146,52 @@ def test_binding_fails_loudly_without_library(tmp_path):
     code = "import sys; sys.path.insert(0, %r); import newton_schulz_ns_b200" % str(tmp_path)
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env)
     assert r.returncode != 0 and "libmuon_ns.so is missing" in r.stderr
+
+
+# ----------------------------------------------------------------- Polar Express schedule (host code)
+
+@pytest.mark.parametrize("lower", [1e-4, 1e-3, 1e-2, 0.1, 0.5])
+def test_polar_express_schedule_matches_lp_oracle(mn, lower):
+    import numpy as np
+    import oracle
+    got, gerr = mn.polar_express_schedule(lower, 8)
+    # Step by step on the library's own intervals: with safety 1 the image of
+    # [lo_t, hi_t] under the minimax quintic is [1 - E_t, 1 + E_t].  (The
+    # recursion itself is ill-conditioned for small `lower`: lo_{t+1} = 1 - E_t
+    # with E_t close to 1, so two solvers 1e-7 apart in E drift apart later.)
+    lo, hi = lower, 1.0
+    for t in range(8):
+        g = np.array(got[t])
+        if hi - lo < 1e-3:
+            w = np.array(oracle.FIXED_POINT_QUINTIC)
+        else:
+            w = np.array(oracle.minimax_quintic_lp(lo, hi)[0])
+        # library: Remez exchange in fp64, stored as float32; oracle: LP on a
+        # 4001-point grid, whose solver tolerance (~1e-9 on E) moves the
+        # coefficients by about that over the interval width cubed (the
+        # conditioning of fitting x, x^3, x^5 on a short interval)
+        tol = 2e-5 + (2e-9 / (hi - lo) ** 3 if hi - lo >= 1e-3 else 0.0)
+        assert np.all(np.abs(g - w) <= tol * np.maximum(1.0, np.abs(w))), (t, g, w)
+        mn_, mx_ = oracle.quintic_image(got[t], lo, hi)
+        assert abs(max(1 - mn_, mx_ - 1) - gerr[t]) <= 1e-5, (t, mn_, mx_, gerr[t])
+        lo, hi = 1.0 - gerr[t], 1.0 + gerr[t]
+    if lower >= 1e-3:
+        # well-conditioned here: the whole recursion agrees too
+        want, werr = oracle.polar_express_lp(lower, 8)
+        assert np.allclose(np.array(got), np.array(want), rtol=1e-4, atol=1e-4)
+        assert np.allclose(gerr, werr, atol=1e-4)
+
+
+def test_polar_express_schedule_safety_and_arguments(mn):
+    import numpy as np
+    (c1,), _ = mn.polar_express_schedule(1e-2, 1, 1.0)
+    (c2,), _ = mn.polar_express_schedule(1e-2, 1, 1.02)
+    s = 1.02
+    assert np.allclose(c2, (c1[0] / s, c1[1] / s ** 3, c1[2] / s ** 5), rtol=1e-6)
+    for bad in [dict(lower=0.0), dict(lower=1.0), dict(steps=0), dict(steps=17), dict(safety=0.99),
+                dict(safety=2.5)]:
+        kw = dict(lower=1e-3, steps=5, safety=1.0)
+        kw.update(bad)
+        with pytest.raises(mn.MuonError) as e:
+            mn.polar_express_schedule(**kw)
+        assert e.value.status == 1      # MUON_INVALID_ARG

@@ -316,3 +316,75 @@ def test_ns_flops_closed_forms():
     tri = orc.ns_flops(m, m, "standard", triangle=True)
     assert full == 30 * m ** 3 and tri == 20 * m ** 3          # one triangle: a third off, square case
     assert orc.ns_flops(256, 1024, "gram") == 256 ** 2 * 1024 * 3 + 17 * 256 ** 3
+
+
+# ----------------------------------------------------------------- Polar Express schedule (LP oracle)
+# The minimax odd quintic for 1 on [lo, hi] is characterized by Chebyshev's
+# alternation theorem: with three free coefficients, the error 1 - p
+# attains its maximum modulus E at four points of alternating sign.  These
+# pins check that property directly, the limit quintic near x = 1, and the
+# interval recursion of the greedy schedule.
+
+def _quintic(coef, x):
+    return coef[0] * x + coef[1] * x ** 3 + coef[2] * x ** 5
+
+
+@pytest.mark.parametrize("lo,hi", [(1e-3, 1.0), (0.1, 1.0), (0.5, 1.2), (0.02, 1.05)])
+def test_polar_express_lp_equioscillates(lo, hi):
+    coef, E = orc.minimax_quintic_lp(lo, hi)
+    x = np.linspace(lo, hi, 400001)
+    e = 1.0 - _quintic(coef, x)
+    assert abs(np.abs(e).max() - E) <= 1e-5 * E
+    # local extrema of e, with the endpoints
+    d = np.diff(e)
+    ext = [0] + [i + 1 for i in range(len(d) - 1) if d[i] * d[i + 1] < 0] + [len(x) - 1]
+    vals = e[ext]
+    big = vals[np.abs(vals) >= E * (1 - 1e-4)]
+    assert len(big) >= 4
+    signs = np.sign(big)
+    assert np.all(signs[1:] != signs[:-1])      # alternating
+
+
+def test_polar_express_lp_narrow_interval_tends_to_fixed_point_quintic():
+    coef, E = orc.minimax_quintic_lp(0.99, 1.01)
+    assert np.allclose(coef, orc.FIXED_POINT_QUINTIC, atol=3e-4)
+    # p(1) = 1, p'(1) = p''(1) = 0 for the limit quintic
+    a, b, c = orc.FIXED_POINT_QUINTIC
+    assert a + b + c == 1.0 and a + 3 * b + 5 * c == 0.0 and 6 * b + 20 * c == 0.0
+
+
+def test_polar_express_lp_schedule_recursion():
+    coeffs, errs = orc.polar_express_lp(1e-3, 6)
+    lo, hi = 1e-3, 1.0
+    for coef, E in zip(coeffs, errs):
+        mn, mx = orc.quintic_image(coef, lo, hi)
+        # equioscillation: the image of the interval is [1 - E, 1 + E]
+        assert abs(mn - (1 - E)) < 1e-5 and abs(mx - (1 + E)) < 1e-5
+        lo, hi = mn, mx
+    assert all(e2 < e1 for e1, e2 in zip(errs, errs[1:]))
+    assert errs[-1] < 1e-3
+
+
+def test_polar_express_lp_safety_scales_the_argument():
+    s = 1.05
+    (c1,), _ = orc.polar_express_lp(1e-2, 1, safety=1.0)
+    (c2,), _ = orc.polar_express_lp(1e-2, 1, safety=s)
+    assert np.allclose(c2, (c1[0] / s, c1[1] / s ** 3, c1[2] / s ** 5), rtol=1e-12)
+
+
+def test_polar_express_schedule_drives_singular_values_into_the_band():
+    # NS with a per-step schedule maps each normalized singular value through
+    # the composed polynomials (odd polynomials act on singular values), so
+    # a matrix whose normalized spectrum lies in [lower, 1] comes out inside
+    # [1 - E_T, 1 + E_T].
+    rng = np.random.default_rng(41)
+    m, n = 24, 40
+    Uo, _ = np.linalg.qr(rng.standard_normal((m, m)))
+    Vo, _ = np.linalg.qr(rng.standard_normal((n, m)))
+    sig = np.geomspace(1.0, 0.05, m)
+    X = (Uo * sig) @ Vo.T
+    lower = sig[-1] / np.linalg.norm(X) * 0.999
+    coeffs, errs = orc.polar_express_lp(lower, 6)
+    O = orc.newton_schulz(X, steps=6, eps=0.0, abc=coeffs)
+    s_out = np.linalg.svd(O, compute_uv=False)
+    assert np.all(np.abs(s_out - 1.0) <= errs[-1] * (1 + 1e-6) + 1e-12)
