@@ -66,6 +66,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scale-down", type=int, default=1, help="divide every parameter count (smoke runs only)")
+    ap.add_argument("--coefficients", choices=["quintic", "polar-express"], default="quintic",
+                    help="quintic: (3.4445, -4.7750, 2.0315) at every step; polar-express: the greedy "
+                         "minimax schedule for singular values in [--pe-lower, 1]")
+    ap.add_argument("--pe-lower", type=float, default=1e-3)
     return ap.parse_args()
 
 
@@ -142,7 +146,13 @@ def default_variant(wl):
 
 # ----------------------------------------------------------------------------- CPU oracle (baseline)
 
-def oracle_sample(wl, variant, budget_s=30.0):
+def coefficients_desc(args):
+    if args.coefficients == "polar-express":
+        return f"polar-express (greedy minimax quintics, singular values in [{args.pe_lower:g}, 1])"
+    return "quintic (3.4445, -4.7750, 2.0315) at every step"
+
+
+def oracle_sample(wl, variant, budget_s=30.0, abc=None):
     """Runs the fp64 oracle's full step on the workload's sample; returns (flops, slices, seconds, cores, desc)."""
     import numpy as np
     import threadpoolctl
@@ -166,7 +176,8 @@ def oracle_sample(wl, variant, budget_s=30.0):
                 M = np.zeros_like(G)
                 v = np.zeros(G.shape[:2]) if wl.normuon else None
                 oracle.muon_step_slices(G, M, W, v, mu=wl.momentum, nesterov=wl.nesterov, ns_eps=wl.ns_eps,
-                                        ns_steps=wl.ns_steps, variant=slice_variant(g.slice_rows, g.cols, variant),
+                                        ns_steps=wl.ns_steps, abc=abc if abc is not None else oracle.QUINTIC_ABC,
+                                        variant=slice_variant(g.slice_rows, g.cols, variant),
                                         normuon=wl.normuon,
                                         beta2=wl.beta2, nor_eps=wl.nor_eps, lr=wl.lr,
                                         weight_decay=wl.weight_decay,
@@ -184,7 +195,7 @@ def oracle_sample(wl, variant, budget_s=30.0):
 
 # ----------------------------------------------------------------------------- GPU state
 
-def build_state(wl, variant, dev):
+def build_state(wl, variant, dev, schedule=None):
     import torch
     import newton_schulz_ns_b200 as mn
     import workloads
@@ -209,6 +220,7 @@ def build_state(wl, variant, dev):
                      lr_scale=mn.spectral_scale(g.rows, g.cols))
         groups.append(b)
     hp = mn.Hparams(mu=wl.momentum, nesterov=wl.nesterov, ns_eps=wl.ns_eps, ns_steps=wl.ns_steps,
+                    abc_schedule=schedule,
                     beta2=wl.beta2, nor_eps=wl.nor_eps, lr=wl.lr, weight_decay=wl.weight_decay)
     ws = mn.allocate_workspace(groups, -1, dev)
     return groups, hp, ws
@@ -304,7 +316,10 @@ def run_ours(args, wl, variant, rank, world, local_rank):
 
     dev = f"cuda:{local_rank}"
     torch.cuda.set_device(dev)
-    groups, hp, ws = build_state(wl, variant, dev)
+    schedule = None
+    if args.coefficients == "polar-express":
+        schedule = mn.polar_express_schedule(args.pe_lower, wl.ns_steps)[0]
+    groups, hp, ws = build_state(wl, variant, dev, schedule)
     if variant == "auto":
         def ns_fn(g, h, w, s):
             mn.muon_ns_auto_batched(g, h, w, AUTO_GRAM_RATIO, s)
@@ -434,7 +449,8 @@ def run_ours(args, wl, variant, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch Philox on the device)",
-        "config": {"workload": DESCRIPTIONS[wl.key], "key": wl.key, "variant": variant, "slices": slices,
+        "config": {"workload": DESCRIPTIONS[wl.key], "key": wl.key, "variant": variant,
+                   "coefficients": coefficients_desc(args), "slices": slices,
                    "ns_flop_per_step": ns_flop, "l2": "inputs larger than L2 (126 MB), no flush",
                    "parallelism": f"replicas x{world} (no exchange)"},
         "pct_bf16_peak": round(100 * value / world / peak_s, 2),
@@ -465,7 +481,7 @@ def run_ours(args, wl, variant, rank, world, local_rank):
                               "from pinned host memory on a second stream (overlapping the previous shape's "
                               "optimizer work) and its per-slice norms read back D2H, all inside the timed region"}
     if world == 1 and not args.no_cpu_baseline:
-        flops, sl, dt, cores, desc = oracle_sample(wl, variant)
+        flops, sl, dt, cores, desc = oracle_sample(wl, variant, abc=oracle_schedule(args, wl))
         out["cpu_baseline"] = {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
                                "kind": "oracle", "sample": desc, "seconds": round(dt, 2),
                                "matrices_per_s": round(sl / dt, 4)}
@@ -474,14 +490,23 @@ def run_ours(args, wl, variant, rank, world, local_rank):
 
 # ----------------------------------------------------------------------------- reference arm
 
+def oracle_schedule(args, wl):
+    """The oracle's own coefficients for the run (its linear-programming schedule for Polar Express)."""
+    if args.coefficients != "polar-express":
+        return None
+    import oracle
+    return oracle.polar_express_lp(args.pe_lower, wl.ns_steps)[0]
+
+
 def run_reference(args, wl, variant):
     peaks, _ = load_peaks()
+    abc = oracle_schedule(args, wl)
     budget = max(5.0, 60.0 / max(1, args.steps + args.warmup))
     per_step = []
     flops = sl = 0
     cores, desc = 1, ""
     for k in range(args.warmup + args.steps):
-        f, s, dt, cores, desc = oracle_sample(wl, variant, budget)
+        f, s, dt, cores, desc = oracle_sample(wl, variant, budget, abc=abc)
         if k >= args.warmup:
             per_step.append(dt)
             flops, sl = f, s
@@ -492,7 +517,7 @@ def run_reference(args, wl, variant):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sec / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": DESCRIPTIONS[wl.key], "key": wl.key, "variant": variant,
-                   "sample": desc},
+                   "coefficients": coefficients_desc(args), "sample": desc},
         "pct_bf16_peak": round(100 * value / peaks.get("bf16_tflops_sustained", 1400.0), 6),
         "matrices_per_s": round(sl * args.steps / sec, 4),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",

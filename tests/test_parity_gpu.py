@@ -491,3 +491,25 @@ def test_ns_maximum_size_closed_form(mn, tall):
     assert err < 1e-2, err
     del ws
     torch.cuda.empty_cache()
+
+
+# ----------------------------------------------------------------- Polar Express schedule
+
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+@pytest.mark.parametrize("shape", [(128, 1024), (300, 200), (512, 1536)])
+def test_ns_polar_express_schedule(mn, variant, shape):
+    # The oracle's own schedule (linear programming) drives both sides: fused
+    # small-side kernel (128 x 1024), GEMM path tall (300 x 200) and wide.
+    coeffs, errs = oracle.polar_express_lp(1e-3, 5)
+    r, c = shape
+    U = _seeded(2, r, c, 60 + r, torch.bfloat16)
+    b = _ns_batch(mn, U)
+    _run_ns(mn, [b], variant, mn.Hparams(ns_steps=5, abc_schedule=coeffs))
+    ref = oracle.ns_batched(f64(U), variant, steps=5, abc=coeffs)
+    got = f64(b.ns_out)
+    for i in range(2):
+        assert rel(got[i], ref[i]) < NS_TOL, (variant, shape, i, rel(got[i], ref[i]))
+        # Gaussian slices: every normalized singular value is above 1e-3, so
+        # the exact result lies in [1 - E_5, 1 + E_5]; bf16 adds a little.
+        s_out = np.linalg.svd(got[i], compute_uv=False)
+        assert np.all(np.abs(s_out - 1.0) <= errs[-1] + 0.05), (s_out.min(), s_out.max(), errs[-1])
