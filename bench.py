@@ -70,6 +70,7 @@ def parse():
                     help="quintic: (3.4445, -4.7750, 2.0315) at every step; polar-express: the greedy "
                          "minimax schedule for singular values in [--pe-lower, 1]")
     ap.add_argument("--pe-lower", type=float, default=1e-3)
+    ap.add_argument("--pe-safety", type=float, default=1.01)
     return ap.parse_args()
 
 
@@ -148,7 +149,8 @@ def default_variant(wl):
 
 def coefficients_desc(args):
     if args.coefficients == "polar-express":
-        return f"polar-express (greedy minimax quintics, singular values in [{args.pe_lower:g}, 1])"
+        return (f"polar-express (greedy minimax quintics, singular values in [{args.pe_lower:g}, 1], "
+                f"safety {args.pe_safety:g})")
     return "quintic (3.4445, -4.7750, 2.0315) at every step"
 
 
@@ -318,7 +320,7 @@ def run_ours(args, wl, variant, rank, world, local_rank):
     torch.cuda.set_device(dev)
     schedule = None
     if args.coefficients == "polar-express":
-        schedule = mn.polar_express_schedule(args.pe_lower, wl.ns_steps)[0]
+        schedule = mn.polar_express_schedule(args.pe_lower, wl.ns_steps, args.pe_safety)[0]
     groups, hp, ws = build_state(wl, variant, dev, schedule)
     if variant == "auto":
         def ns_fn(g, h, w, s):
@@ -495,7 +497,7 @@ def oracle_schedule(args, wl):
     if args.coefficients != "polar-express":
         return None
     import oracle
-    return oracle.polar_express_lp(args.pe_lower, wl.ns_steps)[0]
+    return oracle.polar_express_lp(args.pe_lower, wl.ns_steps, args.pe_safety)[0]
 
 
 def run_reference(args, wl, variant):

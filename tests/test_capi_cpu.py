@@ -154,7 +154,7 @@ def test_binding_fails_loudly_without_library(tmp_path):
 def test_polar_express_schedule_matches_lp_oracle(mn, lower):
     import numpy as np
     import oracle
-    got, gerr = mn.polar_express_schedule(lower, 8)
+    got, gerr = mn.polar_express_schedule(lower, 8, safety=1.0)
     # Step by step on the library's own intervals: with safety 1 the image of
     # [lo_t, hi_t] under the minimax quintic is [1 - E_t, 1 + E_t].  (The
     # recursion itself is ill-conditioned for small `lower`: lo_{t+1} = 1 - E_t

@@ -500,7 +500,9 @@ def test_ns_maximum_size_closed_form(mn, tall):
 def test_ns_polar_express_schedule(mn, variant, shape):
     # The oracle's own schedule (linear programming) drives both sides: fused
     # small-side kernel (128 x 1024), GEMM path tall (300 x 200) and wide.
-    coeffs, errs = oracle.polar_express_lp(1e-3, 5)
+    # Safety 1.01, as bf16 arithmetic needs (with 1.0 a numpy model of bf16
+    # storage is already 0.13 away from fp64 on the 128 x 1024 slice).
+    coeffs, errs = oracle.polar_express_lp(1e-3, 5, safety=1.01)
     r, c = shape
     U = _seeded(2, r, c, 60 + r, torch.bfloat16)
     b = _ns_batch(mn, U)
