@@ -80,6 +80,8 @@ muon_status device_setup(int* sms_out, int* pair_units_out = nullptr) {
           cudaFuncSetAttribute(ns_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                GemmCfg<2>::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SMALL_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(ns_small_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SMALL_SMEM_BYTES) != cudaSuccess) {
         d.ready = false;
         return MUON_CUDA_ERROR;
@@ -597,7 +599,7 @@ bool small_eligible(const muon_batch& b) {
   return sp.C <= SMALL_MAX_CLUSTER && sp.w <= SMALL_MAX_W;
 }
 
-muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const float* sumsq, int* err,
+muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const float* sumsq, int* err, bool gram,
                          cudaStream_t stream) {
   const SmallSplit sp = small_split(b.cols);
   SmallParams P;
@@ -620,6 +622,7 @@ muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const floa
     P.b[k] = cf.b;
     P.c[k] = cf.c;
   }
+  P.kappa = kGramScale;
   P.err = err;
   P.timeout_ns = kWaitLimitNs;
   constexpr int64_t kMaxGridY = 65535;
@@ -637,7 +640,7 @@ muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const floa
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, ns_small_kernel, P) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, gram ? ns_small_gram_kernel : ns_small_kernel, P) != cudaSuccess) {
       (void)cudaGetLastError();
       return MUON_CUDA_ERROR;
     }
@@ -984,7 +987,7 @@ muon_status ns_standard_impl(const muon_batch* batches, int nb, const muon_hpara
   for (int i = 0; i < nb; ++i) {
     if (batch_empty(batches[i]) || !small_eligible(batches[i])) continue;
     fused[i] = 1;
-    if ((st = launch_small(batches[i], hp, sumsq[i], err, stream)) != MUON_OK) return st;
+    if ((st = launch_small(batches[i], hp, sumsq[i], err, false, stream)) != MUON_OK) return st;
   }
   const int S = hp->ns_steps;
   for (int it = 0; it < S; ++it) {
@@ -1037,12 +1040,18 @@ muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* 
   const int S = hp->ns_steps;
   const float kap = kGramScale;
 
+  std::vector<char> fused(nb, 0);
+  for (int i = 0; i < nb; ++i) {
+    if (batch_empty(batches[i]) || !small_eligible(batches[i])) continue;
+    fused[i] = 1;
+    if ((st = launch_small(batches[i], hp, sumsq[i], err, true, stream)) != MUON_OK) return st;
+  }
   // G: kappa * s^2 * X X^T (short side) in fp16.
   {
     std::vector<ProblemSpec> g;
     for (int i = 0; i < nb; ++i) {
       const muon_batch& b = batches[i];
-      if (batch_empty(b)) continue;
+      if (batch_empty(b) || fused[i]) continue;
       const NsBatchWs& w = L.nsb[i];
       g.push_back(syrk_spec(b, view_mat(b, b.ns_in), ws + w.off[0], w.ldm, w.bsm, 1, kap, 2, sumsq[i], hp->ns_eps));
     }
@@ -1057,7 +1066,7 @@ muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* 
     int qnext = qcur;
     for (int i = 0; i < nb; ++i) {
       const muon_batch& b = batches[i];
-      if (batch_empty(b)) continue;
+      if (batch_empty(b) || fused[i]) continue;
       const NsBatchWs& w = L.nsb[i];
       const int m = static_cast<int>(std::min(b.rows, b.cols));
       const int sl = static_cast<int>(b.n);
@@ -1089,7 +1098,7 @@ muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* 
     std::vector<ProblemSpec> o;
     for (int i = 0; i < nb; ++i) {
       const muon_batch& b = batches[i];
-      if (batch_empty(b)) continue;
+      if (batch_empty(b) || fused[i]) continue;
       const NsBatchWs& w = L.nsb[i];
       const int m = static_cast<int>(std::min(b.rows, b.cols));
       const Mat Q{ws + w.off[qcur], m, m, w.ldm, w.bsm, b.n, 0};

@@ -27,6 +27,14 @@
 //     need no other CTA's data, and writes them back over X;
 //   * after the last step the resident columns go to ns_out by TMA.
 //
+// The Gram form (ns_small_gram_kernel) runs the same exchange once, for
+// G = kappa s^2 X0 X0^T in fp16 (kappa = 2^14, as on the GEMM path), and then
+// iterates on the m x m side inside every CTA of the cluster (redundantly:
+// each product is 128^3): P = a I + (b/kappa) A + (c/kappa^2) A^2,
+// Q <- P Q, A <- P (P A), all fp16 with the symmetric results mirrored from
+// their lower triangles; the last Q is rounded to bf16 and O = s Q X0 is
+// formed on the resident columns.
+//
 // Precision follows the GEMM path: bf16 operands, fp32 accumulation, A, B
 // and X rounded to bf16 between products.  Operand layouts are the 128-byte
 // swizzled tiles TMA writes (64 columns x 128 rows per 16 KB block): X is
@@ -40,6 +48,7 @@
 // finish too.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 #include "ptx_sm100.cuh"
 
@@ -70,6 +79,7 @@ struct __align__(64) SmallParams {
   int slice0;                // first slice of this launch
   int steps;
   int tma_store;             // n is a multiple of 8: whole 16-byte chunks, TMA clips exactly
+  float kappa;               // Gram form: A is kept as kappa * A in fp16
   float a[SMALL_MAX_STEPS], b[SMALL_MAX_STEPS], c[SMALL_MAX_STEPS];
   int* err;
   unsigned long long timeout_ns;
@@ -102,6 +112,27 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& u, float (&f)[8]) {
   }
 }
 
+__device__ __forceinline__ uint4 pack_f16x8(const float (&o)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    const __half2 v = __floats2half2_rn(o[2 * h], o[2 * h + 1]);
+    w[h] = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ void unpack_f16x8(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    const __half2 v = *reinterpret_cast<const __half2*>(&w[h]);
+    const float2 t = __half22float2(v);
+    f[2 * h] = t.x;
+    f[2 * h + 1] = t.y;
+  }
+}
+
 // 16-bit element e (0..7, a compile-time constant after unrolling) of 8 packed values.
 __device__ __forceinline__ uint32_t bf16_at(const uint4& u, int e) {
   const uint32_t word = (e >> 1) == 0 ? u.x : (e >> 1) == 1 ? u.y : (e >> 1) == 2 ? u.z : u.w;
@@ -125,7 +156,133 @@ __device__ __forceinline__ void tmem_ld_64(uint32_t taddr, uint32_t (&v)[64]) {
   tmem_ld_wait();
 }
 
-__global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid_constant__ SmallParams P) {
+// Fills the upper triangle of the symmetric m8 x m8 corner (G = m8 / 8 blocks
+// of 8) of a 16-bit SW128 matrix from its lower triangle, in 8 x 8 blocks.
+__device__ __forceinline__ void mirror_upper(uint8_t* M, int G, int tid) {
+  for (int it = tid; it < G * (G + 1) / 2; it += SMALL_THREADS) {
+    int bi = 0, rest = it;
+    while (rest >= G - bi) {
+      rest -= G - bi;
+      ++bi;
+    }
+    const int bj = bi + rest;                       // block (bi, bj) on or above the diagonal
+    uint4 src[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) src[r] = *reinterpret_cast<const uint4*>(M + sw128_chunk(8 * bj + r, bi));
+    // src[r] holds M[8 bj + r][8 bi .. 8 bi + 7]; row r' of the result is
+    // column r' of that block (above the diagonal of a diagonal block, the
+    // row's own entries below it are kept).
+#pragma unroll
+    for (int rp = 0; rp < 8; ++rp) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        uint32_t e2[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int cp = 2 * h + u;                 // column of the result row
+          const uint32_t mine = bf16_at(src[rp], cp);     // M[8 bi + rp][8 bi + cp] (diagonal block)
+          const uint32_t mirr = bf16_at(src[cp], rp);     // M[8 bj + cp][8 bi + rp]
+          e2[u] = (bi == bj && cp <= rp) ? mine : mirr;
+        }
+        w4[h] = e2[0] | (e2[1] << 16);
+      }
+      *reinterpret_cast<uint4*>(M + sw128_chunk(8 * bi + rp, bj)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+  }
+  fence_proxy_async_smem();
+}
+
+// D[tmem, 128 x 128] = X Y^T over K = 128, both 128 x 128 K-major SW128
+// operands in shared memory; issued by one thread, completion on `bar`.
+__device__ __forceinline__ void issue_square(uint32_t d_tmem, uint32_t x0, uint32_t y0, uint32_t idesc, uint64_t* bar) {
+  fence_proxy_async_smem();
+  tc_fence_after();
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t xd = smem_desc_sw128(x0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+    const uint64_t yd = smem_desc_sw128(y0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+    tc_mma_f16(d_tmem, xd, yd, idesc, kk > 0 ? 1u : 0u);
+  }
+  tc_commit(bar);
+}
+
+// Epilogue of a 128 x 128 product for row `row` (< m8), columns
+// [64 half, 64 half + 64): out = alpha acc + beta D + gamma [row == col < m],
+// rounded once to fp16 or bf16.  D may be `out` itself (read first).
+__device__ __forceinline__ void epi_square(uint32_t taddr, int row, int half, int m8, int m, float alpha, float beta,
+                                           const uint8_t* D, bool d_f16, float gamma, uint8_t* out, bool out_f16) {
+  uint32_t v[64];
+  tmem_ld_64(taddr + static_cast<uint32_t>(half * 64), v);
+  if (row >= m8) return;
+  uint4 dv[8];
+  if (D != nullptr) {
+#pragma unroll
+    for (int h = 0; h < 8; ++h) dv[h] = *reinterpret_cast<const uint4*>(D + sw128_chunk(row, half * 8 + h));
+  }
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    float df[8], o[8];
+    if (D != nullptr) {
+      if (d_f16)
+        unpack_f16x8(dv[h], df);
+      else
+        unpack_bf16x8(dv[h], df);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float x = alpha * __uint_as_float(v[h * 8 + e]);
+      if (D != nullptr) x += beta * df[e];
+      const int col = half * 64 + h * 8 + e;
+      if (gamma != 0.0f && col == row && row < m) x += gamma;
+      o[e] = x;
+    }
+    *reinterpret_cast<uint4*>(out + sw128_chunk(row, half * 8 + h)) = out_f16 ? pack_f16x8(o) : pack_bf16x8(o);
+  }
+}
+
+// Epilogue of the product on the resident columns for row `row`, columns
+// [half w/2, half w/2 + w/2): X <- f (acc + a X), in place, bf16.
+__device__ __forceinline__ void epi_columns(uint32_t taddr, int row, int half, int w, int m8, float a, float f,
+                                            uint8_t* Xs) {
+  const int hw = w >> 1;
+  const int cend = half * hw + hw;
+#pragma unroll 1
+  for (int c0 = half * hw; c0 < cend; c0 += 64) {
+    const bool two = c0 + 64 <= cend;               // warp-uniform: 64 or 32 columns
+    uint32_t v[64];
+    if (two) {
+      tmem_ld_64(taddr + static_cast<uint32_t>(c0), v);
+    } else {
+      tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c0), *reinterpret_cast<uint32_t(*)[32]>(v));
+      tmem_ld_wait();
+    }
+    if (row < m8) {
+      const int nch = two ? 8 : 4;
+      uint4 xv[8];
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+        if (h < nch) xv[h] = *reinterpret_cast<const uint4*>(Xs + sw128_chunk(row, (c0 >> 3) + h));
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        if (h < nch) {
+          float xf[8], o[8];
+          unpack_bf16x8(xv[h], xf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float x = __uint_as_float(v[h * 8 + e]);
+            x += a * xf[e];
+            o[e] = x * f;
+          }
+          *reinterpret_cast<uint4*>(Xs + sw128_chunk(row, (c0 >> 3) + h)) = pack_bf16x8(o);
+        }
+      }
+    }
+  }
+  fence_proxy_async_smem();
+}
+
+template <bool GRAM>
+__device__ __forceinline__ void ns_small_body(const SmallParams& P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -210,7 +367,8 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
   const uint32_t rv0 = smem_u32(Rv);
   const uint32_t a0 = smem_u32(As);
 
-  for (int k = 0; k < P.steps; ++k) {
+  const int outer = GRAM ? 1 : P.steps;
+  for (int k = 0; k < outer; ++k) {
     const float ca = P.a[k], cb = P.b[k], cc = P.c[k];
     // ---- partial X_r X_r^T -> TMEM columns [0, 128)
     if (ok) {
@@ -253,7 +411,7 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
     //      the slots in rank order, pushed to every CTA (the diagonal block's
     //      upper half carries unsent entries; the mirror below replaces it)
     if (ok) {
-      const float fA = (k == 0) ? s * s : 1.0f;
+      const float fA = GRAM ? P.kappa * (s * s) : (k == 0) ? s * s : 1.0f;
       int items = 0;
       for (int lb = 0; lb < kb && rank * kb + lb < G; ++lb) items += 8 * (unfold(rank * kb + lb) + 1);
       for (int it = tid; it < items; it += SMALL_THREADS) {
@@ -286,7 +444,7 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] *= fA;
-        const uint4 pk = pack_bf16x8(acc);
+        const uint4 pk = GRAM ? pack_f16x8(acc) : pack_bf16x8(acc);
         const uint32_t dst = a0 + sw128_chunk(8 * b + r8, g);
         for (int q = 0; q < C; ++q) st_cluster_v4(mapa_shared(dst, static_cast<uint32_t>(q)), pk);
       }
@@ -294,42 +452,10 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
     }
     cluster_sync();           // every CTA holds the lower triangle of A; the receive slots are free again
 
-    // ---- upper triangle of A from the lower one, in 8 x 8 blocks (local)
-    if (ok) {
-      for (int it = tid; it < G * (G + 1) / 2; it += SMALL_THREADS) {
-        int bi = 0, rest = it;
-        while (rest >= G - bi) {
-          rest -= G - bi;
-          ++bi;
-        }
-        const int bj = bi + rest;                   // block (bi, bj) on or above the diagonal
-        uint4 src[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) src[r] = *reinterpret_cast<const uint4*>(As + sw128_chunk(8 * bj + r, bi));
-        // src[r] holds A[8 bj + r][8 bi .. 8 bi + 7]; row r' of the result is
-        // column r' of that block (above the diagonal of a diagonal block, the
-        // row's own entries below it are kept).
-#pragma unroll
-        for (int rp = 0; rp < 8; ++rp) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            uint32_t e2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int cp = 2 * h + u;             // column of the result row
-              const uint32_t mine = bf16_at(src[rp], cp);     // A[8 bi + rp][8 bi + cp] (diagonal block)
-              const uint32_t mirr = bf16_at(src[cp], rp);     // A[8 bj + cp][8 bi + rp]
-              e2[u] = (bi == bj && cp <= rp) ? mine : mirr;
-            }
-            w4[h] = e2[0] | (e2[1] << 16);
-          }
-          *reinterpret_cast<uint4*>(As + sw128_chunk(8 * bi + rp, bj)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        }
-      }
-      fence_proxy_async_smem();
-    }
+    // ---- upper triangle of A from the lower one (local)
+    if (ok) mirror_upper(As, G, tid);
     __syncthreads();
+    if (GRAM) break;
 
     // ---- A^2 -> TMEM columns [128, 256)
     if (ok) {
@@ -344,28 +470,10 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
       }
       ok = wait_mma();
     }
-    // ---- B = c A^2 + b A, in place over A (row `row`, columns [64 half, 64 half + 64))
+    // ---- B = c A^2 + b A, in place over A
     if (ok) {
       tc_fence_after();
-      uint32_t v[64];
-      tmem_ld_64(tmem + tlane + 128u + static_cast<uint32_t>(half * 64), v);
-      if (row < m8) {
-        uint4 av[8];
-#pragma unroll
-        for (int h = 0; h < 8; ++h) av[h] = *reinterpret_cast<const uint4*>(As + sw128_chunk(row, half * 8 + h));
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          float af[8], o[8];
-          unpack_bf16x8(av[h], af);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float x = cc * __uint_as_float(v[h * 8 + e]);
-            x += cb * af[e];
-            o[e] = x;
-          }
-          *reinterpret_cast<uint4*>(As + sw128_chunk(row, half * 8 + h)) = pack_bf16x8(o);
-        }
-      }
+      epi_square(tmem + tlane + 128u, row, half, m8, P.m, cc, cb, As, false, 0.0f, As, false);
       fence_proxy_async_smem();
     }
     tc_fence_before();
@@ -389,45 +497,92 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
       }
       ok = wait_mma();
     }
-    // ---- X <- f * (B X + a X), in place (row `row`, columns [half w/2, half w/2 + w/2))
+    // ---- X <- f * (B X + a X), in place
     if (ok) {
       tc_fence_after();
-      const float fX = (k == 0) ? s : 1.0f;
-      const int hw = w >> 1;
-      const int cend = half * hw + hw;
-#pragma unroll 1
-      for (int c0 = half * hw; c0 < cend; c0 += 64) {
-        const bool two = c0 + 64 <= cend;           // warp-uniform: 64 or 32 columns
-        uint32_t v[64];
-        if (two) {
-          tmem_ld_64(tmem + tlane + static_cast<uint32_t>(c0), v);
-        } else {
-          tmem_ld_32x32b_x32(tmem + tlane + static_cast<uint32_t>(c0), *reinterpret_cast<uint32_t(*)[32]>(v));
-          tmem_ld_wait();
-        }
-        if (row < m8) {
-          const int nch = two ? 8 : 4;
-          uint4 xv[8];
-#pragma unroll
-          for (int h = 0; h < 8; ++h)
-            if (h < nch) xv[h] = *reinterpret_cast<const uint4*>(Xs + sw128_chunk(row, (c0 >> 3) + h));
-#pragma unroll
-          for (int h = 0; h < 8; ++h) {
-            if (h < nch) {
-              float xf[8], o[8];
-              unpack_bf16x8(xv[h], xf);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                float x = __uint_as_float(v[h * 8 + e]);
-                x += ca * xf[e];
-                o[e] = x * fX;
-              }
-              *reinterpret_cast<uint4*>(Xs + sw128_chunk(row, (c0 >> 3) + h)) = pack_bf16x8(o);
-            }
-          }
+      epi_columns(tmem + tlane, row, half, w, m8, ca, (k == 0) ? s : 1.0f, Xs);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  if (GRAM) {
+    // ---- m x m iteration (fp16, kappa-scaled A), every CTA of the cluster alike
+    uint8_t* Pb = Rv;                               // P (and, on step 0, the first Q)
+    uint8_t* Qb = Rv + SMALL_A_BYTES;               // Q
+    for (int i = tid; i < 2 * SMALL_A_BYTES / 16; i += SMALL_THREADS)
+      reinterpret_cast<uint4*>(Rv)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+    __syncthreads();
+    const uint32_t idesc_h = mma_idesc_f16(0, 0, 0, 128, 128);
+    const float kap = P.kappa;
+    for (int k = 0; k < P.steps && ok; ++k) {
+      const bool last = k == P.steps - 1;
+      uint8_t* Pd = (k == 0) ? Qb : Pb;             // Q_1 = P_1
+      // P = a I + (b / kappa) A + (c / kappa^2) A^2; bf16 when it is the final Q
+      if (tid == 0) issue_square(tmem, a0, a0, idesc_h, &bars[1]);
+      ok = wait_mma();
+      if (!ok) break;
+      tc_fence_after();
+      epi_square(tmem + tlane, row, half, m8, P.m, P.c[k] / (kap * kap), P.b[k] / kap, As, true, P.a[k], Pd,
+                 !(k == 0 && last));
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      mirror_upper(Pd, G, tid);
+      __syncthreads();
+      if (k > 0) {
+        // Q <- P Q, bf16 when last
+        if (tid == 0) issue_square(tmem, smem_u32(Pb), smem_u32(Qb), idesc_h, &bars[1]);
+        ok = wait_mma();
+        if (!ok) break;
+        tc_fence_after();
+        epi_square(tmem + tlane, row, half, m8, P.m, 1.0f, 0.0f, nullptr, false, 0.0f, Qb, !last);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        mirror_upper(Qb, G, tid);
+        __syncthreads();
+      }
+      if (!last) {
+        // R = P A, then A <- P R (fp16, each over A in place once its product is done)
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (tid == 0) issue_square(tmem, smem_u32(Pd), a0, idesc_h, &bars[1]);
+          ok = wait_mma();
+          if (!ok) break;
+          tc_fence_after();
+          epi_square(tmem + tlane, row, half, m8, P.m, 1.0f, 0.0f, nullptr, false, 0.0f, As, true);
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncthreads();
+          mirror_upper(As, G, tid);
+          __syncthreads();
         }
       }
-      fence_proxy_async_smem();
+    }
+    // ---- O = s Q X0 on the resident columns (Q in bf16)
+    if (ok) {
+      if (tid == 0) {
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t q0 = smem_u32(Qb);
+        const uint32_t x0 = smem_u32(Xs);
+        for (int nc = 0; nc < w; nc += 256) {
+          const int N = min(256, w - nc);
+          const uint32_t idesc = mma_idesc_f16(1, 0, 1, 128, static_cast<uint32_t>(N));
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(x0 + (nc >> 6) * SMALL_BLK + kk * 16 * 128, SMALL_BLK, 1024);
+            tc_mma_f16(tmem + static_cast<uint32_t>(nc), ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+        }
+        tc_commit(&bars[1]);
+      }
+      ok = wait_mma();
+    }
+    if (ok) {
+      tc_fence_after();
+      epi_columns(tmem + tlane, row, half, w, m8, 0.0f, s, Xs);
     }
     tc_fence_before();
     __syncthreads();
@@ -473,6 +628,14 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
   __syncthreads();
   cluster_sync();             // no CTA leaves while a peer may still address its shared memory
   if (warp == 0) tmem_dealloc(tmem, ncols);
+}
+
+__global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid_constant__ SmallParams P) {
+  ns_small_body<false>(P);
+}
+
+__global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_gram_kernel(const __grid_constant__ SmallParams P) {
+  ns_small_body<true>(P);
 }
 
 }  // namespace muon

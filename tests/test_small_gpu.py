@@ -4,6 +4,8 @@ Slices with rows <= cols, rows <= 128 and cols <= 4096 (the per-head
 [32, 128, 4096] batch, the conv megabatch [16, 64, 576]) run the whole
 iteration in one clustered launch: each CTA keeps a column block of X in
 shared memory and the cluster sums X X^T over distributed shared memory.
+Both forms: the standard one exchanges X X^T at every step; the Gram one
+exchanges X0 X0^T once and iterates on the m x m side in every CTA.
 The shapes below cover every cluster split the planner picks (1 to 8 CTAs,
 64 to 512 columns each), ragged last blocks, CTAs that hold only padding,
 and short sides from 1 to 128.  Bars: 3e-2 relative Frobenius error against
@@ -52,16 +54,17 @@ def _seeded(n, r, c, seed, std=1.0):
     return t
 
 
-def _ns(mn, U, hp=None, fused=True):
+def _ns(mn, U, hp=None, fused=True, variant="standard"):
     n, r, c = U.shape
     base, out = _padded(n, r, c, torch.bfloat16, float("nan"))
     b = mn.Batch(n, r, c, ns_in=U, ns_out=out)
-    ws = mn.allocate_workspace([b], 1)
+    ws = mn.allocate_workspace([b], 1 if variant == "standard" else 2)
+    fn = mn.muon_ns_batched if variant == "standard" else mn.muon_gram_ns_batched
     old = os.environ.get("MUON_NS_FUSED_SMALL")
     os.environ["MUON_NS_FUSED_SMALL"] = "1" if fused else "0"
     try:
         before = mn.kernel_launches()
-        mn.muon_ns_batched([b], hp or mn.Hparams(), ws)
+        fn([b], hp or mn.Hparams(), ws)
         launches = mn.kernel_launches() - before
         torch.cuda.synchronize()
     finally:
@@ -89,13 +92,14 @@ SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("variant", ["standard", "gram"])
 @pytest.mark.parametrize("shape", SHAPES)
-def test_fused_small_matches_oracle(mn, shape):
+def test_fused_small_matches_oracle(mn, shape, variant):
     r, c = shape
     U = _seeded(3, r, c, 500 + r + c)
-    base, out, launches = _ns(mn, U)
+    base, out, launches = _ns(mn, U, variant=variant)
     assert launches <= 3      # norms (2) + one fused launch
-    ref = oracle.ns_batched(f64(U), "standard")
+    ref = oracle.ns_batched(f64(U), variant)
     got = f64(out)
     for i in range(3):
         assert rel(got[i], ref[i]) < NS_TOL, (shape, i, rel(got[i], ref[i]))
@@ -104,14 +108,15 @@ def test_fused_small_matches_oracle(mn, shape):
     assert torch.isnan(pad.float()).all()
 
 
+@pytest.mark.parametrize("variant", ["standard", "gram"])
 @pytest.mark.parametrize("shape", [(64, 576), (128, 4096), (100, 1000)])
-def test_fused_small_agrees_with_gemm_path(mn, shape):
+def test_fused_small_agrees_with_gemm_path(mn, shape, variant):
     r, c = shape
     U = _seeded(2, r, c, 900 + r)
-    _, fused, nf = _ns(mn, U, fused=True)
-    _, gemm, ng = _ns(mn, U, fused=False)
+    _, fused, nf = _ns(mn, U, fused=True, variant=variant)
+    _, gemm, ng = _ns(mn, U, fused=False, variant=variant)
     assert nf < ng
-    ref = oracle.ns_batched(f64(U), "standard")
+    ref = oracle.ns_batched(f64(U), variant)
     for i in range(2):
         assert rel(f64(fused)[i], ref[i]) < NS_TOL
         assert rel(f64(gemm)[i], ref[i]) < NS_TOL
@@ -119,35 +124,38 @@ def test_fused_small_agrees_with_gemm_path(mn, shape):
         assert rel(f64(fused)[i], f64(gemm)[i]) < 1e-2
 
 
-def test_fused_small_batch_invariance_and_determinism(mn):
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+def test_fused_small_batch_invariance_and_determinism(mn, variant):
     U = _seeded(40, 128, 1024, 77)
-    _, all_out, _ = _ns(mn, U)
-    _, again, _ = _ns(mn, U)
+    _, all_out, _ = _ns(mn, U, variant=variant)
+    _, again, _ = _ns(mn, U, variant=variant)
     assert torch.equal(all_out, again)
     for i in (0, 17, 39):
-        _, one, _ = _ns(mn, U[i:i + 1].clone())
+        _, one, _ = _ns(mn, U[i:i + 1].clone(), variant=variant)
         assert torch.equal(one[0], all_out[i])
     rev = U.flip(0).contiguous()
-    _, rout, _ = _ns(mn, rev)
+    _, rout, _ = _ns(mn, rev, variant=variant)
     assert torch.equal(rout.flip(0), all_out)
 
 
-def test_fused_small_many_slices(mn):
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+def test_fused_small_many_slices(mn, variant):
     # Many more clusters than fit on the device at once: 300 slices of 8 CTAs.
     U = _seeded(300, 128, 4096, 31)
-    _, out, launches = _ns(mn, U)
+    _, out, launches = _ns(mn, U, variant=variant)
     assert launches <= 3
-    ref = oracle.ns_batched(f64(U[::37]), "standard")
+    ref = oracle.ns_batched(f64(U[::37]), variant)
     got = f64(out[::37])
     for i in range(ref.shape[0]):
         assert rel(got[i], ref[i]) < NS_TOL
 
 
-@pytest.mark.parametrize("steps", [1, 3, 16])
-def test_fused_small_steps_and_schedule(mn, steps):
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+@pytest.mark.parametrize("steps", [1, 2, 3, 16])
+def test_fused_small_steps_and_schedule(mn, steps, variant):
     sched = [(3.4445 - 0.05 * k, -4.7750 + 0.1 * k, 2.0315 - 0.05 * k) for k in range(steps)]
     U = _seeded(2, 96, 700, 8)
-    _, out, _ = _ns(mn, U, mn.Hparams(ns_steps=steps, abc_schedule=sched))
+    _, out, _ = _ns(mn, U, mn.Hparams(ns_steps=steps, abc_schedule=sched), variant=variant)
     X = f64(U)
     for i in range(2):
         x = oracle.frobenius_normalize(X[i], 1e-7)
@@ -176,11 +184,12 @@ def test_fused_small_head_view_of_projection(mn):
         assert rel(got[blk], ref[blk]) < NS_TOL
 
 
-def test_fused_small_zero_slice(mn):
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+def test_fused_small_zero_slice(mn, variant):
     U = _seeded(3, 64, 576, 5)
     U[1].zero_()
-    _, out, _ = _ns(mn, U)
+    _, out, _ = _ns(mn, U, variant=variant)
     assert torch.count_nonzero(out[1]) == 0
-    ref = oracle.ns_batched(f64(U), "standard")
+    ref = oracle.ns_batched(f64(U), variant)
     for i in (0, 2):
         assert rel(f64(out)[i], ref[i]) < NS_TOL
