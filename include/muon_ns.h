@@ -151,6 +151,12 @@ MUON_API muon_status muon_momentum_norm(const muon_batch* batches, int nb, const
  * rows > cols is iterated transposed; the result O is in the slice's own
  * orientation.  X0 = U / (sqrt(sumsq) + ns_eps), with sumsq from
  * muon_momentum_norm when batch.sumsq is non-NULL, else computed here.
+ * Batches whose slices have rows <= cols, rows <= 128 and cols <= 4096 run
+ * every iteration in one launch (a thread-block cluster per slice, the slice
+ * held in shared memory, X X^T summed across the cluster in a fixed order);
+ * the choice depends on the shape only, so a slice's result does not depend
+ * on the rest of the batch.  Setting the environment variable
+ * MUON_NS_FUSED_SMALL=0 sends them through the GEMM path instead.
  * Reads ns_in (left unchanged), sumsq; writes ns_out.
  */
 MUON_API muon_status muon_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp,
@@ -163,6 +169,8 @@ MUON_API muon_status muon_ns_batched(const muon_batch* batches, int nb, const mu
  * G = X0 X0^T: A = G, Q = I; per iteration P = a*I + b*A + c*A^2,
  * Q <- P Q, A <- P A P; O = Q X0.  The m x m products use fp16 operands
  * (10-bit mantissa) with fp32 accumulation; X-side products use bf16.
+ * Small slices (as for muon_ns_batched) run in one launch: the cluster forms
+ * G once and every CTA iterates on the m x m side.
  * Reads ns_in (left unchanged), sumsq; writes ns_out.
  */
 MUON_API muon_status muon_gram_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp,
