@@ -71,6 +71,9 @@ def parse():
                          "minimax schedule for singular values in [--pe-lower, 1]")
     ap.add_argument("--pe-lower", type=float, default=1e-3)
     ap.add_argument("--pe-safety", type=float, default=1.01)
+    ap.add_argument("--graph", choices=["on", "off"], default="on",
+                    help="on: the timed steps replay a CUDA graph of one whole step (the per-stage split "
+                         "comes from eager steps after it); off: eager calls")
     return ap.parse_args()
 
 
@@ -333,17 +336,18 @@ def run_ours(args, wl, variant, rank, world, local_rank):
     slices = sum(b.n for b in groups)
 
     def step(ev=None):
+        st = torch.cuda.current_stream()            # the capture stream while a graph is recorded
         if ev is not None:
-            ev[0].record(stream)
-        mn.muon_momentum_norm(groups, hp, ws, stream)
+            ev[0].record(st)
+        mn.muon_momentum_norm(groups, hp, ws, st)
         if ev is not None:
-            ev[1].record(stream)
-        ns_fn(groups, hp, ws, stream)
+            ev[1].record(st)
+        ns_fn(groups, hp, ws, st)
         if ev is not None:
-            ev[2].record(stream)
-        mn.normuon_update(groups, hp, wl.normuon, ws, stream)
+            ev[2].record(st)
+        mn.normuon_update(groups, hp, wl.normuon, ws, st)
         if ev is not None:
-            ev[3].record(stream)
+            ev[3].record(st)
 
     def barrier():
         if world > 1:
@@ -359,19 +363,48 @@ def run_ours(args, wl, variant, rank, world, local_rank):
         if os.environ.get("CUDA_VISIBLE_DEVICES") else str(local_rank)
     ns_events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    graph = None
+    if args.graph == "on":
+        # One whole step (every kernel of momentum, Newton-Schulz and the
+        # update) captured once and replayed: the timed region then measures
+        # the device, not the host's enqueue rate.
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        l0 = mn.kernel_launches()
+        with torch.cuda.graph(graph):
+            step()
+        per_step_launches = mn.kernel_launches() - l0
+        torch.cuda.synchronize()
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     clocks = Clocks(gpu_id)
     launches0 = mn.kernel_launches()
     start.record(stream)
     for k in range(args.steps):
-        step(ns_events[k])
+        if graph is not None:
+            graph.replay()
+        else:
+            step(ns_events[k])
     end.record(stream)
     torch.cuda.synchronize()
-    launches = mn.kernel_launches() - launches0
+    launches = (per_step_launches * args.steps) if graph is not None else mn.kernel_launches() - launches0
     clk = clocks.stop()
     barrier()
     ms_total = start.elapsed_time(end)
+    if graph is not None:
+        del graph
+        # the per-stage split, from eager steps after the timed region
+        for k in range(args.steps):
+            step(ns_events[k])
+        torch.cuda.synchronize()
     ns_ms = [e[1].elapsed_time(e[2]) for e in ns_events]
     mom_ms = [e[0].elapsed_time(e[1]) for e in ns_events]
     upd_ms = [e[2].elapsed_time(e[3]) for e in ns_events]
@@ -453,6 +486,8 @@ def run_ours(args, wl, variant, rank, world, local_rank):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch Philox on the device)",
         "config": {"workload": DESCRIPTIONS[wl.key], "key": wl.key, "variant": variant,
                    "coefficients": coefficients_desc(args), "slices": slices,
+                   "launch": ("CUDA graph of one whole step, replayed for each timed step" if args.graph == "on"
+                              else "eager calls"),
                    "ns_flop_per_step": ns_flop, "l2": "inputs larger than L2 (126 MB), no flush",
                    "parallelism": f"replicas x{world} (no exchange)"},
         "pct_bf16_peak": round(100 * value / world / peak_s, 2),

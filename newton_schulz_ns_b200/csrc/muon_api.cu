@@ -463,13 +463,37 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
     P.num_problems = np;
     P.total_tiles = static_cast<int>(tiles);
   }
+  // Programmatic dependent launch: each GEMM may start its prologue (barrier
+  // setup, TMEM allocation) on idle SMs while the previous kernel drains; the
+  // kernel waits for its predecessor before touching global memory.
+  // MUON_NS_PDL=0 launches them plainly.
+  static const bool pdl = [] {
+    const char* e = std::getenv("MUON_NS_PDL");
+    return !(e && std::atoi(e) == 0);
+  }();
   for (const Launch& L : launches) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaError_t e;
     if (L.cg == 2) {
       const int units = std::max(1, std::min(L.P.total_tiles, pair_units));
-      ns_gemm_pair_kernel<<<2 * units, GEMM_THREADS, GemmCfg<2>::SMEM_BYTES, stream>>>(L.P);
+      cfg.gridDim = dim3(static_cast<unsigned>(2 * units), 1, 1);
+      cfg.dynamicSmemBytes = GemmCfg<2>::SMEM_BYTES;
+      e = cudaLaunchKernelEx(&cfg, ns_gemm_pair_kernel, L.P);
     } else {
-      const int grid = std::min(L.P.total_tiles, sms);
-      ns_gemm_kernel<<<grid, GEMM_THREADS, GemmCfg<1>::SMEM_BYTES, stream>>>(L.P);
+      cfg.gridDim = dim3(static_cast<unsigned>(std::min(L.P.total_tiles, sms)), 1, 1);
+      cfg.dynamicSmemBytes = GemmCfg<1>::SMEM_BYTES;
+      e = cudaLaunchKernelEx(&cfg, ns_gemm_kernel, L.P);
+    }
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      return MUON_CUDA_ERROR;
     }
     if (!launched()) return MUON_CUDA_ERROR;
   }

@@ -226,6 +226,11 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
   if (CG == 2) cluster_sync();   // the peer signals the leader's barriers only once they exist
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above touched no global memory; the previous kernel of the
+  // stream may still be running (programmatic dependent launch).  Let the
+  // next one start its own prologue, then wait for the previous one's results.
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
 
   if (warp == 0) {
     if (lane == 0) {
