@@ -351,4 +351,30 @@ __global__ void __launch_bounds__(EW_THREADS) update_kernel(const __grid_constan
   }
 }
 
+// out[s][j][i] = in[s][i][j] for i < rows, j < cols: 16-bit elements, 32 x 32
+// tiles staged in shared memory (one padded column against bank conflicts).
+// Lets tall small slices use the fused Newton-Schulz kernel, which works on
+// the short side laid out as rows.  Block (32, 8); grid (cols/32, rows/32, z)
+// with the slices strided over z.
+__global__ void __launch_bounds__(256) transpose16_kernel(const uint16_t* in, long long in_ld, long long in_bs,
+                                                          uint16_t* out, long long out_ld, long long out_bs,
+                                                          int rows, int cols, int slices) {
+  __shared__ uint16_t tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int s = blockIdx.z; s < slices; s += gridDim.z) {
+    const uint16_t* src = in + static_cast<long long>(s) * in_bs;
+    uint16_t* dst = out + static_cast<long long>(s) * out_bs;
+    for (int k = threadIdx.y; k < 32; k += 8) {
+      const int i = r0 + k, j = c0 + threadIdx.x;
+      if (i < rows && j < cols) tile[k][threadIdx.x] = src[static_cast<long long>(i) * in_ld + j];
+    }
+    __syncthreads();
+    for (int k = threadIdx.y; k < 32; k += 8) {
+      const int j = c0 + k, i = r0 + threadIdx.x;
+      if (j < cols && i < rows) dst[static_cast<long long>(j) * out_ld + i] = tile[threadIdx.x][k];
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace muon

@@ -190,7 +190,11 @@ struct NsBatchWs {
   size_t off[5] = {0, 0, 0, 0, 0};   // standard: A, B, X ; gram: Ah, P, Qa, Qb, R
   int64_t ldm = 0, bsm = 0;         // m x m buffers
   int64_t ldx = 0, bsx = 0;         // X buffer
+  size_t t_off = 0;                 // tall slices on the fused path: the transposed slice [cols][rows]
+  int64_t ldt = 0, bst = 0;
 };
+
+bool small_shape_ok(int64_t rows, int64_t cols);
 
 struct Layout {
   size_t total = 0;
@@ -237,6 +241,11 @@ Layout plan_layout(const muon_batch* bs, int nb, int which) {
         w.off[2] = take(sizeof(uint16_t) * static_cast<size_t>(w.bsx) * static_cast<size_t>(b.n));
       } else {
         for (int k = 0; k < 5; ++k) w.off[k] = take(mm);
+      }
+      if (b.rows > b.cols && small_shape_ok(b.cols, b.rows)) {
+        w.ldt = round_up64(b.rows, 64);
+        w.bst = w.ldt * b.cols;
+        w.t_off = take(sizeof(uint16_t) * static_cast<size_t>(w.bst) * static_cast<size_t>(b.n));
       }
     }
   }
@@ -611,16 +620,24 @@ SmallSplit small_split(int64_t n) {
   return SmallSplit{C, 64 * static_cast<int>(cdiv(blocks, C))};
 }
 
-// Slices with rows <= cols, rows <= 128 and cols <= 8 * 512 run the whole
-// iteration in one clustered launch (ns_small.cuh).  The choice depends on the shape only,
-// so a slice's result never depends on the rest of the batch.  Setting
-// MUON_NS_FUSED_SMALL=0 sends them through the GEMM path instead.
+// A wide slice (rows <= cols) the fused kernel takes: rows <= 128 and
+// cols <= 8 * 512.
+bool small_shape_ok(int64_t rows, int64_t cols) {
+  if (rows > cols || rows > SMALL_MAX_M) return false;
+  const SmallSplit sp = small_split(cols);
+  return sp.C <= SMALL_MAX_CLUSTER && sp.w <= SMALL_MAX_W;
+}
+
+// Slices whose short side is at most 128 and long side at most 8 * 512 run
+// the whole iteration in one clustered launch (ns_small.cuh); tall ones
+// (rows > cols) are transposed into the workspace first and back after.
+// The choice depends on the shape only, so a slice's result never depends
+// on the rest of the batch.  Setting MUON_NS_FUSED_SMALL=0 sends them
+// through the GEMM path instead.
 bool small_eligible(const muon_batch& b) {
   const char* e = std::getenv("MUON_NS_FUSED_SMALL");
   if (e && std::atoi(e) == 0) return false;
-  if (b.rows > b.cols || b.rows > SMALL_MAX_M) return false;
-  const SmallSplit sp = small_split(b.cols);
-  return sp.C <= SMALL_MAX_CLUSTER && sp.w <= SMALL_MAX_W;
+  return b.rows > b.cols ? small_shape_ok(b.cols, b.rows) : small_shape_ok(b.rows, b.cols);
 }
 
 muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const float* sumsq, int* err, bool gram,
@@ -671,6 +688,37 @@ muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const floa
     if (!launched()) return MUON_CUDA_ERROR;
   }
   return MUON_OK;
+}
+
+muon_status launch_transpose16(const void* in, int64_t in_ld, int64_t in_bs, void* out, int64_t out_ld,
+                               int64_t out_bs, int64_t rows, int64_t cols, int64_t slices, cudaStream_t stream) {
+  const dim3 grid(static_cast<unsigned>(cdiv(cols, 32)), static_cast<unsigned>(cdiv(rows, 32)),
+                  static_cast<unsigned>(std::min<int64_t>(slices, 65535)));
+  transpose16_kernel<<<grid, dim3(32, 8, 1), 0, stream>>>(
+      static_cast<const uint16_t*>(in), in_ld, in_bs, static_cast<uint16_t*>(out), out_ld, out_bs,
+      static_cast<int>(rows), static_cast<int>(cols), static_cast<int>(slices));
+  return launched() ? MUON_OK : MUON_CUDA_ERROR;
+}
+
+// The fused kernel on one batch; a tall batch goes through its transposed
+// copy in the workspace (the kernel then works in place on that copy: each
+// CTA reads its columns before writing them back).
+muon_status run_small(const muon_batch& b, const NsBatchWs& w, uint8_t* ws, const muon_hparams* hp,
+                      const float* sumsq, int* err, bool gram, cudaStream_t stream) {
+  if (b.rows <= b.cols) return launch_small(b, hp, sumsq, err, gram, stream);
+  void* T = ws + w.t_off;
+  const int64_t in_bs = b.n > 1 ? b.ns_in.batch_stride : b.rows * b.ns_in.ld;
+  const int64_t out_bs = b.n > 1 ? b.ns_out.batch_stride : b.rows * b.ns_out.ld;
+  muon_status st = launch_transpose16(b.ns_in.ptr, b.ns_in.ld, in_bs, T, w.ldt, w.bst, b.rows, b.cols, b.n, stream);
+  if (st != MUON_OK) return st;
+  muon_batch v = b;
+  v.rows = b.cols;
+  v.cols = b.rows;
+  v.ns_in = muon_view{T, w.ldt, w.bst, MUON_BF16, 0};
+  v.ns_out = v.ns_in;
+  if ((st = launch_small(v, hp, sumsq, err, gram, stream)) != MUON_OK) return st;
+  return launch_transpose16(T, w.ldt, w.bst, const_cast<void*>(b.ns_out.ptr), b.ns_out.ld, out_bs, b.cols, b.rows,
+                            b.n, stream);
 }
 
 // SYRK of the slice storage X ([rows][cols]) on the short side: out = f * X X^T (rows <= cols)
@@ -1011,7 +1059,7 @@ muon_status ns_standard_impl(const muon_batch* batches, int nb, const muon_hpara
   for (int i = 0; i < nb; ++i) {
     if (batch_empty(batches[i]) || !small_eligible(batches[i])) continue;
     fused[i] = 1;
-    if ((st = launch_small(batches[i], hp, sumsq[i], err, false, stream)) != MUON_OK) return st;
+    if ((st = run_small(batches[i], L.nsb[i], ws, hp, sumsq[i], err, false, stream)) != MUON_OK) return st;
   }
   const int S = hp->ns_steps;
   for (int it = 0; it < S; ++it) {
@@ -1068,7 +1116,7 @@ muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* 
   for (int i = 0; i < nb; ++i) {
     if (batch_empty(batches[i]) || !small_eligible(batches[i])) continue;
     fused[i] = 1;
-    if ((st = launch_small(batches[i], hp, sumsq[i], err, true, stream)) != MUON_OK) return st;
+    if ((st = run_small(batches[i], L.nsb[i], ws, hp, sumsq[i], err, true, stream)) != MUON_OK) return st;
   }
   // G: kappa * s^2 * X X^T (short side) in fp16.
   {
