@@ -150,6 +150,21 @@ def default_variant(wl):
 
 # ----------------------------------------------------------------------------- CPU oracle (baseline)
 
+def ns_kernels_label(groups):
+    """Which kernels one Newton-Schulz call of these batches runs (the library's shape rule)."""
+    def fused(r, c):
+        m, n = min(r, c), max(r, c)
+        return m <= 128 and n <= 4096
+    kinds = {fused(b.rows, b.cols) for b in groups}
+    if kinds == {True}:
+        name = "ns_small_kernel (fused: one clustered launch per batch)"
+    elif kinds == {False}:
+        name = "ns_gemm_pair_kernel / ns_gemm_kernel"
+    else:
+        name = "ns_small_kernel + ns_gemm_pair_kernel"
+    return name + " (all launches of one Newton-Schulz call)"
+
+
 def coefficients_desc(args):
     if args.coefficients == "polar-express":
         return (f"polar-express (greedy minimax quintics, singular values in [{args.pe_lower:g}, 1], "
@@ -498,7 +513,7 @@ def run_ours(args, wl, variant, rank, world, local_rank):
         "hbm_kernels": {"momentum_gbs": round(momentum_bytes(groups) / (mom_mean / 1e3) / 1e9, 1),
                         "update_gbs": round(update_bytes(groups, wl.normuon) / (upd_mean / 1e3) / 1e9, 1),
                         "peak_gbs": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])},
-        "roofline": {"bound": "tensor", "kernel": "ns_gemm_kernel (all launches of one Newton-Schulz call)",
+        "roofline": {"bound": "tensor", "kernel": ns_kernels_label(groups),
                      "achieved": round(achieved, 2), "peak": peak_s, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_s, 4), "frac_of_burst": round(achieved / peak_b, 4),
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a long step)",
