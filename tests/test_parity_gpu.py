@@ -380,7 +380,8 @@ def test_auto_dispatch_routes_by_shape(mn):
     # n >= 1.25 m goes through the Gram form, square and near-square through
     # the standard form; each batch must come out exactly as its own form's
     # call produces it.
-    shapes = [(64, 576, 3), (256, 256, 2), (300, 340, 2), (1000, 200, 1)]
+    # (64 x 576, 640 x 100 tall, 100 x 110: the fused small-side kernel in both forms)
+    shapes = [(64, 576, 3), (256, 256, 2), (300, 340, 2), (1000, 200, 1), (640, 100, 2), (100, 110, 2)]
     Us = [_seeded(n, r, c, 500 + k, torch.bfloat16) for k, (r, c, n) in enumerate(shapes)]
     auto = [_ns_batch(mn, U) for U in Us]
     ws = mn.allocate_workspace(auto, -1)

@@ -200,3 +200,39 @@ def test_fused_small_zero_slice(mn, variant):
     ref = oracle.ns_batched(f64(U), variant)
     for i in (0, 2):
         assert rel(f64(out)[i], ref[i]) < NS_TOL
+
+
+def test_fused_small_step_captured_in_cuda_graph(mn):
+    # Fused launches (cluster attribute), tall transposes and the GEMM path's
+    # programmatic dependent launches, captured together and replayed.
+    Us = [_seeded(2, 128, 1024, 41), _seeded(2, 700, 96, 42), _seeded(1, 300, 520, 43)]
+    outs = []
+    bs = []
+    for U in Us:
+        n, r, c = U.shape
+        _, out = _padded(n, r, c, torch.bfloat16, float("nan"))
+        outs.append(out)
+        bs.append(mn.Batch(n, r, c, ns_in=U, ns_out=out))
+    ws = mn.allocate_workspace(bs, -1)
+    hp = mn.Hparams()
+    mn.muon_ns_batched(bs, hp, ws)          # per-device set-up happens eagerly
+    torch.cuda.synchronize()
+    eager = [o.clone() for o in outs]
+    for o in outs:
+        o.fill_(float("nan"))
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        mn.muon_ns_batched(bs, hp, ws)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for o in outs:
+        o.fill_(float("nan"))
+    with torch.cuda.graph(g):
+        mn.muon_ns_batched(bs, hp, ws, torch.cuda.current_stream())
+    g.replay()
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0
+    for e, o in zip(eager, outs):
+        assert torch.equal(e, o)
