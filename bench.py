@@ -517,7 +517,7 @@ def run_ours(args, wl, variant, rank, world, local_rank):
                      "achieved": round(achieved, 2), "peak": peak_s, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_s, 4), "frac_of_burst": round(achieved / peak_b, 4),
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a long step)",
-                     "traffic": measured_traffic(wl.key, variant),
+                     "traffic": measured_traffic(wl.key, variant) if args.scale_down == 1 else None,
                      "traffic_unit": "bytes per Newton-Schulz call (ncu dram__bytes_read.sum + write.sum)"},
         "gpu_launches": int(launches),
         "clocks": clk,
