@@ -215,3 +215,34 @@ def test_polar_express_schedule_safety_and_arguments(mn):
         with pytest.raises(mn.MuonError) as e:
             mn.polar_express_schedule(**kw)
         assert e.value.status == 1      # MUON_INVALID_ARG
+
+
+def test_workspace_holds_the_transposed_copy_of_tall_small_slices(mn):
+    # A tall slice with a short side <= 128 and a long side <= 4096 runs the
+    # fused kernel on a transposed copy [n][cols][rows] (rows rounded to 64)
+    # in the workspace of both Newton-Schulz forms; a wide slice, and a tall
+    # one outside those limits, needs none.
+    from newton_schulz_ns_b200 import _capi
+
+    def size(b, which):
+        return _capi.lib.muon_workspace_size((_capi.MuonBatch * 1)(b), 1, which)
+
+    n, r, c = 3, 700, 96                       # tall, fused
+    copy = n * c * ((r + 63) // 64 * 64) * 2
+    for which in (1, 2):
+        tall = size(_fake_batch(mn, n, r, c), which)
+        # the same buffers without the copy: m x m ones of the same m, plus
+        # (standard) the X-sized buffer of a rows x cols slice
+        m = c
+        mm = n * ((m + 63) // 64 * 64) * m * 2
+        base = 256 + 2 * 256                   # error word, norm partials and sums (rounded up)
+        if which == 1:
+            base_bufs = 2 * mm + n * r * ((c + 63) // 64 * 64) * 2
+        else:
+            base_bufs = 5 * mm
+        assert tall >= base_bufs + copy
+        assert tall - copy < base_bufs + base + 5 * 256 + 8 * n * ((r * c + 8191) // 8192) + 64
+    # wide twin and a tall slice with a long side past 4096: no copy
+    assert size(_fake_batch(mn, n, c, r), 1) < size(_fake_batch(mn, n, r, c), 1)
+    t_big = size(_fake_batch(mn, 1, 5000, 96), 2)
+    assert t_big < 5 * ((96 + 63) // 64 * 64) * 96 * 2 + 256 * 8 + 4 * ((5000 * 96 + 8191) // 8192) + 4096
