@@ -13,6 +13,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
+#include "ptx_sm100.cuh"
 
 namespace muon {
 
@@ -138,6 +139,8 @@ __device__ __forceinline__ float block_sum(float v, float* scratch) {
 // ---------------------------------------------------------------------------
 template <int MODE>
 __global__ void __launch_bounds__(EW_THREADS) momentum_chunks_kernel(const __grid_constant__ EwParams P) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   __shared__ float scratch[32];
   for (long long c = blockIdx.x; c < P.total_chunks; c += gridDim.x) {
     const int si = find_seg_by_chunk(P, c);
@@ -208,6 +211,8 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_chunks_kernel(const __gri
 
 // One warp per slice sums that slice's chunk partials in chunk order.
 __global__ void __launch_bounds__(EW_THREADS) sumsq_finalize_kernel(const __grid_constant__ EwParams P) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (EW_THREADS / 32);
   for (long long gs = blockIdx.x * (EW_THREADS / 32) + (threadIdx.x >> 5); gs < P.total_slices; gs += warps) {
@@ -232,6 +237,8 @@ __global__ void __launch_bounds__(EW_THREADS) sumsq_finalize_kernel(const __grid
 //   ss = sum_j O_ij^2;  v <- beta2*v + (1-beta2)*ss/cols;  d = 1/(sqrt(v)+eps)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(EW_THREADS) normuon_rows_kernel(const __grid_constant__ EwParams P) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (EW_THREADS / 32);
   for (long long gr = blockIdx.x * (EW_THREADS / 32) + (threadIdx.x >> 5); gr < P.total_rows; gr += warps) {
@@ -269,6 +276,8 @@ __global__ void __launch_bounds__(EW_THREADS) normuon_rows_kernel(const __grid_c
 
 // One block per slice: factor = ||O||_F / ||O * d||_F (0 when the latter is 0).
 __global__ void __launch_bounds__(EW_THREADS) normuon_slices_kernel(const __grid_constant__ EwParams P) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   __shared__ float scratch[32];
   for (long long gs = blockIdx.x; gs < P.total_slices; gs += gridDim.x) {
     int si = 0;
@@ -292,6 +301,8 @@ __global__ void __launch_bounds__(EW_THREADS) normuon_slices_kernel(const __grid
 // W <- W*(1 - lr*wd) - lr*lr_scale*factor*d_row * O ; optional bf16 copy.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(EW_THREADS) update_kernel(const __grid_constant__ EwParams P) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   const float keep = 1.0f - P.lr * P.wd;
   for (long long c = blockIdx.x; c < P.total_chunks; c += gridDim.x) {
     const int si = find_seg_by_chunk(P, c);
@@ -351,6 +362,14 @@ __global__ void __launch_bounds__(EW_THREADS) update_kernel(const __grid_constan
   }
 }
 
+// Clears the error word at the start of a call, as a kernel so that it keeps
+// the stream's chain of programmatically dependent launches.
+__global__ void clear_word_kernel(int* word) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
+  if (threadIdx.x == 0) *word = 0;
+}
+
 // out[s][j][i] = in[s][i][j] for i < rows, j < cols: 16-bit elements, 32 x 32
 // tiles staged in shared memory (one padded column against bank conflicts).
 // Lets tall small slices use the fused Newton-Schulz kernel, which works on
@@ -360,6 +379,8 @@ __global__ void __launch_bounds__(256) transpose16_kernel(const uint16_t* in, lo
                                                           uint16_t* out, long long out_ld, long long out_bs,
                                                           int rows, int cols, int slices) {
   __shared__ uint16_t tile[32][33];
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
   for (int s = blockIdx.z; s < slices; s += gridDim.z) {
     const uint16_t* src = in + static_cast<long long>(s) * in_bs;

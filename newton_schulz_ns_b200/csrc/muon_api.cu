@@ -58,6 +58,41 @@ inline bool launched() {
   return true;
 }
 
+// Programmatic dependent launch for every kernel of the step: each kernel
+// lets the next one start its prologue and waits for its predecessor before
+// its first global access.  MUON_NS_PDL=0 launches them plainly.
+inline bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("MUON_NS_PDL");
+    return !(e && std::atoi(e) == 0);
+  }();
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+bool launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  return launched();
+}
+
+// Zeroes the error word at workspace offset 0 (a kernel, so the launch chain holds).
+inline bool clear_error_word(void* ws, cudaStream_t stream) {
+  return launch_pdl(clear_word_kernel, dim3(1), dim3(32), 0, stream, reinterpret_cast<int*>(ws));
+}
+
 muon_status device_setup(int* sms_out, int* pair_units_out = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MUON_CUDA_ERROR;
@@ -476,10 +511,7 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
   // setup, TMEM allocation) on idle SMs while the previous kernel drains; the
   // kernel waits for its predecessor before touching global memory.
   // MUON_NS_PDL=0 launches them plainly.
-  static const bool pdl = [] {
-    const char* e = std::getenv("MUON_NS_PDL");
-    return !(e && std::atoi(e) == 0);
-  }();
+  const bool pdl = pdl_enabled();
   for (const Launch& L : launches) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -569,13 +601,15 @@ muon_status launch_norm(const muon_batch* bs, int nb, const muon_hparams* hp, in
     P.nesterov = hp ? hp->nesterov : 0;
     P.partials = partials;
     P.sumsq_ws = sumsq_ws_dev;
-    if (mode == 0)
-      momentum_chunks_kernel<0><<<ew_grid(chunk, sms), EW_THREADS, 0, stream>>>(P);
-    else
-      momentum_chunks_kernel<1><<<ew_grid(chunk, sms), EW_THREADS, 0, stream>>>(P);
-    if (!launched()) return MUON_CUDA_ERROR;
-    sumsq_finalize_kernel<<<ew_grid(cdiv(slice, EW_THREADS / 32), sms), EW_THREADS, 0, stream>>>(P);
-    if (!launched()) return MUON_CUDA_ERROR;
+    const bool ok = mode == 0
+                        ? launch_pdl(momentum_chunks_kernel<0>, dim3(ew_grid(chunk, sms)), dim3(EW_THREADS), 0,
+                                     stream, P)
+                        : launch_pdl(momentum_chunks_kernel<1>, dim3(ew_grid(chunk, sms)), dim3(EW_THREADS), 0,
+                                     stream, P);
+    if (!ok) return MUON_CUDA_ERROR;
+    if (!launch_pdl(sumsq_finalize_kernel, dim3(ew_grid(cdiv(slice, EW_THREADS / 32), sms)), dim3(EW_THREADS), 0,
+                    stream, P))
+      return MUON_CUDA_ERROR;
     partials += chunk;
     sumsq_ws_dev += slice;
   }
@@ -674,13 +708,15 @@ muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const floa
     cfg.blockDim = dim3(SMALL_THREADS, 1, 1);
     cfg.dynamicSmemBytes = SMALL_SMEM_BYTES;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(sp.C);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
     if (cudaLaunchKernelEx(&cfg, gram ? ns_small_gram_kernel : ns_small_kernel, P) != cudaSuccess) {
       (void)cudaGetLastError();
       return MUON_CUDA_ERROR;
@@ -694,10 +730,11 @@ muon_status launch_transpose16(const void* in, int64_t in_ld, int64_t in_bs, voi
                                int64_t out_bs, int64_t rows, int64_t cols, int64_t slices, cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>(cdiv(cols, 32)), static_cast<unsigned>(cdiv(rows, 32)),
                   static_cast<unsigned>(std::min<int64_t>(slices, 65535)));
-  transpose16_kernel<<<grid, dim3(32, 8, 1), 0, stream>>>(
-      static_cast<const uint16_t*>(in), in_ld, in_bs, static_cast<uint16_t*>(out), out_ld, out_bs,
-      static_cast<int>(rows), static_cast<int>(cols), static_cast<int>(slices));
-  return launched() ? MUON_OK : MUON_CUDA_ERROR;
+  const bool ok = launch_pdl(transpose16_kernel, grid, dim3(32, 8, 1), 0, stream, static_cast<const uint16_t*>(in),
+                             static_cast<long long>(in_ld), static_cast<long long>(in_bs), static_cast<uint16_t*>(out),
+                             static_cast<long long>(out_ld), static_cast<long long>(out_bs), static_cast<int>(rows),
+                             static_cast<int>(cols), static_cast<int>(slices));
+  return ok ? MUON_OK : MUON_CUDA_ERROR;
 }
 
 // The fused kernel on one batch; a tall batch goes through its transposed
@@ -845,7 +882,7 @@ muon_status validate_ns(const muon_batch* bs, int nb, const muon_hparams* hp) {
 // Returns the per-batch sumsq pointers to use.
 muon_status prepare_norms(const muon_batch* bs, int nb, const Layout& L, uint8_t* ws, int sms, cudaStream_t stream,
                           std::vector<const float*>& sumsq, bool clear_err = true) {
-  if (clear_err && cudaMemsetAsync(ws, 0, sizeof(int32_t), stream) != cudaSuccess) return MUON_CUDA_ERROR;
+  if (clear_err && !clear_error_word(ws, stream)) return MUON_CUDA_ERROR;
   sumsq.assign(nb, nullptr);
   std::vector<muon_batch> missing;
   float* base = reinterpret_cast<float*>(ws + L.sumsq);
@@ -1203,7 +1240,7 @@ muon_status muon_ns_auto_batched(const muon_batch* batches, int nb, const muon_h
   if (!std_b.empty() || !gram_b.empty())
     if ((st = check_ws(workspace, workspace_bytes, need)) != MUON_OK) return st;
   // One error word for the whole call: cleared once, kept across both forms.
-  if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), stream) != cudaSuccess) return MUON_CUDA_ERROR;
+  if (!clear_error_word(workspace, stream)) return MUON_CUDA_ERROR;
   if (!std_b.empty() && (st = ns_standard_impl(std_b.data(), static_cast<int>(std_b.size()), hp, workspace,
                                                workspace_bytes, stream, false)) != MUON_OK)
     return st;
@@ -1280,13 +1317,14 @@ muon_status normuon_update(const muon_batch* batches, int nb, const muon_hparams
     P.row_d = row_d;
     P.slice_factor = factor;
     if (use_normuon) {
-      normuon_rows_kernel<<<ew_grid(cdiv(row, EW_THREADS / 32), sms), EW_THREADS, 0, stream>>>(P);
-      if (!launched()) return MUON_CUDA_ERROR;
-      normuon_slices_kernel<<<ew_grid(slice, sms), EW_THREADS, 0, stream>>>(P);
-      if (!launched()) return MUON_CUDA_ERROR;
+      if (!launch_pdl(normuon_rows_kernel, dim3(ew_grid(cdiv(row, EW_THREADS / 32), sms)), dim3(EW_THREADS), 0,
+                      stream, P))
+        return MUON_CUDA_ERROR;
+      if (!launch_pdl(normuon_slices_kernel, dim3(ew_grid(slice, sms)), dim3(EW_THREADS), 0, stream, P))
+        return MUON_CUDA_ERROR;
     }
-    update_kernel<<<ew_grid(chunk, sms), EW_THREADS, 0, stream>>>(P);
-    if (!launched()) return MUON_CUDA_ERROR;
+    if (!launch_pdl(update_kernel, dim3(ew_grid(chunk, sms)), dim3(EW_THREADS), 0, stream, P))
+      return MUON_CUDA_ERROR;
   }
   return MUON_OK;
 }

@@ -339,6 +339,11 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Nothing above touched global memory: let the next kernel of the stream
+  // start its prologue, then wait for the previous one's results.
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
+
   // ---- resident columns of the slice (zero outside it)
   if (tid == 0) {
     mbar_arrive_expect_tx(&bars[0], static_cast<uint32_t>(nblk * SMALL_BLK));

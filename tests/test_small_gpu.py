@@ -105,7 +105,8 @@ def test_fused_small_matches_oracle(mn, shape, variant):
     r, c = shape
     U = _seeded(3, r, c, 500 + r + c)
     base, out, launches = _ns(mn, U, variant=variant)
-    assert launches <= (5 if r > c else 3)      # norms (2) + one fused launch (+ 2 transposes)
+    # error-word clear (1) + norms (2) + one fused launch (+ 2 transposes)
+    assert launches <= (6 if r > c else 4)
     ref = oracle.ns_batched(f64(U), variant)
     got = f64(out)
     for i in range(3):
@@ -150,7 +151,7 @@ def test_fused_small_many_slices(mn, variant):
     # Many more clusters than fit on the device at once: 300 slices of 8 CTAs.
     U = _seeded(300, 128, 4096, 31)
     _, out, launches = _ns(mn, U, variant=variant)
-    assert launches <= 3
+    assert launches <= 4
     ref = oracle.ns_batched(f64(U[::37]), variant)
     got = f64(out[::37])
     for i in range(ref.shape[0]):
