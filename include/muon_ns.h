@@ -35,6 +35,14 @@
  * the given stream.  Scratch memory is the caller's workspace, sized by
  * muon_workspace_size.
  *
+ * Streams and graphs.  A call enqueues only kernels on `stream`, launched
+ * with programmatic stream serialization: each may start its prologue while
+ * the previous kernel of the stream finishes and waits for it before
+ * touching memory (set MUON_NS_PDL=0 to launch them plainly).  A whole step
+ * can be captured in a CUDA graph; the first call on a device does one-time
+ * set-up (kernel attributes, the driver's tensor-map encoder) and must run
+ * before any capture on that device.
+ *
  * Errors.  Every argument is checked on the host before anything is
  * enqueued.  On any error the call returns a non-zero status and touches no
  * memory ("reject before mutating").  There is no fallback to another

@@ -400,7 +400,7 @@ def test_auto_dispatch_routes_by_shape(mn):
 
 @pytest.mark.parametrize("variant", ["standard", "gram"])
 def test_step_captured_in_cuda_graph_matches_eager(mn, variant):
-    # The calls enqueue only kernels and memsets on the given stream, so a
+    # The calls enqueue only kernels on the given stream, so a
     # whole step can be captured once and replayed.  Per-device set-up runs
     # on the first call, which therefore happens eagerly before capture.
     w = workloads.WORKLOADS["conv_megabatch"]
