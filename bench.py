@@ -44,14 +44,6 @@ DESCRIPTIONS = {
     "single_256": "one 256x256 fp32 gradient, Muon, lr 0.05",
 }
 
-# Oracle sample per workload for the CPU baseline: (group index, parameters of it).
-CPU_SAMPLE = {
-    "llama8b": [(0, 1), (1, 1), (2, 1)],          # layer 0 q_proj, k_proj, v_proj
-    "moe": [(0, 1), (1, 1)],                      # expert 0 w1 and w2
-    "per_head": [(0, 1), (1, 1), (2, 1)],         # all of it
-    "conv_megabatch": [(0, 16)],
-    "single_256": [(0, 1)],
-}
 
 
 def parse():
@@ -96,21 +88,34 @@ def slice_variant(rows, cols, variant):
     return "gram" if n > m and n >= AUTO_GRAM_RATIO * m else "standard"
 
 
-def ns_flops(rows, cols, variant, steps):
+GRAM_RESTART = 3        # the library's default restart period of the Gram form
+
+
+def ns_flops(rows, cols, variant, steps, restart=GRAM_RESTART):
     """Work of one slice's orthogonalization, as the metric counts it (m = short side, n = long side).
 
     Standard, one triangle of each symmetric product: per step m^2 n (X X^T)
     + m^3 (b*A + c*A^2) + 2 m^2 n (B X).  Gram: m^2 n for X X^T, 2 m^2 n for
-    the final Q X, and per step one-triangle m^3 products: A^2, P Q (from the
-    second step), and the two factors of P A P (up to the second-to-last).
+    the final Q X, per step one-triangle m^3 products: A^2, P Q (except at a
+    segment's first step), the two factors of P A P (except at a segment's
+    last step); each restart adds Q X (2 m^2 n) and X X^T (m^2 n).
     Both arms of the benchmark count the same work for the same variant.
     """
     m, n = min(rows, cols), max(rows, cols)
     variant = slice_variant(rows, cols, variant)
     if variant == "standard":
         return float(steps * (3 * m * m * n + m ** 3))
-    prods = sum(1 + (k > 0) + 2 * (k < steps - 1) for k in range(steps))
-    return float(3 * m * m * n + prods * m ** 3)
+
+    def restart_at(k):
+        return restart > 0 and 0 < k < steps and k % restart == 0
+
+    prods, restarts, seg = 0, 0, 0
+    for k in range(steps):
+        if restart_at(k):
+            restarts += 1
+            seg = k
+        prods += 1 + (k != seg) + 2 * (not (k == steps - 1 or restart_at(k + 1)))
+    return float(3 * m * m * n + restarts * 3 * m * m * n + prods * m ** 3)
 
 
 TRAFFIC_SOURCES = ("newton_schulz_ns_b200/csrc/ns_gemm.cuh", "newton_schulz_ns_b200/csrc/ptx_sm100.cuh",
@@ -172,45 +177,90 @@ def coefficients_desc(args):
     return "quintic (3.4445, -4.7750, 2.0315) at every step"
 
 
-def oracle_sample(wl, variant, budget_s=30.0, abc=None):
-    """Runs the fp64 oracle's full step on the workload's sample; returns (flops, slices, seconds, cores, desc)."""
+def cpu_sample_units(wl, variant):
+    """The workload's distinct Newton-Schulz work shapes, one parameter each, with their counts.
+
+    A unit is one parameter of a group (all its head slices); groups whose
+    parameters have the same short side, long side, slices per parameter and
+    variant cost the oracle the same and share a unit (Llama-8B: q/o, k/v and
+    gate/up/down).  Each unit's weight is how many such parameters the
+    workload holds.
+    """
+    units = {}
+    for g in wl.groups:
+        r, c = g.slice_rows, g.cols
+        key = (min(r, c), max(r, c), g.slices // g.count, slice_variant(r, c, variant))
+        if key in units:
+            units[key][1] += g.count
+            units[key][2].append(g.name)
+        else:
+            units[key] = [g, g.count, [g.name]]
+    return [tuple(u) for u in units.values()]
+
+
+def oracle_unit(wl, g, variant, abc=None):
+    """The fp64 oracle's full step on parameter 0 of group g; returns (flops, slices, seconds)."""
     import numpy as np
-    import threadpoolctl
     import oracle
     import workloads
 
-    ncores = os.cpu_count() or 1
-    with threadpoolctl.threadpool_limits(limits=ncores):
-        info = threadpoolctl.threadpool_info()
-        cores = max([i.get("num_threads", 1) for i in info] or [1])
-        flops = 0.0
-        slices = 0
-        parts = []
-        t0 = time.perf_counter()
-        for gi, count in CPU_SAMPLE[wl.key]:
-            g = wl.groups[gi]
-            for p in range(count):
-                G = workloads.gradient(wl, g, p, 0).float().double().numpy().reshape(g.slices // g.count,
-                                                                                     g.slice_rows, g.cols)
-                W = workloads.initial_weight(wl, g, p).float().double().numpy().reshape(G.shape)
-                M = np.zeros_like(G)
-                v = np.zeros(G.shape[:2]) if wl.normuon else None
-                oracle.muon_step_slices(G, M, W, v, mu=wl.momentum, nesterov=wl.nesterov, ns_eps=wl.ns_eps,
-                                        ns_steps=wl.ns_steps, abc=abc if abc is not None else oracle.QUINTIC_ABC,
-                                        variant=slice_variant(g.slice_rows, g.cols, variant),
-                                        normuon=wl.normuon,
-                                        beta2=wl.beta2, nor_eps=wl.nor_eps, lr=wl.lr,
-                                        weight_decay=wl.weight_decay,
-                                        lr_scale=math.sqrt(max(1.0, g.rows / g.cols)))
-                flops += G.shape[0] * ns_flops(g.slice_rows, g.cols, variant, wl.ns_steps)
-                slices += G.shape[0]
-            parts.append(f"{g.name} x{count}")
-            if time.perf_counter() - t0 > budget_s:
-                break
-        dt = time.perf_counter() - t0
-    desc = (f"oracle (numpy fp64, full step incl. momentum/NorMuon/update) on {', '.join(parts)} of "
-            f"{wl.key}; {slices} slices")
-    return flops, slices, dt, cores, desc
+    G = workloads.gradient(wl, g, 0, 0).float().double().numpy().reshape(g.slices // g.count, g.slice_rows, g.cols)
+    W = workloads.initial_weight(wl, g, 0).float().double().numpy().reshape(G.shape)
+    M = np.zeros_like(G)
+    v = np.zeros(G.shape[:2]) if wl.normuon else None
+    sv = slice_variant(g.slice_rows, g.cols, variant)
+    t0 = time.perf_counter()
+    oracle.muon_step_slices(G, M, W, v, mu=wl.momentum, nesterov=wl.nesterov, ns_eps=wl.ns_eps,
+                            ns_steps=wl.ns_steps, abc=abc if abc is not None else oracle.QUINTIC_ABC,
+                            variant=sv, restart=GRAM_RESTART if sv == "gram" else 0, normuon=wl.normuon,
+                            beta2=wl.beta2, nor_eps=wl.nor_eps, lr=wl.lr, weight_decay=wl.weight_decay,
+                            lr_scale=oracle.update_scale(g.rows, g.cols))
+    dt = time.perf_counter() - t0
+    return G.shape[0] * ns_flops(g.slice_rows, g.cols, variant, wl.ns_steps), G.shape[0], dt
+
+
+def oracle_rate(units, times):
+    """Workload-weighted rate from per-unit oracle times: (flops/s, slices/s) = sum w f / sum w t."""
+    flops = sum(w * f for (_, w, _), (f, _, _) in zip(units, times))
+    slices = sum(w * sl for (_, w, _), (_, sl, _) in zip(units, times))
+    sec = sum(w * t for (_, w, _), (_, _, t) in zip(units, times))
+    return flops / sec, slices / sec
+
+
+def oracle_sample_desc(wl, units):
+    names = "; ".join(f"{'/'.join(n)} (x{w})" for (_, w, n) in units)
+    return (f"oracle (numpy fp64, full step incl. momentum/NorMuon/update) on ONE parameter of each distinct "
+            f"Newton-Schulz shape of {wl.key}: {names}; the rate weights each shape's oracle time by its count "
+            f"(an extrapolation from {len(units)} parameter(s) to the whole workload)")
+
+
+def host_threads():
+    import threadpoolctl
+    info = threadpoolctl.threadpool_info()
+    return max([i.get("num_threads", 1) for i in info] or [1])
+
+
+def oracle_sample(wl, variant, abc=None):
+    """Runs the oracle once on every unit; returns (flops/s, slices/s, seconds, cores, desc)."""
+    import threadpoolctl
+    units = cpu_sample_units(wl, variant)
+    with threadpoolctl.threadpool_limits(limits=os.cpu_count() or 1):
+        cores = host_threads()
+        times = [oracle_unit(wl, g, variant, abc) for (g, _, _) in units]
+    rate, slice_rate = oracle_rate(units, times)
+    return rate, slice_rate, sum(t for (_, _, t) in times), cores, oracle_sample_desc(wl, units)
+
+
+def workload_config(args, wl, variant):
+    """The `config` both arms print: what workload, variant and coefficients the metric is on."""
+    slices = wl.slices
+    return {"workload": DESCRIPTIONS[wl.key], "key": wl.key, "variant": variant,
+            "coefficients": coefficients_desc(args), "slices": slices,
+            "ns_flop_per_step": sum(g.slices * ns_flops(g.slice_rows, g.cols, variant, wl.ns_steps)
+                                    for g in wl.groups),
+            "l2": "inputs larger than L2 (126 MB), no flush" if wl.key in ("llama8b", "moe")
+            else "inputs smaller than L2: device-resident, no flush (latency-bound configuration)",
+            "scale_down": args.scale_down}
 
 
 # ----------------------------------------------------------------------------- GPU state
@@ -237,7 +287,8 @@ def build_state(wl, variant, dev, schedule=None):
                      if wl.weight_copy_bf16 else None,
                      sumsq=torch.zeros(n, dtype=torch.float32, device=dev),
                      variance=torch.zeros(n * r, dtype=torch.float32, device=dev) if wl.normuon else None,
-                     lr_scale=mn.spectral_scale(g.rows, g.cols))
+                     row_sumsq=torch.zeros(n * r, dtype=torch.float32, device=dev) if wl.normuon else None,
+                     fan_out=g.rows, fan_in=g.cols)
         groups.append(b)
     hp = mn.Hparams(mu=wl.momentum, nesterov=wl.nesterov, ns_eps=wl.ns_eps, ns_steps=wl.ns_steps,
                     abc_schedule=schedule,
@@ -302,11 +353,17 @@ def momentum_bytes(groups):
 
 
 def update_bytes(groups, normuon):
-    """Algorithmic bytes of normuon_update: read O (twice with NorMuon: row sums, update), W; write W, copy."""
+    """Algorithmic bytes of normuon_update: read O and W, write W and the bf16 copy.
+
+    With NorMuon the row sums of squares come from the Newton-Schulz call's
+    last epilogue (row_sumsq), so O is read once; the per-row statistics
+    (a few bytes per row) are not counted.
+    """
     tot = 0
     for b in groups:
         e = b.n * b.rows * b.cols
-        tot += e * ((4 if normuon else 2) + 2 * b.weight.element_size() + (2 if b.weight_copy is not None else 0))
+        o_reads = 1 if (not normuon or b.row_sumsq is not None) else 2
+        tot += e * (2 * o_reads + 2 * b.weight.element_size() + (2 if b.weight_copy is not None else 0))
     return tot
 
 
@@ -499,12 +556,9 @@ def run_ours(args, wl, variant, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch Philox on the device)",
-        "config": {"workload": DESCRIPTIONS[wl.key], "key": wl.key, "variant": variant,
-                   "coefficients": coefficients_desc(args), "slices": slices,
-                   "launch": ("CUDA graph of one whole step, replayed for each timed step" if args.graph == "on"
-                              else "eager calls"),
-                   "ns_flop_per_step": ns_flop, "l2": "inputs larger than L2 (126 MB), no flush",
-                   "parallelism": f"replicas x{world} (no exchange)"},
+        "config": dict(workload_config(args, wl, variant), parallelism=f"replicas x{world} (no exchange)"),
+        "launch": ("CUDA graph of one whole step, replayed for each timed step" if args.graph == "on"
+                   else "eager calls"),
         "pct_bf16_peak": round(100 * value / world / peak_s, 2),
         "pct_bf16_peak_burst": round(100 * value / world / peak_b, 2),
         "matrices_per_s": round(world * slices * args.steps / sec, 2),
@@ -533,10 +587,10 @@ def run_ours(args, wl, variant, rank, world, local_rank):
                               "from pinned host memory on a second stream (overlapping the previous shape's "
                               "optimizer work) and its per-slice norms read back D2H, all inside the timed region"}
     if world == 1 and not args.no_cpu_baseline:
-        flops, sl, dt, cores, desc = oracle_sample(wl, variant, abc=oracle_schedule(args, wl))
-        out["cpu_baseline"] = {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+        rate, slice_rate, dt, cores, desc = oracle_sample(wl, variant, abc=oracle_schedule(args, wl))
+        out["cpu_baseline"] = {"value": round(rate / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
                                "kind": "oracle", "sample": desc, "seconds": round(dt, 2),
-                               "matrices_per_s": round(sl / dt, 4)}
+                               "matrices_per_s": round(slice_rate, 4)}
     return out
 
 
@@ -551,27 +605,37 @@ def oracle_schedule(args, wl):
 
 
 def run_reference(args, wl, variant):
+    """The oracle on the host cores: step j runs the oracle on unit j mod U of the workload's sample
+    (one parameter of each distinct shape), so every step stays a few seconds; the rate weights the
+    units' mean times by their counts, as the cpu_baseline of the other arm does."""
+    import threadpoolctl
     peaks, _ = load_peaks()
     abc = oracle_schedule(args, wl)
-    budget = max(5.0, 60.0 / max(1, args.steps + args.warmup))
-    per_step = []
-    flops = sl = 0
-    cores, desc = 1, ""
-    for k in range(args.warmup + args.steps):
-        f, s, dt, cores, desc = oracle_sample(wl, variant, budget, abc=abc)
-        if k >= args.warmup:
-            per_step.append(dt)
-            flops, sl = f, s
-    sec = sum(per_step)
-    value = flops * args.steps / sec / 1e12
+    units = cpu_sample_units(wl, variant)
+    per_unit = [[] for _ in units]
+    step_s = []
+    with threadpoolctl.threadpool_limits(limits=os.cpu_count() or 1):
+        cores = host_threads()
+        for k in range(args.warmup + args.steps):
+            u = (k - args.warmup) % len(units) if k >= args.warmup else k % len(units)
+            res = oracle_unit(wl, units[u][0], variant, abc)
+            if k >= args.warmup:
+                per_unit[u].append(res)
+                step_s.append(res[2])
+        for u in range(len(units)):          # fewer timed steps than units: time the rest once
+            if not per_unit[u]:
+                per_unit[u].append(oracle_unit(wl, units[u][0], variant, abc))
+    means = [(r[0][0], r[0][1], statistics.mean(x[2] for x in r)) for r in per_unit]
+    rate, slice_rate = oracle_rate(units, means)
+    value = rate / 1e12
+    desc = oracle_sample_desc(wl, units) + f"; step j times unit j mod {len(units)}"
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sec / args.steps, 3),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(step_s), 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": DESCRIPTIONS[wl.key], "key": wl.key, "variant": variant,
-                   "coefficients": coefficients_desc(args), "sample": desc},
+        "config": dict(workload_config(args, wl, variant), parallelism=f"replicas x{args.gpus} (no exchange)"),
         "pct_bf16_peak": round(100 * value / peaks.get("bf16_tflops_sustained", 1400.0), 6),
-        "matrices_per_s": round(sl * args.steps / sec, 4),
+        "matrices_per_s": round(slice_rate, 4),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

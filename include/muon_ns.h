@@ -38,10 +38,12 @@
  * Streams and graphs.  A call enqueues only kernels on `stream`, launched
  * with programmatic stream serialization: each may start its prologue while
  * the previous kernel of the stream finishes and waits for it before
- * touching memory (set MUON_NS_PDL=0 to launch them plainly).  A whole step
+ * touching memory.  A whole step
  * can be captured in a CUDA graph; the first call on a device does one-time
  * set-up (kernel attributes, the driver's tensor-map encoder) and must run
- * before any capture on that device.
+ * before any capture on that device.  The set-up is redone when the device's
+ * context changes (after cudaDeviceReset); that call, too, must come before
+ * any capture.
  *
  * Errors.  Every argument is checked on the host before anything is
  * enqueued.  On any error the call returns a non-zero status and touches no
@@ -110,12 +112,22 @@ typedef struct {
   muon_view weight_copy;       /* optional bf16 copy of an f32 W (ptr NULL: none) */
   float* sumsq;                /* [n] f32: ||U||_F^2 per slice, or NULL */
   float* variance;             /* [n*rows] f32 NorMuon variance, slice-major; NULL without NorMuon */
-  float lr_scale;              /* shape factor of the update, from the PARAMETER's
-                                  (fan_out, fan_in): sqrt(max(1, fan_out/fan_in)) * extra
-                                  ([dion-121] review "Correctness — confirmed";
-                                  [mcore-lsm] scale_mode='spectral') */
-  int32_t reserved;
+  float* row_sumsq;            /* [n*rows] f32, slice-major, or NULL: the Newton-Schulz calls
+                                  write sum_j O_ij^2 of each stored (bf16) output row here, and
+                                  normuon_update takes the NorMuon row statistics from it instead
+                                  of reading O a second time */
+  int64_t fan_out;             /* the PARAMETER's fan_out = shape[0] and fan_in = prod(shape[1:])  */
+  int64_t fan_in;              /* (not the slice's: a head or a megabatch slice takes the whole
+                                  parameter's); they set the update's scale (muon_update_scale) */
 } muon_batch;
+
+/* Update scale modes ([mcore-lsm] LayerShardedMuon constructor: scale_mode,
+ * default 'spectral', times extra_scale_factor).  See muon_update_scale. */
+typedef enum { MUON_SCALE_SPECTRAL = 0, MUON_SCALE_RMS_NORM = 1 } muon_scale_mode;
+
+/* Gram form: re-form the Gram matrix from the current iterate every this many
+ * iterations (see muon_gram_ns_batched); 0 never. */
+#define MUON_GRAM_RESTART_DEFAULT 3
 
 /* Hyperparameters of one step ([mcore-lsm] LayerShardedMuon constructor). */
 typedef struct {
@@ -130,6 +142,12 @@ typedef struct {
   float weight_decay;          /* decoupled: W *= 1 - lr*weight_decay before the update */
   const float* abc_schedule;   /* optional HOST array [ns_steps][3] of per-iteration
                                   coefficients; NULL: (a, b, c) at every iteration */
+  int32_t scale_mode;          /* muon_scale_mode of the update's shape factor */
+  float extra_scale_factor;    /* multiplies the shape factor, 1.0 */
+  int32_t gram_restart;        /* Gram form: restart period in iterations, 0 = none;
+                                  MUON_GRAM_RESTART_DEFAULT (3) keeps rank-deficient inputs
+                                  in band with fp16 m x m iterates */
+  int32_t reserved;
 } muon_hparams;
 
 /* Bytes of workspace the given call needs for these batches.
@@ -163,9 +181,10 @@ MUON_API muon_status muon_momentum_norm(const muon_batch* batches, int nb, const
  * every iteration in one launch (a thread-block cluster per slice, the slice
  * held in shared memory, X X^T summed across the cluster in a fixed order);
  * the choice depends on the shape only, so a slice's result does not depend
- * on the rest of the batch.  Setting the environment variable
- * MUON_NS_FUSED_SMALL=0 sends them through the GEMM path instead.
- * Reads ns_in (left unchanged), sumsq; writes ns_out.
+ * on the rest of the batch.
+ * Reads ns_in (left unchanged), sumsq; writes ns_out, and row_sumsq when it
+ * is non-NULL (per output row, the sum of squares of the stored bf16 values,
+ * summed in a fixed order: tile partials from the last product's epilogue).
  */
 MUON_API muon_status muon_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp,
                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
@@ -177,9 +196,18 @@ MUON_API muon_status muon_ns_batched(const muon_batch* batches, int nb, const mu
  * G = X0 X0^T: A = G, Q = I; per iteration P = a*I + b*A + c*A^2,
  * Q <- P Q, A <- P A P; O = Q X0.  The m x m products use fp16 operands
  * (10-bit mantissa) with fp32 accumulation; X-side products use bf16.
+ * Restarts (hp->gram_restart = R > 0): before iterations R, 2R, ... the
+ * iterate X = Q X0 is formed (bf16) and the iteration starts again from it
+ * (A = X X^T, Q = I).  In exact arithmetic nothing changes (X_k = Q_k X0 and
+ * X_k X_k^T = Q_k G Q_k); in fp16, rounding can give A small negative
+ * eigenvalues on rank-deficient slices, which A <- P A P amplifies by about
+ * a^2 per iteration, and a restart bounds that growth.  Each restart costs
+ * one X-sized product and one Gram product (3 m^2 n) and saves three m x m
+ * products.
  * Small slices (as for muon_ns_batched) run in one launch: the cluster forms
- * G once and every CTA iterates on the m x m side.
- * Reads ns_in (left unchanged), sumsq; writes ns_out.
+ * G once (again at each restart) and every CTA iterates on the m x m side.
+ * Reads ns_in (left unchanged), sumsq; writes ns_out and row_sumsq (as
+ * muon_ns_batched).
  */
 MUON_API muon_status muon_gram_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp,
                                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
@@ -208,9 +236,14 @@ MUON_API muon_status muon_ns_auto_batched(const muon_batch* batches, int nb, con
  * With use_normuon:
  *   v_i <- beta2*v_i + (1-beta2) * mean_j O_ij^2           (per slice row i)
  *   Oh   = O_i / (sqrt(v_i) + nor_eps),  Oh *= ||O||_F / ||Oh||_F (0 stays 0)
- * else Oh = O.  Then W <- W*(1 - lr*weight_decay) - lr*lr_scale*Oh, and
- * weight_copy <- bf16(W) when given.
- * Reads ns_out, variance; writes variance, weight, weight_copy.
+ * else Oh = O.  Then W <- W*(1 - lr*weight_decay) - lr*scale*Oh, with
+ * scale = muon_update_scale(fan_out, fan_in, hp->scale_mode,
+ * hp->extra_scale_factor) of the batch's parameter, and weight_copy <- bf16(W)
+ * when given.  With use_normuon and row_sumsq non-NULL, sum_j O_ij^2 is taken
+ * from row_sumsq (as the preceding Newton-Schulz call wrote it) and O is read
+ * once; a caller whose ns_out did not come from those calls passes NULL.
+ * Reads ns_out, variance, row_sumsq; writes variance, weight, weight_copy.
+ * MUON_INVALID_ARG if fan_out or fan_in < 1 or the scale mode is unknown.
  */
 MUON_API muon_status normuon_update(const muon_batch* batches, int nb, const muon_hparams* hp,
                            int use_normuon, void* workspace, size_t workspace_bytes,
@@ -280,6 +313,26 @@ MUON_API muon_status muon_workspace_error(const void* workspace, cudaStream_t st
  */
 MUON_API muon_status muon_polar_express_schedule(double lower, int steps, double safety, float* abc_out,
                                                  double* err_out);
+
+/*
+ * The update's shape factor of one parameter of shape [fan_out, fan_in]
+ * (fan_in = prod of the other dims; [dion-121] review "Correctness —
+ * confirmed": a single parameter's shape, never a slice's), times `extra`
+ * ([mcore-lsm] extra_scale_factor):
+ *   MUON_SCALE_SPECTRAL  sqrt(max(1, fan_out / fan_in))    ([mcore-lsm] default
+ *                        'spectral'; the update's RMS-to-RMS operator norm is 1
+ *                        when fan_out >= fan_in)
+ *   MUON_SCALE_RMS_NORM  0.2 * sqrt(max(fan_out, fan_in))  (the pages name the
+ *                        mode, [dion-121] adjust_lr_rms_norm, but not its formula;
+ *                        this is the RMS matching of Liu et al., "Muon is Scalable
+ *                        for LLM Training" (2025): an orthogonal update then has
+ *                        element RMS 0.2, as AdamW's typically does)
+ * Host computation (double precision, rounded once to float).
+ * MUON_INVALID_ARG for fan_out or fan_in < 1, an unknown mode, a non-finite
+ * extra, or a NULL scale_out.
+ */
+MUON_API muon_status muon_update_scale(int64_t fan_out, int64_t fan_in, int32_t scale_mode, float extra,
+                                       float* scale_out);
 
 MUON_API const char* muon_status_string(muon_status status);
 

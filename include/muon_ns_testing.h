@@ -52,6 +52,28 @@ MUON_API muon_status muon_testing_gemm(int M, int N, int K, int slices, int tri,
 MUON_API muon_status muon_testing_bounded_wait(uint64_t limit_ns, void* workspace, size_t workspace_bytes,
                                                cudaStream_t stream);
 
+/*
+ * Kernel-selection switches for tests and experiments, process-wide (all
+ * devices, all threads); production callers never need them.  Defaults:
+ *   fused_small   1: slices with short side <= 128 and long side <= 4096 run
+ *                    the fused clustered kernel; 0: the GEMM path
+ *   max_waves    32: waves of tiles per GEMM launch (0: no cap)
+ *   max_problems  1: problems that share a GEMM launch beyond one wave (1..8)
+ *   pdl           1: programmatic dependent launch; 0: plain launches
+ * Sets *opts when non-NULL (after range checks: MUON_INVALID_ARG and no
+ * change when a value is out of range) and returns the previous switches in
+ * *previous when non-NULL.  Not to be called while another thread enqueues
+ * work through the library.
+ */
+typedef struct {
+  int32_t fused_small;
+  int32_t max_waves;
+  int32_t max_problems;
+  int32_t pdl;
+} muon_testing_options;
+
+MUON_API muon_status muon_testing_set_options(const muon_testing_options* opts, muon_testing_options* previous);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,9 +8,9 @@ streams only.  Every arithmetic step runs in the library's sm_100a kernels.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import dataclasses
-import math
 from typing import List, Optional, Sequence
 
 import torch
@@ -19,8 +19,9 @@ from . import _capi
 from ._capi import MUON_BF16, MUON_F16, MUON_F32, MuonError  # noqa: F401
 
 __all__ = ["Batch", "Hparams", "muon_workspace_size", "muon_momentum_norm", "muon_ns_batched",
-           "muon_gram_ns_batched", "normuon_update", "workspace_error", "testing_gemm", "spectral_scale",
-           "ns_flops", "version", "kernel_launches", "muon_momentum_norm_noalloc", "muon_ns_auto_batched", "polar_express_schedule", "allocate_workspace", "MuonError", "LIB_PATH"]
+           "muon_gram_ns_batched", "normuon_update", "workspace_error", "testing_gemm", "update_scale",
+           "ns_flops", "version", "kernel_launches", "muon_momentum_norm_noalloc", "muon_ns_auto_batched",
+           "polar_express_schedule", "allocate_workspace", "testing_options", "MuonError", "LIB_PATH"]
 
 LIB_PATH = _capi.LIB_PATH
 
@@ -57,24 +58,42 @@ def polar_express_schedule(lower: float = 1e-3, steps: int = 5, safety: float = 
     return coeffs, [err[t] for t in range(steps)]
 
 
-def spectral_scale(fan_out: int, fan_in: int, extra: float = 1.0) -> float:
-    """Update shape factor sqrt(max(1, fan_out/fan_in)) * extra of ONE parameter."""
-    return math.sqrt(max(1.0, fan_out / fan_in)) * extra
+def update_scale(fan_out: int, fan_in: int, mode: str = "spectral", extra: float = 1.0) -> float:
+    """The update's shape factor of ONE parameter [fan_out, fan_in], as the library computes it.
+
+    ``mode``: "spectral" or "rms_norm" (include/muon_ns.h, muon_update_scale).
+    """
+    out = ctypes.c_float(0.0)
+    _capi.check(_capi.lib.muon_update_scale(int(fan_out), int(fan_in), _capi.SCALE_MODES[mode], float(extra),
+                                            ctypes.byref(out)), "muon_update_scale")
+    return float(out.value)
 
 
-def ns_flops(rows: int, cols: int, variant: str = "standard", steps: int = 5) -> float:
+def ns_flops(rows: int, cols: int, variant: str = "standard", steps: int = 5,
+             gram_restart: int = _capi.MUON_GRAM_RESTART_DEFAULT) -> float:
     """Floating-point operations the library's kernels perform for one slice.
 
     Standard: per step X X^T (one triangle, m^2 n), b*A + c*A^2 (one
-    triangle, m^3) and B X (2 m^2 n).  Gram: X X^T (m^2 n), per step A^2,
-    P Q (from the second step) and the two factors of P A P (up to the
-    second-to-last step), each a one-triangle m^3, then Q X (2 m^2 n).
+    triangle, m^3) and B X (2 m^2 n).  Gram: X X^T (m^2 n); per step A^2,
+    P Q (except at a segment's first step, where Q = P) and the two factors
+    of P A P (except at a segment's last step), each a one-triangle m^3; at
+    each restart Q X (2 m^2 n) and X X^T (m^2 n); finally Q X (2 m^2 n).
     """
     m, n = min(rows, cols), max(rows, cols)
     if variant == "standard":
         return float(steps * (3 * m * m * n + m ** 3))
-    prods = sum(1 + (k > 0) + 2 * (k < steps - 1) for k in range(steps))
-    return float(3 * m * m * n + prods * m ** 3)
+    R = gram_restart
+
+    def restart_at(k):
+        return R > 0 and 0 < k < steps and k % R == 0
+
+    prods, restarts, seg = 0, 0, 0
+    for k in range(steps):
+        if restart_at(k):
+            restarts += 1
+            seg = k
+        prods += 1 + (k != seg) + 2 * (not (k == steps - 1 or restart_at(k + 1)))
+    return float(3 * m * m * n + restarts * 3 * m * m * n + prods * m ** 3)
 
 
 def _view(t: Optional[torch.Tensor], n: int, rows: int, cols: int, name: str) -> _capi.MuonView:
@@ -101,7 +120,10 @@ class Batch:
     """Same-shape slices [n, rows, cols] and the buffers one step touches.
 
     Tensors are 3-D [n, rows, cols] views (2-D is taken as n = 1) whose rows
-    are contiguous; ``sumsq`` is [n] and ``variance`` [n, rows], both fp32.
+    are contiguous; ``sumsq`` is [n], ``variance`` and ``row_sumsq`` [n, rows],
+    all fp32.  ``fan_out`` / ``fan_in`` are the shape of the PARAMETER the
+    slices come from (shape[0], prod(shape[1:])), which sets the update's
+    scale; ``normuon_update`` needs them.
     """
     n: int
     rows: int
@@ -114,7 +136,9 @@ class Batch:
     weight_copy: Optional[torch.Tensor] = None
     sumsq: Optional[torch.Tensor] = None
     variance: Optional[torch.Tensor] = None
-    lr_scale: float = 1.0
+    row_sumsq: Optional[torch.Tensor] = None
+    fan_out: int = 0
+    fan_in: int = 0
 
     def to_c(self) -> _capi.MuonBatch:
         b = _capi.MuonBatch()
@@ -126,7 +150,7 @@ class Batch:
         b.ns_out = _view(self.ns_out, *args, "ns_out")
         b.weight = _view(self.weight, *args, "weight")
         b.weight_copy = _view(self.weight_copy, *args, "weight_copy")
-        for name in ("sumsq", "variance"):
+        for name in ("sumsq", "variance", "row_sumsq"):
             t = getattr(self, name)
             if t is not None:
                 if t.dtype != torch.float32 or not t.is_contiguous():
@@ -135,7 +159,7 @@ class Batch:
                 if t.numel() != want:
                     raise ValueError(f"{name}: {want} elements expected, got {t.numel()}")
                 setattr(b, name, t.data_ptr())
-        b.lr_scale = float(self.lr_scale)
+        b.fan_out, b.fan_in = int(self.fan_out), int(self.fan_in)
         return b
 
 
@@ -151,6 +175,9 @@ class Hparams:
     lr: float = 0.02
     weight_decay: float = 0.0
     abc_schedule: Optional[Sequence[Sequence[float]]] = None
+    scale_mode: str = "spectral"
+    extra_scale_factor: float = 1.0
+    gram_restart: int = _capi.MUON_GRAM_RESTART_DEFAULT
 
     def to_c(self):
         h = _capi.MuonHparams()
@@ -158,6 +185,9 @@ class Hparams:
         h.a, h.b, h.c = (float(x) for x in self.abc)
         h.ns_steps = int(self.ns_steps)
         h.beta2, h.nor_eps, h.lr, h.weight_decay = self.beta2, self.nor_eps, self.lr, self.weight_decay
+        h.scale_mode = _capi.SCALE_MODES[self.scale_mode]
+        h.extra_scale_factor = float(self.extra_scale_factor)
+        h.gram_restart = int(self.gram_restart)
         keep = None
         if self.abc_schedule is not None:
             flat = [float(v) for row in self.abc_schedule for v in row]
@@ -257,6 +287,27 @@ def workspace_error(workspace: torch.Tensor, stream=None) -> int:
     _capi.check(_capi.lib.muon_workspace_error(workspace.data_ptr(), _stream_ptr(stream), ctypes.byref(out)),
                 "muon_workspace_error")
     return int(out.value)
+
+
+@contextlib.contextmanager
+def testing_options(**switches):
+    """Temporarily sets the library's kernel-selection switches (include/muon_ns_testing.h).
+
+    Keys: fused_small, max_waves, max_problems, pdl.  For tests and
+    experiments; production calls use the defaults.
+    """
+    prev = _capi.MuonTestingOptions()
+    _capi.check(_capi.lib.muon_testing_set_options(None, ctypes.byref(prev)), "muon_testing_set_options")
+    new = _capi.MuonTestingOptions(prev.fused_small, prev.max_waves, prev.max_problems, prev.pdl)
+    for k, v in switches.items():
+        if not hasattr(new, k):
+            raise KeyError(k)
+        setattr(new, k, int(v))
+    _capi.check(_capi.lib.muon_testing_set_options(ctypes.byref(new), None), "muon_testing_set_options")
+    try:
+        yield
+    finally:
+        _capi.lib.muon_testing_set_options(ctypes.byref(prev), None)
 
 
 def testing_gemm(A: torch.Tensor, a_mn: bool, B: torch.Tensor, b_mn: bool, C: torch.Tensor, *, K: int,

@@ -35,8 +35,8 @@ class MuonBatch(ctypes.Structure):
     _fields_ = [("n", ctypes.c_int64), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
                 ("grad", MuonView), ("momentum", MuonView), ("ns_in", MuonView), ("ns_out", MuonView),
                 ("weight", MuonView), ("weight_copy", MuonView),
-                ("sumsq", ctypes.c_void_p), ("variance", ctypes.c_void_p),
-                ("lr_scale", ctypes.c_float), ("reserved", ctypes.c_int32)]
+                ("sumsq", ctypes.c_void_p), ("variance", ctypes.c_void_p), ("row_sumsq", ctypes.c_void_p),
+                ("fan_out", ctypes.c_int64), ("fan_in", ctypes.c_int64)]
 
 
 class MuonHparams(ctypes.Structure):
@@ -44,13 +44,26 @@ class MuonHparams(ctypes.Structure):
                 ("a", ctypes.c_float), ("b", ctypes.c_float), ("c", ctypes.c_float),
                 ("ns_steps", ctypes.c_int32), ("beta2", ctypes.c_float), ("nor_eps", ctypes.c_float),
                 ("lr", ctypes.c_float), ("weight_decay", ctypes.c_float),
-                ("abc_schedule", ctypes.POINTER(ctypes.c_float))]
+                ("abc_schedule", ctypes.POINTER(ctypes.c_float)),
+                ("scale_mode", ctypes.c_int32), ("extra_scale_factor", ctypes.c_float),
+                ("gram_restart", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class MuonTestingOptions(ctypes.Structure):
+    _fields_ = [("fused_small", ctypes.c_int32), ("max_waves", ctypes.c_int32), ("max_problems", ctypes.c_int32),
+                ("pdl", ctypes.c_int32)]
+
+
+MUON_SCALE_SPECTRAL, MUON_SCALE_RMS_NORM = 0, 1
+SCALE_MODES = {"spectral": MUON_SCALE_SPECTRAL, "rms_norm": MUON_SCALE_RMS_NORM}
+MUON_GRAM_RESTART_DEFAULT = 3
 
 
 EXPORTS = ("muon_workspace_size", "muon_momentum_norm", "muon_ns_batched", "muon_gram_ns_batched",
            "normuon_update", "muon_workspace_error", "muon_status_string", "muon_version",
            "muon_testing_gemm", "muon_kernel_launches", "muon_momentum_norm_noalloc",
-           "muon_testing_bounded_wait", "muon_ns_auto_batched", "muon_polar_express_schedule")
+           "muon_testing_bounded_wait", "muon_ns_auto_batched", "muon_polar_express_schedule", "muon_update_scale",
+           "muon_testing_set_options")
 
 
 def _load() -> ctypes.CDLL:
@@ -95,6 +108,11 @@ def _load() -> ctypes.CDLL:
     lib.muon_testing_gemm.restype = ctypes.c_int
     lib.muon_testing_bounded_wait.argtypes = [ctypes.c_uint64, P, ctypes.c_size_t, P]
     lib.muon_testing_bounded_wait.restype = ctypes.c_int
+    lib.muon_update_scale.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_float,
+                                      ctypes.POINTER(ctypes.c_float)]
+    lib.muon_update_scale.restype = ctypes.c_int
+    lib.muon_testing_set_options.argtypes = [ctypes.POINTER(MuonTestingOptions), ctypes.POINTER(MuonTestingOptions)]
+    lib.muon_testing_set_options.restype = ctypes.c_int
     return lib
 
 

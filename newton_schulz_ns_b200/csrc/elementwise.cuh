@@ -37,6 +37,7 @@ struct EwSeg {
   void* w; long long w_ld, w_bs; int w_dt;
   void* wc; long long wc_ld, wc_bs;              // optional bf16 copy
   float* variance;                               // [n*rows]
+  const float* rsq;                              // [n*rows] per-row sum of O^2 from the NS call, or null
   float lr_scale;
 };
 
@@ -170,14 +171,16 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_chunks_kernel(const __gri
           float g[8], m[8];
           ld8(S.g, og, S.g_dt, g);
           ld8(S.m, om, S.m_dt, m);
+          // One rounding per operation (fused multiply-adds), in this order:
+          //   M_new = fl(mu*M + G),  U = fl(mu*M_new + G)  (from the unrounded M_new)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) m[i] = P.mu * m[i] + g[i];
+          for (int i = 0; i < 8; ++i) m[i] = fmaf(P.mu, m[i], g[i]);
           float mn[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) mn[i] = m[i];
           st8(S.m, om, S.m_dt, m);                                  // m now holds the stored values
 #pragma unroll
-          for (int i = 0; i < 8; ++i) u[i] = P.nesterov ? g[i] + P.mu * mn[i] : mn[i];
+          for (int i = 0; i < 8; ++i) u[i] = P.nesterov ? fmaf(P.mu, mn[i], g[i]) : mn[i];
           st8(S.u, ou, 1, u);                                       // u now holds bf16(U)
         } else {
           ld8(S.u, ou, 1, u);
@@ -192,9 +195,9 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_chunks_kernel(const __gri
         if (MODE == 0) {
           const float g = ld_f(S.g, slice * S.g_bs + r * S.g_ld + col, S.g_dt);
           const float mo = ld_f(S.m, slice * S.m_bs + r * S.m_ld + col, S.m_dt);
-          const float mn = P.mu * mo + g;
+          const float mn = fmaf(P.mu, mo, g);
           st_f(S.m, slice * S.m_bs + r * S.m_ld + col, mn, S.m_dt);
-          const float u = P.nesterov ? g + P.mu * mn : mn;
+          const float u = P.nesterov ? fmaf(P.mu, mn, g) : mn;
           const __nv_bfloat16 ub = __float2bfloat16_rn(u);
           reinterpret_cast<__nv_bfloat16*>(S.u)[slice * S.u_bs + r * S.u_ld + col] = ub;
           uv = __bfloat162float(ub);
@@ -233,18 +236,48 @@ __global__ void __launch_bounds__(EW_THREADS) sumsq_finalize_kernel(const __grid
 }
 
 // ---------------------------------------------------------------------------
-// NorMuon row statistics: one warp per row of O.
+// NorMuon row statistics.
 //   ss = sum_j O_ij^2;  v <- beta2*v + (1-beta2)*ss/cols;  d = 1/(sqrt(v)+eps)
+// Segments whose Newton-Schulz call left the row sums (rsq) take them from
+// there, one thread per row; the others read O, one warp per row.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void normuon_row_finish(const EwParams& P, const EwSeg& S, long long lr, long long gr,
+                                                   float ss) {
+  float* vp = S.variance + lr;
+  const float vn = P.beta2 * (*vp) + (1.0f - P.beta2) * (ss / static_cast<float>(S.cols));
+  *vp = vn;
+  P.row_ss[gr] = ss;
+  P.row_d[gr] = 1.0f / (sqrtf(vn) + P.nor_eps);
+}
+
+__device__ __forceinline__ int find_seg_by_row(const EwParams& P, long long gr) {
+  int si = 0;
+  while (si + 1 < P.nseg && gr >= P.seg[si + 1].row_begin) ++si;
+  return si;
+}
+
+__global__ void __launch_bounds__(EW_THREADS) normuon_rows_from_sums_kernel(const __grid_constant__ EwParams P) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
+  const long long threads = static_cast<long long>(gridDim.x) * EW_THREADS;
+  for (long long gr = static_cast<long long>(blockIdx.x) * EW_THREADS + threadIdx.x; gr < P.total_rows;
+       gr += threads) {
+    const EwSeg& S = P.seg[find_seg_by_row(P, gr)];
+    if (S.rsq == nullptr) continue;
+    const long long lr = gr - S.row_begin;
+    normuon_row_finish(P, S, lr, gr, S.rsq[lr]);
+  }
+}
+
 __global__ void __launch_bounds__(EW_THREADS) normuon_rows_kernel(const __grid_constant__ EwParams P) {
   pdl_launch_dependents();
   pdl_wait_prerequisites();
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (EW_THREADS / 32);
   for (long long gr = blockIdx.x * (EW_THREADS / 32) + (threadIdx.x >> 5); gr < P.total_rows; gr += warps) {
-    int si = 0;
-    while (si + 1 < P.nseg && gr >= P.seg[si + 1].row_begin) ++si;
+    const int si = find_seg_by_row(P, gr);
     const EwSeg& S = P.seg[si];
+    if (S.rsq != nullptr) continue;                 // warp-uniform
     const long long lr = gr - S.row_begin;
     const long long slice = lr / S.rows, r = lr - slice * S.rows;
     const __nv_bfloat16* o = reinterpret_cast<const __nv_bfloat16*>(S.o) + slice * S.o_bs + r * S.o_ld;
@@ -264,13 +297,47 @@ __global__ void __launch_bounds__(EW_THREADS) normuon_rows_kernel(const __grid_c
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      float* vp = S.variance + lr;
-      const float vn = P.beta2 * (*vp) + (1.0f - P.beta2) * (acc / static_cast<float>(S.cols));
-      *vp = vn;
-      P.row_ss[gr] = acc;
-      P.row_d[gr] = 1.0f / (sqrtf(vn) + P.nor_eps);
+    if (lane == 0) normuon_row_finish(P, S, lr, gr, acc);
+  }
+}
+
+// Per-row sums of squares of a Newton-Schulz output from per-tile partials:
+// out[s][r] = sum over t < nt, in order, of part[(s nt + t) rows + r].
+__global__ void __launch_bounds__(EW_THREADS) row_partials_finalize_kernel(const float* part, int nt, long long rows,
+                                                                           long long n, float* out) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
+  const long long total = n * rows;
+  const long long threads = static_cast<long long>(gridDim.x) * EW_THREADS;
+  for (long long i = static_cast<long long>(blockIdx.x) * EW_THREADS + threadIdx.x; i < total; i += threads) {
+    const long long sl = i / rows, r = i - sl * rows;
+    const float* p = part + sl * nt * rows + r;
+    float acc = 0.0f;
+    for (int t = 0; t < nt; ++t) acc += p[static_cast<long long>(t) * rows];
+    out[i] = acc;
+  }
+}
+
+// Per-row sums of squares of a bf16 [n][rows][cols] strided view, one warp
+// per row: out[s][r] = sum_j O[s][r][j]^2.
+__global__ void __launch_bounds__(EW_THREADS) rows_sumsq_kernel(const __nv_bfloat16* O, long long ld, long long bs,
+                                                                long long rows, long long cols, long long n,
+                                                                float* out) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (EW_THREADS / 32);
+  for (long long i = blockIdx.x * (EW_THREADS / 32) + (threadIdx.x >> 5); i < n * rows; i += warps) {
+    const long long sl = i / rows, r = i - sl * rows;
+    const __nv_bfloat16* o = O + sl * bs + r * ld;
+    float acc = 0.0f;
+    for (long long j = lane; j < cols; j += 32) {
+      const float v = __bfloat162float(o[j]);
+      acc += v * v;
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) out[i] = acc;
   }
 }
 

@@ -43,6 +43,7 @@ inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 struct DeviceInfo {
   bool ready = false;
   bool ok = false;
+  unsigned long long ctx_id = 0;   // context the set-up was done in (0: none yet)
   int sms = 0;
   int pair_units = 0;   // 2-CTA clusters of the pair GEMM that fit on the device at once
 };
@@ -50,6 +51,48 @@ std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::atomic<unsigned long long> g_launches{0};
+
+// Kernel-selection switches (muon_testing_set_options); production values by default.
+struct Options {
+  std::atomic<int> fused_small{1};
+  std::atomic<int> max_waves{32};
+  std::atomic<int> max_problems{1};
+  std::atomic<int> pdl{1};
+};
+Options g_opt;
+
+// The driver's context queries, resolved at run time like the tensor-map
+// encoder (the library does not link the driver).
+typedef CUresult (*PFN_ctx_get_current)(CUcontext*);
+typedef CUresult (*PFN_ctx_get_id)(CUcontext, unsigned long long*);
+PFN_ctx_get_current g_ctx_current = nullptr;
+PFN_ctx_get_id g_ctx_id = nullptr;
+
+template <typename F>
+bool driver_entry(const char* name, F* out) {
+  if (*out) return true;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess ||
+      fn == nullptr) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  *out = reinterpret_cast<F>(fn);
+  return true;
+}
+
+// Unique id of the calling thread's current context (0 when there is none
+// yet or the query is unavailable).  Per-device set-up is keyed by it, so a
+// context torn down and re-created (cudaDeviceReset) gets fresh set-up.
+unsigned long long current_ctx_id() {
+  if (!driver_entry("cuCtxGetCurrent", &g_ctx_current) || !driver_entry("cuCtxGetId", &g_ctx_id)) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Checks the launch just enqueued and counts it.
 inline bool launched() {
@@ -60,14 +103,8 @@ inline bool launched() {
 
 // Programmatic dependent launch for every kernel of the step: each kernel
 // lets the next one start its prologue and waits for its predecessor before
-// its first global access.  MUON_NS_PDL=0 launches them plainly.
-inline bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = std::getenv("MUON_NS_PDL");
-    return !(e && std::atoi(e) == 0);
-  }();
-  return on;
-}
+// its first global access (switchable for tests, muon_testing_set_options).
+inline bool pdl_enabled() { return g_opt.pdl.load(std::memory_order_relaxed) != 0; }
 
 template <typename... KArgs, typename... Args>
 bool launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args&&... args) {
@@ -98,6 +135,8 @@ muon_status device_setup(int* sms_out, int* pair_units_out = nullptr) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MUON_CUDA_ERROR;
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceInfo& d = g_dev[dev];
+  const unsigned long long ctx = current_ctx_id();
+  if (d.ready && ctx != 0 && ctx != d.ctx_id) d.ready = false;   // a new context: kernel attributes are gone
   if (!d.ready) {
     d.ready = true;
     int major = 0, minor = 0, sms = 0;
@@ -142,6 +181,7 @@ muon_status device_setup(int* sms_out, int* pair_units_out = nullptr) {
       }
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
+    d.ctx_id = current_ctx_id();   // the calls above made the context current if it was not
   }
   if (!d.ok) return MUON_UNSUPPORTED_DEVICE;
   *sms_out = d.sms;
@@ -209,7 +249,28 @@ muon_status check_hp(const muon_hparams* hp) {
   if (hp->abc_schedule)
     for (int i = 0; i < 3 * hp->ns_steps; ++i)
       if (!std::isfinite(hp->abc_schedule[i])) return MUON_INVALID_ARG;
+  if (hp->scale_mode != MUON_SCALE_SPECTRAL && hp->scale_mode != MUON_SCALE_RMS_NORM) return MUON_INVALID_ARG;
+  if (!std::isfinite(hp->extra_scale_factor)) return MUON_INVALID_ARG;
+  if (hp->gram_restart < 0 || hp->gram_restart > 16) return MUON_INVALID_ARG;
   return MUON_OK;
+}
+
+// The update's shape factor of a parameter [fan_out, fan_in] (see
+// muon_update_scale in the header for the two modes and their sources).
+bool update_scale(int64_t fan_out, int64_t fan_in, int32_t mode, float extra, float* out) {
+  if (fan_out < 1 || fan_in < 1 || !std::isfinite(extra)) return false;
+  const double fo = static_cast<double>(fan_out), fi = static_cast<double>(fan_in);
+  double base;
+  if (mode == MUON_SCALE_SPECTRAL)
+    base = std::sqrt(std::max(1.0, fo / fi));
+  else if (mode == MUON_SCALE_RMS_NORM)
+    base = 0.2 * std::sqrt(std::max(fo, fi));
+  else
+    return false;
+  const double v = base * static_cast<double>(extra);
+  if (!std::isfinite(v)) return false;
+  *out = static_cast<float>(v);
+  return true;
 }
 
 muon_status check_ws(void* ws, size_t have, size_t need) {
@@ -222,12 +283,21 @@ muon_status check_ws(void* ws, size_t have, size_t need) {
 
 // ---------------------------------------------------------------- workspace layout
 struct NsBatchWs {
-  size_t off[5] = {0, 0, 0, 0, 0};   // standard: A, B, X ; gram: Ah, P, Qa, Qb, R
+  size_t off[6] = {0, 0, 0, 0, 0, 0};   // standard: A, B, X ; gram: Ah, P, Qa, Qb, R, X
   int64_t ldm = 0, bsm = 0;         // m x m buffers
   int64_t ldx = 0, bsx = 0;         // X buffer
   size_t t_off = 0;                 // tall slices on the fused path: the transposed slice [cols][rows]
   int64_t ldt = 0, bst = 0;
+  size_t rs_off = 0;                // row_sumsq requested: per-tile partial row sums [n][rs_nt][rows]
+  int rs_nt = 0;
 };
+
+// Partial row sums per output row that the last product leaves: one per
+// 256-column tile on the GEMM path, one per CTA and column half on the fused
+// path (clusters of at most SMALL_MAX_CLUSTER CTAs).
+inline int row_partials_per_row(int64_t cols) {
+  return static_cast<int>(std::max<int64_t>((cols + BN - 1) / BN, 2 * SMALL_MAX_CLUSTER));
+}
 
 bool small_shape_ok(int64_t rows, int64_t cols);
 
@@ -268,14 +338,21 @@ Layout plan_layout(const muon_batch* bs, int nb, int which) {
       w.ldm = round_up64(m, 64);
       w.bsm = w.ldm * m;
       const size_t mm = sizeof(uint16_t) * static_cast<size_t>(w.bsm) * static_cast<size_t>(b.n);
+      w.ldx = round_up64(b.cols, 64);
+      w.bsx = w.ldx * b.rows;
+      const size_t xbytes = sizeof(uint16_t) * static_cast<size_t>(w.bsx) * static_cast<size_t>(b.n);
       if (which == 1) {
-        w.ldx = round_up64(b.cols, 64);
-        w.bsx = w.ldx * b.rows;
         w.off[0] = take(mm);
         w.off[1] = take(mm);
-        w.off[2] = take(sizeof(uint16_t) * static_cast<size_t>(w.bsx) * static_cast<size_t>(b.n));
+        w.off[2] = take(xbytes);
       } else {
         for (int k = 0; k < 5; ++k) w.off[k] = take(mm);
+        w.off[5] = take(xbytes);    // the iterate a restart forms (the fused kernel keeps it on chip)
+      }
+      if (b.row_sumsq != nullptr) {
+        w.rs_nt = row_partials_per_row(b.cols);
+        w.rs_off = take(sizeof(float) * static_cast<size_t>(b.n) * static_cast<size_t>(w.rs_nt) *
+                        static_cast<size_t>(b.rows));
       }
       if (b.rows > b.cols && small_shape_ok(b.cols, b.rows)) {
         w.ldt = round_up64(b.rows, 64);
@@ -360,16 +437,10 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
   // projection shapes read 3x the DRAM bytes of per-shape launches).
   // Launches are therefore kept short: at most `max_problems` problems and
   // about `max_waves` waves of tiles each (a problem's slices are split
-  // across launches when needed).  Both can be overridden through the
-  // environment (MUON_NS_MAX_PROBLEMS, MUON_NS_MAX_WAVES; 0 waves = no cap).
-  static const int max_problems = [] {
-    const char* e = std::getenv("MUON_NS_MAX_PROBLEMS");
-    return e ? std::max(1, std::min(MAX_PROBLEMS, std::atoi(e))) : 1;
-  }();
-  static const int max_waves = [] {
-    const char* e = std::getenv("MUON_NS_MAX_WAVES");
-    return e ? std::max(0, std::atoi(e)) : 32;
-  }();
+  // across launches when needed).  Tests can change both
+  // (muon_testing_set_options; 0 waves = no cap).
+  const int max_problems = std::max(1, std::min(MAX_PROBLEMS, g_opt.max_problems.load(std::memory_order_relaxed)));
+  const int max_waves = std::max(0, g_opt.max_waves.load(std::memory_order_relaxed));
   auto pick_cg = [&](const ProblemSpec& s) {
     if (cta_pair == 2) return 2;
     if (cta_pair == 1 || pair_units <= 0) return 1;
@@ -510,7 +581,6 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
   // Programmatic dependent launch: each GEMM may start its prologue (barrier
   // setup, TMEM allocation) on idle SMs while the previous kernel drains; the
   // kernel waits for its predecessor before touching global memory.
-  // MUON_NS_PDL=0 launches them plainly.
   const bool pdl = pdl_enabled();
   for (const Launch& L : launches) {
     cudaLaunchConfig_t cfg = {};
@@ -666,19 +736,41 @@ bool small_shape_ok(int64_t rows, int64_t cols) {
 // the whole iteration in one clustered launch (ns_small.cuh); tall ones
 // (rows > cols) are transposed into the workspace first and back after.
 // The choice depends on the shape only, so a slice's result never depends
-// on the rest of the batch.  Setting MUON_NS_FUSED_SMALL=0 sends them
-// through the GEMM path instead.
+// on the rest of the batch (tests can send them through the GEMM path,
+// muon_testing_set_options).
 bool small_eligible(const muon_batch& b) {
-  const char* e = std::getenv("MUON_NS_FUSED_SMALL");
-  if (e && std::atoi(e) == 0) return false;
+  if (g_opt.fused_small.load(std::memory_order_relaxed) == 0) return false;
   return b.rows > b.cols ? small_shape_ok(b.cols, b.rows) : small_shape_ok(b.rows, b.cols);
 }
 
+// Row sums of squares of a Newton-Schulz output from its tile partials
+// ([n][nt][rows], summed in tile order) into the caller's row_sumsq.
+muon_status launch_row_finalize(const float* part, int nt, int64_t rows, int64_t n, float* out, int sms,
+                                cudaStream_t stream) {
+  const bool ok = launch_pdl(row_partials_finalize_kernel, dim3(ew_grid(cdiv(n * rows, EW_THREADS), sms)),
+                             dim3(EW_THREADS), 0, stream, part, nt, static_cast<long long>(rows),
+                             static_cast<long long>(n), out);
+  return ok ? MUON_OK : MUON_CUDA_ERROR;
+}
+
+// Row sums of squares read from the output itself (tall slices of the fused path).
+muon_status launch_rows_sumsq(const muon_batch& b, int sms, cudaStream_t stream) {
+  const int64_t bs = b.n > 1 ? b.ns_out.batch_stride : b.rows * b.ns_out.ld;
+  const bool ok = launch_pdl(rows_sumsq_kernel, dim3(ew_grid(cdiv(b.n * b.rows, EW_THREADS / 32), sms)),
+                             dim3(EW_THREADS), 0, stream, static_cast<const __nv_bfloat16*>(b.ns_out.ptr),
+                             static_cast<long long>(b.ns_out.ld), static_cast<long long>(bs),
+                             static_cast<long long>(b.rows), static_cast<long long>(b.cols),
+                             static_cast<long long>(b.n), b.row_sumsq);
+  return ok ? MUON_OK : MUON_CUDA_ERROR;
+}
+
 muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const float* sumsq, int* err, bool gram,
-                         cudaStream_t stream) {
+                         float* row_partials, cudaStream_t stream) {
   const SmallSplit sp = small_split(b.cols);
   SmallParams P;
   std::memset(&P, 0, sizeof(P));
+  P.row_ss = row_partials;
+  P.restart = gram ? hp->gram_restart : 0;
   if (!encode_map(&P.map_in, view_mat(b, b.ns_in), 64, 128)) return MUON_CUDA_ERROR;
   if (!encode_map(&P.map_out, view_mat(b, b.ns_out), 64, 128)) return MUON_CUDA_ERROR;
   P.tma_store = (b.cols % 8 == 0) ? 1 : 0;
@@ -741,8 +833,13 @@ muon_status launch_transpose16(const void* in, int64_t in_ld, int64_t in_bs, voi
 // copy in the workspace (the kernel then works in place on that copy: each
 // CTA reads its columns before writing them back).
 muon_status run_small(const muon_batch& b, const NsBatchWs& w, uint8_t* ws, const muon_hparams* hp,
-                      const float* sumsq, int* err, bool gram, cudaStream_t stream) {
-  if (b.rows <= b.cols) return launch_small(b, hp, sumsq, err, gram, stream);
+                      const float* sumsq, int* err, bool gram, int sms, cudaStream_t stream) {
+  if (b.rows <= b.cols) {
+    float* part = b.row_sumsq ? reinterpret_cast<float*>(ws + w.rs_off) : nullptr;
+    muon_status st = launch_small(b, hp, sumsq, err, gram, part, stream);
+    if (st != MUON_OK || part == nullptr) return st;
+    return launch_row_finalize(part, 2 * small_split(b.cols).C, b.rows, b.n, b.row_sumsq, sms, stream);
+  }
   void* T = ws + w.t_off;
   const int64_t in_bs = b.n > 1 ? b.ns_in.batch_stride : b.rows * b.ns_in.ld;
   const int64_t out_bs = b.n > 1 ? b.ns_out.batch_stride : b.rows * b.ns_out.ld;
@@ -753,9 +850,12 @@ muon_status run_small(const muon_batch& b, const NsBatchWs& w, uint8_t* ws, cons
   v.cols = b.rows;
   v.ns_in = muon_view{T, w.ldt, w.bst, MUON_BF16, 0};
   v.ns_out = v.ns_in;
-  if ((st = launch_small(v, hp, sumsq, err, gram, stream)) != MUON_OK) return st;
-  return launch_transpose16(T, w.ldt, w.bst, const_cast<void*>(b.ns_out.ptr), b.ns_out.ld, out_bs, b.cols, b.rows,
-                            b.n, stream);
+  if ((st = launch_small(v, hp, sumsq, err, gram, nullptr, stream)) != MUON_OK) return st;
+  if ((st = launch_transpose16(T, w.ldt, w.bst, const_cast<void*>(b.ns_out.ptr), b.ns_out.ld, out_bs, b.cols, b.rows,
+                               b.n, stream)) != MUON_OK)
+    return st;
+  // The kernel's rows were the slice's columns: the output rows' sums are read back from ns_out.
+  return b.row_sumsq ? launch_rows_sumsq(b, sms, stream) : MUON_OK;
 }
 
 // SYRK of the slice storage X ([rows][cols]) on the short side: out = f * X X^T (rows <= cols)
@@ -916,17 +1016,24 @@ static __device__ __align__(256) float g_noalloc_partials[MUON_NOALLOC_SCRATCH_F
 namespace {
 std::mutex g_noalloc_mu;
 float* g_noalloc_addr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};
 
 // Device address of g_noalloc_partials on the current device, looked up once
-// per device with that device current.
+// per device (and again if the device's context was re-created, which can
+// load the module at another address) with that device current.
 muon_status noalloc_scratch(float** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MUON_CUDA_ERROR;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
+  const unsigned long long ctx = current_ctx_id();
+  if (!g_noalloc_addr[dev] || (ctx != 0 && ctx != g_noalloc_ctx[dev])) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_partials) != cudaSuccess || p == nullptr) return MUON_CUDA_ERROR;
+    if (cudaGetSymbolAddress(&p, g_noalloc_partials) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      return MUON_CUDA_ERROR;
+    }
     g_noalloc_addr[dev] = static_cast<float*>(p);
+    g_noalloc_ctx[dev] = current_ctx_id();
   }
   *out = g_noalloc_addr[dev];
   return MUON_OK;
@@ -970,6 +1077,35 @@ muon_status muon_polar_express_schedule(double lower, int steps, double safety, 
 }
 
 uint64_t muon_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+muon_status muon_update_scale(int64_t fan_out, int64_t fan_in, int32_t scale_mode, float extra, float* scale_out) {
+  if (scale_out == nullptr) return MUON_INVALID_ARG;
+  float v = 0.0f;
+  if (!update_scale(fan_out, fan_in, scale_mode, extra, &v)) return MUON_INVALID_ARG;
+  *scale_out = v;
+  return MUON_OK;
+}
+
+muon_status muon_testing_set_options(const muon_testing_options* opts, muon_testing_options* previous) {
+  muon_testing_options cur;
+  cur.fused_small = g_opt.fused_small.load();
+  cur.max_waves = g_opt.max_waves.load();
+  cur.max_problems = g_opt.max_problems.load();
+  cur.pdl = g_opt.pdl.load();
+  if (opts) {
+    if ((opts->fused_small != 0 && opts->fused_small != 1) || opts->max_waves < 0 || opts->max_waves > 1000000 ||
+        opts->max_problems < 1 || opts->max_problems > MAX_PROBLEMS || (opts->pdl != 0 && opts->pdl != 1))
+      return MUON_INVALID_ARG;
+  }
+  if (previous) *previous = cur;
+  if (opts) {
+    g_opt.fused_small.store(opts->fused_small);
+    g_opt.max_waves.store(opts->max_waves);
+    g_opt.max_problems.store(opts->max_problems);
+    g_opt.pdl.store(opts->pdl);
+  }
+  return MUON_OK;
+}
 
 const char* muon_status_string(muon_status s) {
   switch (s) {
@@ -1076,6 +1212,20 @@ muon_status muon_gram_ns_batched(const muon_batch* batches, int nb, const muon_h
 
 }  // extern "C"
 
+// Row sums of squares of the GEMM path's outputs from the last product's tile partials.
+muon_status finalize_gemm_row_sums(const muon_batch* batches, int nb, const Layout& L, uint8_t* ws,
+                                   const std::vector<char>& fused, int sms, cudaStream_t stream) {
+  for (int i = 0; i < nb; ++i) {
+    const muon_batch& b = batches[i];
+    if (batch_empty(b) || fused[i] || !b.row_sumsq) continue;
+    const muon_status st = launch_row_finalize(reinterpret_cast<const float*>(ws + L.nsb[i].rs_off),
+                                               static_cast<int>(cdiv(b.cols, BN)), b.rows, b.n, b.row_sumsq, sms,
+                                               stream);
+    if (st != MUON_OK) return st;
+  }
+  return MUON_OK;
+}
+
 muon_status ns_standard_impl(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
                              size_t workspace_bytes, cudaStream_t stream, bool clear_err) {
   muon_status st = validate_ns(batches, nb, hp);
@@ -1096,7 +1246,7 @@ muon_status ns_standard_impl(const muon_batch* batches, int nb, const muon_hpara
   for (int i = 0; i < nb; ++i) {
     if (batch_empty(batches[i]) || !small_eligible(batches[i])) continue;
     fused[i] = 1;
-    if ((st = run_small(batches[i], L.nsb[i], ws, hp, sumsq[i], err, false, stream)) != MUON_OK) return st;
+    if ((st = run_small(batches[i], L.nsb[i], ws, hp, sumsq[i], err, false, sms, stream)) != MUON_OK) return st;
   }
   const int S = hp->ns_steps;
   for (int it = 0; it < S; ++it) {
@@ -1121,14 +1271,15 @@ muon_status ns_standard_impl(const muon_batch* batches, int nb, const muon_hpara
       const Mat Bm{Bbuf, m, m, w.ldm, w.bsm, b.n, 0};
       syrk.push_back(syrk_spec(b, src, Abuf, w.ldm, w.bsm, 0, 1.0f, it == 0 ? 2 : 0, sumsq[i], hp->ns_eps));
       poly.push_back(sym_spec(m, static_cast<int>(b.n), Am, Am, Bbuf, w.ldm, w.bsm, 0, cf.c, cf.b, Abuf, 0, 0.0f));
+      float* rs = (it == S - 1 && b.row_sumsq) ? reinterpret_cast<float*>(ws + w.rs_off) : nullptr;
       apply.push_back(apply_spec(b, Bm, src, const_cast<void*>(dst.ptr), dst.ld, dst.bs, cf.a, it == 0 ? 1 : 0,
-                                 sumsq[i], hp->ns_eps, nullptr));
+                                 sumsq[i], hp->ns_eps, rs));
     }
     if ((st = launch_gemms(syrk, sms, err, stream)) != MUON_OK) return st;
     if ((st = launch_gemms(poly, sms, err, stream)) != MUON_OK) return st;
     if ((st = launch_gemms(apply, sms, err, stream)) != MUON_OK) return st;
   }
-  return MUON_OK;
+  return finalize_gemm_row_sums(batches, nb, L, ws, fused, sms, stream);
 }
 
 muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
@@ -1153,7 +1304,7 @@ muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* 
   for (int i = 0; i < nb; ++i) {
     if (batch_empty(batches[i]) || !small_eligible(batches[i])) continue;
     fused[i] = 1;
-    if ((st = run_small(batches[i], L.nsb[i], ws, hp, sumsq[i], err, true, stream)) != MUON_OK) return st;
+    if ((st = run_small(batches[i], L.nsb[i], ws, hp, sumsq[i], err, true, sms, stream)) != MUON_OK) return st;
   }
   // G: kappa * s^2 * X X^T (short side) in fp16.
   {
@@ -1166,11 +1317,46 @@ muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* 
     }
     if ((st = launch_gemms(g, sms, err, stream)) != MUON_OK) return st;
   }
-  // Buffers: 0 Ah (kappa*A), 1 P, 2 Qa, 3 Qb, 4 R.  P of step 0 is written to Qa (Q_1 = P_1).
+  // Restarts: before iterations R, 2R, ... (R = gram_restart) the iterate
+  // X = f Q X_prev is formed in bf16 (f = s while X_prev is the unnormalized
+  // input) and the iteration starts again from it: A = kappa X X^T, Q = I.
+  // Writes of X alternate between the X workspace and ns_out so that the
+  // final O = f Q X lands in ns_out; ns_in is only read.
+  const int R = hp->gram_restart;
+  auto restart_at = [&](int k) { return R > 0 && k > 0 && k < S && k % R == 0; };
+  const int restarts = R > 0 ? (S - 1) / R : 0;
+  int xwrites = 0;                     // X-sized outputs written so far (restarts, then O)
+  const int xtotal = restarts + 1;
+  auto x_dst_is_out = [&](int j) { return (xtotal - 1 - j) % 2 == 0; };
+  // Buffers: 0 Ah (kappa*A), 1 P, 2 Qa, 3 Qb, 4 R, 5 X.  At the start of a
+  // segment P is written straight into the current Q buffer (Q = P).
   int qcur = 2;
+  int seg_start = 0;
   for (int k = 0; k < S; ++k) {
     const Coefs cf = coefs_at(hp, k);
     const bool last = (k == S - 1);
+    const bool end = last || restart_at(k + 1);   // last iteration of its segment: Q goes into an X product
+    if (restart_at(k)) {
+      std::vector<ProblemSpec> xs, gs;
+      for (int i = 0; i < nb; ++i) {
+        const muon_batch& b = batches[i];
+        if (batch_empty(b) || fused[i]) continue;
+        const NsBatchWs& w = L.nsb[i];
+        const int m = static_cast<int>(std::min(b.rows, b.cols));
+        const Mat Q{ws + w.off[qcur], m, m, w.ldm, w.bsm, b.n, 0};
+        const Mat xws{ws + w.off[5], b.rows, b.cols, w.ldx, w.bsx, b.n, 0};
+        const Mat src = xwrites == 0 ? view_mat(b, b.ns_in) : (x_dst_is_out(xwrites - 1) ? view_mat(b, b.ns_out) : xws);
+        const Mat dst = x_dst_is_out(xwrites) ? view_mat(b, b.ns_out) : xws;
+        xs.push_back(apply_spec(b, Q, src, const_cast<void*>(dst.ptr), dst.ld, dst.bs, 0.0f, xwrites == 0 ? 1 : 0,
+                                sumsq[i], hp->ns_eps, nullptr));
+        gs.push_back(syrk_spec(b, dst, ws + w.off[0], w.ldm, w.bsm, 1, kap, 0, sumsq[i], hp->ns_eps));
+      }
+      if ((st = launch_gemms(xs, sms, err, stream)) != MUON_OK) return st;
+      if ((st = launch_gemms(gs, sms, err, stream)) != MUON_OK) return st;
+      ++xwrites;
+      seg_start = k;
+    }
+    const bool first = (k == seg_start);
     std::vector<ProblemSpec> t_l, qr_l, a_l;
     int qnext = qcur;
     for (int i = 0; i < nb; ++i) {
@@ -1180,17 +1366,17 @@ muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* 
       const int m = static_cast<int>(std::min(b.rows, b.cols));
       const int sl = static_cast<int>(b.n);
       auto M16 = [&](int idx, int f16) { return Mat{ws + w.off[idx], m, m, w.ldm, w.bsm, b.n, f16}; };
-      const int pidx = (k == 0) ? 2 : 1;
-      // P = a I + (b/kappa) Ah + (c/kappa^2) Ah^2 ; bf16 when it is the final Q (one step only).
-      const int p_f16 = (k == 0 && last) ? 0 : 1;
+      const int pidx = first ? qcur : 1;
+      // P = a I + (b/kappa) Ah + (c/kappa^2) Ah^2 ; bf16 when it is the segment's final Q.
+      const int p_f16 = (first && end) ? 0 : 1;
       t_l.push_back(sym_spec(m, sl, M16(0, 1), M16(0, 1), ws + w.off[pidx], w.ldm, w.bsm, p_f16, cf.c / (kap * kap),
                              cf.b / kap, ws + w.off[0], 1, cf.a));
-      if (k > 0) {
+      if (!first) {
         qnext = (qcur == 2) ? 3 : 2;
-        qr_l.push_back(sym_spec(m, sl, M16(1, 1), M16(qcur, 1), ws + w.off[qnext], w.ldm, w.bsm, last ? 0 : 1, 1.0f,
+        qr_l.push_back(sym_spec(m, sl, M16(1, 1), M16(qcur, 1), ws + w.off[qnext], w.ldm, w.bsm, end ? 0 : 1, 1.0f,
                                 0.0f, nullptr, 1, 0.0f));
       }
-      if (!last) {
+      if (!end) {
         qr_l.push_back(sym_spec(m, sl, M16(pidx, 1), M16(0, 1), ws + w.off[4], w.ldm, w.bsm, 1, 1.0f, 0.0f, nullptr,
                                 1, 0.0f));
         a_l.push_back(sym_spec(m, sl, M16(pidx, 1), M16(4, 1), ws + w.off[0], w.ldm, w.bsm, 1, 1.0f, 0.0f, nullptr,
@@ -1202,7 +1388,7 @@ muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* 
     if ((st = launch_gemms(a_l, sms, err, stream)) != MUON_OK) return st;
     qcur = qnext;
   }
-  // O = s * Q X0 on the short side, Q in bf16.
+  // O = f Q X on the short side, Q in bf16 (f = s when no restart happened).
   {
     std::vector<ProblemSpec> o;
     for (int i = 0; i < nb; ++i) {
@@ -1211,13 +1397,16 @@ muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* 
       const NsBatchWs& w = L.nsb[i];
       const int m = static_cast<int>(std::min(b.rows, b.cols));
       const Mat Q{ws + w.off[qcur], m, m, w.ldm, w.bsm, b.n, 0};
+      const Mat xws{ws + w.off[5], b.rows, b.cols, w.ldx, w.bsx, b.n, 0};
+      const Mat src = xwrites == 0 ? view_mat(b, b.ns_in) : (x_dst_is_out(xwrites - 1) ? view_mat(b, b.ns_out) : xws);
       const Mat out = view_mat(b, b.ns_out);
-      o.push_back(apply_spec(b, Q, view_mat(b, b.ns_in), const_cast<void*>(out.ptr), out.ld, out.bs, 0.0f, 1,
-                             sumsq[i], hp->ns_eps, nullptr));
+      float* rs = b.row_sumsq ? reinterpret_cast<float*>(ws + w.rs_off) : nullptr;
+      o.push_back(apply_spec(b, Q, src, const_cast<void*>(out.ptr), out.ld, out.bs, 0.0f, xwrites == 0 ? 1 : 0,
+                             sumsq[i], hp->ns_eps, rs));
     }
     if ((st = launch_gemms(o, sms, err, stream)) != MUON_OK) return st;
   }
-  return MUON_OK;
+  return finalize_gemm_row_sums(batches, nb, L, ws, fused, sms, stream);
 }
 
 extern "C" {
@@ -1265,7 +1454,8 @@ muon_status normuon_update(const muon_batch* batches, int nb, const muon_hparams
     if ((st = check_view(b, b.weight, {MUON_F32, MUON_BF16}, false)) != MUON_OK) return st;
     if (b.weight_copy.ptr && (st = check_view(b, b.weight_copy, {MUON_BF16}, false)) != MUON_OK) return st;
     if (use_normuon && !b.variance) return MUON_INVALID_ARG;
-    if (!std::isfinite(b.lr_scale)) return MUON_INVALID_ARG;
+    float scale = 0.0f;
+    if (!update_scale(b.fan_out, b.fan_in, hp->scale_mode, hp->extra_scale_factor, &scale)) return MUON_INVALID_ARG;
   }
   if (!any) return MUON_OK;
   const Layout L = plan_layout(batches, nb, 3);
@@ -1282,6 +1472,7 @@ muon_status normuon_update(const muon_batch* batches, int nb, const muon_hparams
     std::memset(&P, 0, sizeof(P));
     long long chunk = 0, slice = 0, row = 0;
     int ns = 0;
+    bool any_rsq = false, any_o = false;   // segments with row sums from the NS call / without
     for (; i < nb && ns < MAX_SEGS; ++i) {
       const muon_batch& b = batches[i];
       if (batch_empty(b)) continue;
@@ -1298,7 +1489,10 @@ muon_status normuon_update(const muon_batch* batches, int nb, const muon_hparams
       S.wc_ld = b.weight_copy.ld;
       S.wc_bs = b.weight_copy.batch_stride;
       S.variance = b.variance;
-      S.lr_scale = b.lr_scale;
+      S.rsq = use_normuon ? b.row_sumsq : nullptr;
+      (void)update_scale(b.fan_out, b.fan_in, hp->scale_mode, hp->extra_scale_factor, &S.lr_scale);
+      any_rsq |= S.rsq != nullptr;
+      any_o |= S.rsq == nullptr;
       S.vec8 = vec8_ok(b, {&b.ns_out, &b.weight, &b.weight_copy});
       S.flat = flat_ok(b, {&b.ns_out, &b.weight, &b.weight_copy});
       ++ns;
@@ -1317,8 +1511,11 @@ muon_status normuon_update(const muon_batch* batches, int nb, const muon_hparams
     P.row_d = row_d;
     P.slice_factor = factor;
     if (use_normuon) {
-      if (!launch_pdl(normuon_rows_kernel, dim3(ew_grid(cdiv(row, EW_THREADS / 32), sms)), dim3(EW_THREADS), 0,
-                      stream, P))
+      if (any_rsq && !launch_pdl(normuon_rows_from_sums_kernel, dim3(ew_grid(cdiv(row, EW_THREADS), sms)),
+                                 dim3(EW_THREADS), 0, stream, P))
+        return MUON_CUDA_ERROR;
+      if (any_o && !launch_pdl(normuon_rows_kernel, dim3(ew_grid(cdiv(row, EW_THREADS / 32), sms)), dim3(EW_THREADS),
+                               0, stream, P))
         return MUON_CUDA_ERROR;
       if (!launch_pdl(normuon_slices_kernel, dim3(ew_grid(slice, sms)), dim3(EW_THREADS), 0, stream, P))
         return MUON_CUDA_ERROR;

@@ -83,6 +83,9 @@ struct __align__(64) SmallParams {
   float a[SMALL_MAX_STEPS], b[SMALL_MAX_STEPS], c[SMALL_MAX_STEPS];
   int* err;
   unsigned long long timeout_ns;
+  float* row_ss;             // optional [slices][2 C][m]: per CTA and column half, each output
+                             // row's sum of squares of its stored bf16 values
+  int restart;               // Gram form: restart period in iterations (0: none)
 };
 
 // Byte offset of the 16-byte chunk holding columns [8 ch, 8 ch + 8) of row r
@@ -241,11 +244,14 @@ __device__ __forceinline__ void epi_square(uint32_t taddr, int row, int half, in
 }
 
 // Epilogue of the product on the resident columns for row `row`, columns
-// [half w/2, half w/2 + w/2): X <- f (acc + a X), in place, bf16.
+// [half w/2, half w/2 + w/2): X <- f (acc + a X), in place, bf16.  With
+// rss non-null, also the sum of squares of the stored values of those
+// columns (zero outside the slice) is written to *rss for rows below m.
 __device__ __forceinline__ void epi_columns(uint32_t taddr, int row, int half, int w, int m8, float a, float f,
-                                            uint8_t* Xs) {
+                                            uint8_t* Xs, float* rss = nullptr, int m = 0) {
   const int hw = w >> 1;
   const int cend = half * hw + hw;
+  float ss = 0.0f;
 #pragma unroll 1
   for (int c0 = half * hw; c0 < cend; c0 += 64) {
     const bool two = c0 + 64 <= cend;               // warp-uniform: 64 or 32 columns
@@ -273,11 +279,19 @@ __device__ __forceinline__ void epi_columns(uint32_t taddr, int row, int half, i
             x += a * xf[e];
             o[e] = x * f;
           }
-          *reinterpret_cast<uint4*>(Xs + sw128_chunk(row, (c0 >> 3) + h)) = pack_bf16x8(o);
+          const uint4 pk = pack_bf16x8(o);
+          *reinterpret_cast<uint4*>(Xs + sw128_chunk(row, (c0 >> 3) + h)) = pk;
+          if (rss != nullptr) {
+            float st[8];
+            unpack_bf16x8(pk, st);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss += st[e] * st[e];
+          }
         }
       }
     }
   }
+  if (rss != nullptr && row < m) *rss = ss;
   fence_proxy_async_smem();
 }
 
@@ -317,6 +331,10 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
   };
   auto unfold = [G](int p) { return (p & 1) ? G - 1 - (p >> 1) : (p >> 1); };
   const uint32_t ncols = w > 256 ? 512u : 256u;     // P and A^2 take 256 columns; a X + B X takes w
+  // This thread's slot for its row's partial sum of squares of the output.
+  float* row_slot = P.row_ss == nullptr ? nullptr
+                                        : P.row_ss + (static_cast<long long>(slice) * (2 * C) + 2 * static_cast<int>(rank) + half) *
+                                                         P.m + row;
 
   if (tid == 0) {
     *abort_flag = 0;
@@ -372,10 +390,12 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
   const uint32_t rv0 = smem_u32(Rv);
   const uint32_t a0 = smem_u32(As);
 
-  const int outer = GRAM ? 1 : P.steps;
-  for (int k = 0; k < outer; ++k) {
-    const float ca = P.a[k], cb = P.b[k], cc = P.c[k];
-    // ---- partial X_r X_r^T -> TMEM columns [0, 128)
+  // ---- A = fA * X X^T over the cluster, into every CTA's As (bf16; fp16 in
+  //      the Gram form), upper triangle mirrored.  Every CTA takes both
+  //      cluster barriers whether or not it is still working, so a CTA that
+  //      gave up never strands its peers.
+  auto exchange = [&](float fA) {
+    // partial X_r X_r^T -> TMEM columns [0, 128)
     if (ok) {
       if (tid == 0) {
         tc_fence_after();
@@ -388,9 +408,9 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
       }
       ok = wait_mma();
     }
-    // ---- push row `row` of the partial, its lower triangle (4-column chunks
-    //      up to the diagonal) within columns [64 half, 64 half + 64), to the
-    //      CTA that owns the row's 8-row block
+    // push row `row` of the partial, its lower triangle (4-column chunks up
+    // to the diagonal) within columns [64 half, 64 half + 64), to the CTA
+    // that owns the row's 8-row block
     if (ok && half * 64 < m8) {
       tc_fence_after();
       uint32_t v[64];
@@ -412,11 +432,10 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
     tc_fence_before();
     cluster_sync();           // every partial row has reached its owner
 
-    // ---- owner: for its row blocks b, A[8b .. 8b+7][0 .. 8b+7] = f * sum over
-    //      the slots in rank order, pushed to every CTA (the diagonal block's
-    //      upper half carries unsent entries; the mirror below replaces it)
+    // owner: for its row blocks b, A[8b .. 8b+7][0 .. 8b+7] = fA * sum over
+    // the slots in rank order, pushed to every CTA (the diagonal block's
+    // upper half carries unsent entries; the mirror below replaces it)
     if (ok) {
-      const float fA = GRAM ? P.kappa * (s * s) : (k == 0) ? s * s : 1.0f;
       int items = 0;
       for (int lb = 0; lb < kb && rank * kb + lb < G; ++lb) items += 8 * (unfold(rank * kb + lb) + 1);
       for (int it = tid; it < items; it += SMALL_THREADS) {
@@ -457,43 +476,24 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
     }
     cluster_sync();           // every CTA holds the lower triangle of A; the receive slots are free again
 
-    // ---- upper triangle of A from the lower one (local)
+    // upper triangle of A from the lower one (local)
     if (ok) mirror_upper(As, G, tid);
     __syncthreads();
-    if (GRAM) break;
+  };
 
-    // ---- A^2 -> TMEM columns [128, 256)
+  // ---- (B, X) <- (Q, X) product on the resident columns: TMEM [0, w) = F X
+  //      with F a 128 x 128 bf16 K-major matrix in shared memory
+  auto left_product = [&](uint32_t f0) {
     if (ok) {
       if (tid == 0) {
         fence_proxy_async_smem();
-        tc_fence_after();
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t d = smem_desc_sw128(a0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
-          tc_mma_f16(tmem + 128, d, d, idesc_sq, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bars[1]);
-      }
-      ok = wait_mma();
-    }
-    // ---- B = c A^2 + b A, in place over A
-    if (ok) {
-      tc_fence_after();
-      epi_square(tmem + tlane + 128u, row, half, m8, P.m, cc, cb, As, false, 0.0f, As, false);
-      fence_proxy_async_smem();
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- B X_r -> TMEM columns [0, w)
-    if (ok) {
-      if (tid == 0) {
         tc_fence_after();
         const uint32_t x0 = smem_u32(Xs);
         for (int nc = 0; nc < w; nc += 256) {
           const int N = min(256, w - nc);
           const uint32_t idesc = mma_idesc_f16(1, 0, 1, 128, static_cast<uint32_t>(N));
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = smem_desc_sw128(a0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+            const uint64_t ad = smem_desc_sw128(f0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = smem_desc_sw128(x0 + (nc >> 6) * SMALL_BLK + kk * 16 * 128, SMALL_BLK, 1024);
             tc_mma_f16(tmem + static_cast<uint32_t>(nc), ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
@@ -502,92 +502,141 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
       }
       ok = wait_mma();
     }
-    // ---- X <- f * (B X + a X), in place
-    if (ok) {
-      tc_fence_after();
-      epi_columns(tmem + tlane, row, half, w, m8, ca, (k == 0) ? s : 1.0f, Xs);
-    }
-    tc_fence_before();
-    __syncthreads();
-  }
+  };
 
-  if (GRAM) {
-    // ---- m x m iteration (fp16, kappa-scaled A), every CTA of the cluster alike
-    uint8_t* Pb = Rv;                               // P (and, on step 0, the first Q)
-    uint8_t* Qb = Rv + SMALL_A_BYTES;               // Q
-    for (int i = tid; i < 2 * SMALL_A_BYTES / 16; i += SMALL_THREADS)
-      reinterpret_cast<uint4*>(Rv)[i] = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
-    __syncthreads();
-    const uint32_t idesc_h = mma_idesc_f16(0, 0, 0, 128, 128);
-    const float kap = P.kappa;
-    for (int k = 0; k < P.steps && ok; ++k) {
-      const bool last = k == P.steps - 1;
-      uint8_t* Pd = (k == 0) ? Qb : Pb;             // Q_1 = P_1
-      // P = a I + (b / kappa) A + (c / kappa^2) A^2; bf16 when it is the final Q
-      if (tid == 0) issue_square(tmem, a0, a0, idesc_h, &bars[1]);
-      ok = wait_mma();
-      if (!ok) break;
-      tc_fence_after();
-      epi_square(tmem + tlane, row, half, m8, P.m, P.c[k] / (kap * kap), P.b[k] / kap, As, true, P.a[k], Pd,
-                 !(k == 0 && last));
-      fence_proxy_async_smem();
+  if (!GRAM) {
+    for (int k = 0; k < P.steps; ++k) {
+      const float ca = P.a[k], cb = P.b[k], cc = P.c[k];
+      exchange((k == 0) ? s * s : 1.0f);
+
+      // ---- A^2 -> TMEM columns [128, 256)
+      if (ok) {
+        if (tid == 0) {
+          fence_proxy_async_smem();
+          tc_fence_after();
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t d = smem_desc_sw128(a0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+            tc_mma_f16(tmem + 128, d, d, idesc_sq, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars[1]);
+        }
+        ok = wait_mma();
+      }
+      // ---- B = c A^2 + b A, in place over A
+      if (ok) {
+        tc_fence_after();
+        epi_square(tmem + tlane + 128u, row, half, m8, P.m, cc, cb, As, false, 0.0f, As, false);
+        fence_proxy_async_smem();
+      }
       tc_fence_before();
       __syncthreads();
-      mirror_upper(Pd, G, tid);
-      __syncthreads();
-      if (k > 0) {
-        // Q <- P Q, bf16 when last
-        if (tid == 0) issue_square(tmem, smem_u32(Pb), smem_u32(Qb), idesc_h, &bars[1]);
-        ok = wait_mma();
-        if (!ok) break;
+
+      // ---- B X_r -> TMEM columns [0, w)
+      left_product(a0);
+      // ---- X <- f * (B X + a X), in place (the last step also leaves row sums of squares)
+      if (ok) {
         tc_fence_after();
-        epi_square(tmem + tlane, row, half, m8, P.m, 1.0f, 0.0f, nullptr, false, 0.0f, Qb, !last);
-        fence_proxy_async_smem();
+        float* rss = (P.row_ss != nullptr && k == P.steps - 1) ? row_slot : nullptr;
+        epi_columns(tmem + tlane, row, half, w, m8, ca, (k == 0) ? s : 1.0f, Xs, rss, P.m);
+      }
+      tc_fence_before();
+      __syncthreads();
+    }
+  } else {
+    // ---- G = kappa s^2 X0 X0^T, then the m x m iteration (fp16, kappa-scaled
+    //      A), every CTA of the cluster alike.  Restarts (every P.restart
+    //      iterations): X <- f Q X on the resident columns, A = kappa X X^T
+    //      over the cluster again, Q = I.
+    exchange(P.kappa * (s * s));
+    uint8_t* Pb = Rv;                               // P (and, at a segment's start, the first Q)
+    uint8_t* Qb = Rv + SMALL_A_BYTES;               // Q
+    auto clear_pq = [&]() {
+      for (int i = tid; i < 2 * SMALL_A_BYTES / 16; i += SMALL_THREADS)
+        reinterpret_cast<uint4*>(Rv)[i] = make_uint4(0u, 0u, 0u, 0u);
+      fence_proxy_async_smem();
+      __syncthreads();
+    };
+    clear_pq();
+    const uint32_t idesc_h = mma_idesc_f16(0, 0, 0, 128, 128);
+    const float kap = P.kappa;
+    const int R = P.restart;
+    auto restart_at = [&](int k) { return R > 0 && k > 0 && k < P.steps && k % R == 0; };
+    float xf = s;                                   // X's factor: s while X is the input
+    int seg_start = 0;
+    for (int k = 0; k < P.steps; ++k) {
+      if (restart_at(k)) {
+        // X <- xf Q X (Q in bf16), in place
+        left_product(smem_u32(Qb));
+        if (ok) {
+          tc_fence_after();
+          epi_columns(tmem + tlane, row, half, w, m8, 0.0f, xf, Xs);
+        }
+        xf = 1.0f;
         tc_fence_before();
         __syncthreads();
-        mirror_upper(Qb, G, tid);
+        cluster_sync();       // no CTA still reads its Q when peers push partial rows over it
+        exchange(kap);
+        clear_pq();
+        seg_start = k;
+      }
+      const bool first = k == seg_start;
+      const bool end = k == P.steps - 1 || restart_at(k + 1);
+      uint8_t* Pd = first ? Qb : Pb;               // Q = P at a segment's start
+      // P = a I + (b / kappa) A + (c / kappa^2) A^2; bf16 when it is the segment's final Q
+      if (ok) {
+        if (tid == 0) issue_square(tmem, a0, a0, idesc_h, &bars[1]);
+        ok = wait_mma();
+      }
+      if (ok) {
+        tc_fence_after();
+        epi_square(tmem + tlane, row, half, m8, P.m, P.c[k] / (kap * kap), P.b[k] / kap, As, true, P.a[k], Pd,
+                   !(first && end));
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (ok) mirror_upper(Pd, G, tid);
+      __syncthreads();
+      if (!first) {
+        // Q <- P Q, bf16 when the segment ends
+        if (ok) {
+          if (tid == 0) issue_square(tmem, smem_u32(Pb), smem_u32(Qb), idesc_h, &bars[1]);
+          ok = wait_mma();
+        }
+        if (ok) {
+          tc_fence_after();
+          epi_square(tmem + tlane, row, half, m8, P.m, 1.0f, 0.0f, nullptr, false, 0.0f, Qb, !end);
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (ok) mirror_upper(Qb, G, tid);
         __syncthreads();
       }
-      if (!last) {
+      if (!end) {
         // R = P A, then A <- P R (fp16, each over A in place once its product is done)
-        for (int h = 0; h < 2 && ok; ++h) {
-          if (tid == 0) issue_square(tmem, smem_u32(Pd), a0, idesc_h, &bars[1]);
-          ok = wait_mma();
-          if (!ok) break;
-          tc_fence_after();
-          epi_square(tmem + tlane, row, half, m8, P.m, 1.0f, 0.0f, nullptr, false, 0.0f, As, true);
-          fence_proxy_async_smem();
+        for (int h = 0; h < 2; ++h) {
+          if (ok) {
+            if (tid == 0) issue_square(tmem, smem_u32(Pd), a0, idesc_h, &bars[1]);
+            ok = wait_mma();
+          }
+          if (ok) {
+            tc_fence_after();
+            epi_square(tmem + tlane, row, half, m8, P.m, 1.0f, 0.0f, nullptr, false, 0.0f, As, true);
+            fence_proxy_async_smem();
+          }
           tc_fence_before();
           __syncthreads();
-          mirror_upper(As, G, tid);
+          if (ok) mirror_upper(As, G, tid);
           __syncthreads();
         }
       }
     }
-    // ---- O = s Q X0 on the resident columns (Q in bf16)
-    if (ok) {
-      if (tid == 0) {
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const uint32_t q0 = smem_u32(Qb);
-        const uint32_t x0 = smem_u32(Xs);
-        for (int nc = 0; nc < w; nc += 256) {
-          const int N = min(256, w - nc);
-          const uint32_t idesc = mma_idesc_f16(1, 0, 1, 128, static_cast<uint32_t>(N));
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(x0 + (nc >> 6) * SMALL_BLK + kk * 16 * 128, SMALL_BLK, 1024);
-            tc_mma_f16(tmem + static_cast<uint32_t>(nc), ad, bd, idesc, kk > 0 ? 1u : 0u);
-          }
-        }
-        tc_commit(&bars[1]);
-      }
-      ok = wait_mma();
-    }
+    // ---- O = xf Q X on the resident columns (Q in bf16)
+    left_product(smem_u32(Qb));
     if (ok) {
       tc_fence_after();
-      epi_columns(tmem + tlane, row, half, w, m8, 0.0f, s, Xs);
+      epi_columns(tmem + tlane, row, half, w, m8, 0.0f, xf, Xs, P.row_ss != nullptr ? row_slot : nullptr, P.m);
     }
     tc_fence_before();
     __syncthreads();

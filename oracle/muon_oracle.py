@@ -48,7 +48,8 @@ QUINTIC_ABC = (3.4445, -4.7750, 2.0315)
 __all__ = [
     "QUINTIC_ABC", "bf16_round", "fp32_round", "momentum_nesterov", "frobenius_normalize",
     "newton_schulz", "gram_newton_schulz", "ns_batched", "per_head_ns", "flatten_megabatch",
-    "normuon_normalize", "spectral_scale", "weight_update", "muon_step_slices", "ns_flops",
+    "normuon_normalize", "spectral_scale", "rms_norm_scale", "update_scale", "weight_update", "muon_step_slices",
+    "ns_flops",
 ]
 
 
@@ -166,7 +167,7 @@ def newton_schulz(U: np.ndarray, steps: int = 5, eps: float = 1e-7,
 
 
 def gram_newton_schulz(U: np.ndarray, steps: int = 5, eps: float = 1e-7,
-                       abc: Sequence[float] = QUINTIC_ABC) -> np.ndarray:
+                       abc: Sequence[float] = QUINTIC_ABC, restart: int = 0) -> np.ndarray:
     """Gram Newton-Schulz of one slice: the same map, iterated on the small side.
 
     [ds-8437] "Why it happens" / "Measurement": the Gram kernel also
@@ -178,37 +179,51 @@ def gram_newton_schulz(U: np.ndarray, steps: int = 5, eps: float = 1e-7,
     they commute, ``X_k = Q_k X0`` and ``X_k X_k^T = Q_k G Q_k``, so this equals
     the standard iteration in exact arithmetic (also with a per-step
     schedule of (a, b, c)).
+
+    ``restart = R > 0``: before steps R, 2R, ... the iterate ``X = Q X`` is
+    formed and the iteration starts again from it (``A = X X^T``, ``Q = I``).
+    By the same identities this changes nothing in exact arithmetic; it is the
+    reading the library takes to keep low-precision iterates of ``A`` from
+    drifting (rank-deficient slices), and it is kept here so that the oracle
+    computes the same sequence of products.
     """
-    X0, transposed = _orient(U)
-    X0 = frobenius_normalize(X0, eps)
-    m = X0.shape[0]
+    X, transposed = _orient(U)
+    X = frobenius_normalize(X, eps)
+    m = X.shape[0]
     I = np.eye(m)
-    A = X0 @ X0.T
+    A = X @ X.T
     Q = I.copy()
-    for a, b, c in _step_coefs(abc, steps):
+    for k, (a, b, c) in enumerate(_step_coefs(abc, steps)):
+        if restart and k > 0 and k % restart == 0:
+            X = Q @ X
+            A = X @ X.T
+            Q = I.copy()
         P = a * I + b * A + c * (A @ A)
         Q = P @ Q
         A = P @ A @ P
-    O = Q @ X0
+    O = Q @ X
     return O.T if transposed else O
 
 
 def ns_batched(U: np.ndarray, variant: str = "standard", steps: int = 5, eps: float = 1e-7,
-               abc: Sequence[float] = QUINTIC_ABC) -> np.ndarray:
+               abc: Sequence[float] = QUINTIC_ABC, restart: int = 0) -> np.ndarray:
     """Newton-Schulz of every slice of a [N, rows, cols] megabatch, one slice at a time.
 
     [dion-121] "Problem and fix": a megabatch is orthogonalized per slice
-    [N, out, prod(rest)], never across slices.
+    [N, out, prod(rest)], never across slices.  ``restart`` applies to the
+    Gram variant only.
     """
     U = np.asarray(U, dtype=np.float64)
     if U.ndim != 3:
         raise ValueError("megabatch must be [N, rows, cols]")
-    fn = newton_schulz if variant == "standard" else gram_newton_schulz
     if variant not in ("standard", "gram"):
         raise ValueError(f"unknown variant {variant!r}")
     out = np.empty_like(U)
     for i in range(U.shape[0]):
-        out[i] = fn(U[i], steps=steps, eps=eps, abc=abc)
+        if variant == "standard":
+            out[i] = newton_schulz(U[i], steps=steps, eps=eps, abc=abc)
+        else:
+            out[i] = gram_newton_schulz(U[i], steps=steps, eps=eps, abc=abc, restart=restart)
     return out
 
 
@@ -281,6 +296,30 @@ def spectral_scale(fan_out: int, fan_in: int, extra: float = 1.0) -> float:
     return math.sqrt(max(1.0, fan_out / fan_in)) * extra
 
 
+def rms_norm_scale(fan_out: int, fan_in: int, extra: float = 1.0) -> float:
+    """Shape factor of the ``rms_norm`` mode: ``0.2 * sqrt(max(fan_out, fan_in)) * extra``.
+
+    The pages name the mode ([dion-121] review: ``adjust_lr_rms_norm``;
+    [mcore-lsm] ``scale_mode``) but print no formula.  Reading: the RMS
+    matching of Liu et al., "Muon is Scalable for LLM Training" (2025): an
+    orthogonalized m x n update (m <= n, unit singular values) has element
+    RMS ``1/sqrt(n)``, so this factor gives it RMS 0.2 -- a typical AdamW
+    update's -- whatever the shape.
+    """
+    return 0.2 * math.sqrt(max(fan_out, fan_in)) * extra
+
+
+def update_scale(fan_out: int, fan_in: int, mode: str = "spectral", extra: float = 1.0) -> float:
+    """The update's shape factor of one parameter in the given ``scale_mode``."""
+    if fan_out < 1 or fan_in < 1:
+        raise ValueError("fan_out and fan_in must be positive")
+    if mode == "spectral":
+        return spectral_scale(fan_out, fan_in, extra)
+    if mode == "rms_norm":
+        return rms_norm_scale(fan_out, fan_in, extra)
+    raise ValueError(f"unknown scale mode {mode!r}")
+
+
 def weight_update(W: np.ndarray, Oh: np.ndarray, lr: float, weight_decay: float,
                   scale: float, store: str = "f64") -> np.ndarray:
     """Decoupled weight decay then ``W -= lr * scale * Oh``, rounded once on store.
@@ -299,7 +338,7 @@ def weight_update(W: np.ndarray, Oh: np.ndarray, lr: float, weight_decay: float,
 def muon_step_slices(G: np.ndarray, M: np.ndarray, W: np.ndarray, v: Optional[np.ndarray], *,
                      mu: float = 0.95, nesterov: bool = True, ns_eps: float = 1e-7,
                      ns_steps: int = 5, abc: Sequence[float] = QUINTIC_ABC,
-                     variant: str = "standard", normuon: bool = False, beta2: float = 0.95,
+                     variant: str = "standard", restart: int = 0, normuon: bool = False, beta2: float = 0.95,
                      nor_eps: float = 1e-8, lr: float = 0.02, weight_decay: float = 0.0,
                      lr_scale: float = 1.0, mom_store: str = "f64", w_store: str = "f64",
                      O_override: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
@@ -314,7 +353,7 @@ def muon_step_slices(G: np.ndarray, M: np.ndarray, W: np.ndarray, v: Optional[np
     G = np.asarray(G, np.float64)
     M_new, U = momentum_nesterov(G, M, mu, nesterov, mom_store)
     if O_override is None:
-        O = ns_batched(U, variant, ns_steps, ns_eps, abc)
+        O = ns_batched(U, variant, ns_steps, ns_eps, abc, restart)
     else:
         O = np.asarray(O_override, np.float64)
     Oh = np.empty_like(O)
@@ -330,27 +369,34 @@ def muon_step_slices(G: np.ndarray, M: np.ndarray, W: np.ndarray, v: Optional[np
 
 
 def ns_flops(m: int, n: int, variant: str = "standard", steps: int = 5,
-             triangle: bool = True) -> float:
+             triangle: bool = True, restart: int = 0) -> float:
     """Floating-point operations of one slice's orthogonalization (m <= n).
 
     Standard, full products: per step ``2m^2n`` (X X^T) + ``2m^3`` (A^2) +
     ``2m^2n`` (B X).  With one triangle of the two symmetric products
     ([mcore-lsm] ``use_syrk``): ``m^2n + m^3 + 2m^2n``.  Gram, triangle
-    products: ``m^2n`` for ``G`` and ``2m^2n`` for the final ``Q X0``, plus per
-    step a triangle ``m^3`` for each of ``A^2``, ``P Q`` (none on the first
-    step, where Q = P), and the two factors of ``P A P`` (none on the last
-    step, whose A is never used).
+    products: ``m^2n`` for ``G`` and ``2m^2n`` for the final ``Q X``, plus per
+    step a triangle ``m^3`` for each of ``A^2``, ``P Q`` (none on a segment's
+    first step, where Q = P), and the two factors of ``P A P`` (none on a
+    segment's last step, whose A is never used); a restart adds ``Q X``
+    (``2m^2n``) and ``X X^T`` (``m^2n``, one triangle).
     """
     m, n = min(m, n), max(m, n)
     if variant == "standard":
         per = (m * m * n + m ** 3 + 2 * m * m * n) if triangle else (4 * m * m * n + 2 * m ** 3)
         return float(steps * per)
     if variant == "gram":
-        prods = 0
+        def restart_at(k):
+            return bool(restart) and 0 < k < steps and k % restart == 0
+        prods, restarts, seg = 0, 0, 0
         for k in range(steps):
-            prods += 1                                  # A^2
-            prods += 0 if k == 0 else 1                 # P Q
-            prods += 0 if k == steps - 1 else 2         # P (P A)
+            if restart_at(k):
+                restarts += 1
+                seg = k
+            prods += 1                                                     # A^2
+            prods += 0 if k == seg else 1                                  # P Q
+            prods += 0 if (k == steps - 1 or restart_at(k + 1)) else 2     # P (P A)
         per_prod = m ** 3 if triangle else 2 * m ** 3
-        return float(m * m * n * (1 if triangle else 2) + 2 * m * m * n + prods * per_prod)
+        gram = m * m * n * (1 if triangle else 2)
+        return float(gram + 2 * m * m * n + restarts * (gram + 2 * m * m * n) + prods * per_prod)
     raise ValueError(variant)

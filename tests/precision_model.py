@@ -38,3 +38,53 @@ def ns_standard_bf16(U, steps=5, eps=1e-7, abc=(3.4445, -4.7750, 2.0315)):
         B = _bf16(_f32(c * _f32(A @ A) + b * A))
         Xb = _bf16(_f32((s if k == 0 else 1.0) * (_f32(B @ Xb) + a * Xb)))
     return Xb.T if tr else Xb
+
+
+def _f16(x):
+    return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float16).astype(np.float64)
+
+
+def ns_gram_f16(U, steps=5, eps=1e-7, abc=(3.4445, -4.7750, 2.0315), restart=3, kappa=16384.0):
+    """Gram iteration with the library's storage precisions.
+
+    The m x m iterates are stored in fp16 with A kept as kappa*A (kappa = 2^14
+    keeps A's O(1/m) entries out of fp16's subnormal range); a Q that goes
+    into a product with the m x n side is stored in bf16, as are X and O.
+    Restarts (every `restart` steps) form X = f Q X in bf16 and start again
+    from A = kappa X X^T, Q = I.
+    """
+    a, b, c = abc
+    X = np.asarray(U, dtype=np.float64)
+    tr = X.shape[0] > X.shape[1]
+    if tr:
+        X = X.T
+    X = _bf16(X)
+    m = X.shape[0]
+    s = 1.0 / (np.sqrt(np.sum(X * X)) + eps)
+    I = np.eye(m)
+    Ah = _f16(_f32(X @ X.T) * (kappa * s * s))
+    f = s                                  # X's factor: s while X is the unnormalized input
+    Q = None
+
+    def restart_at(k):
+        return restart > 0 and 0 < k < steps and k % restart == 0
+
+    for k in range(steps):
+        if restart_at(k):
+            X = _bf16(f * _f32(Q @ X))
+            f = 1.0
+            Ah = _f16(_f32(X @ X.T) * kappa)
+            Q = None
+        end = k == steps - 1 or restart_at(k + 1)
+        Pm = _f32(c / (kappa * kappa) * _f32(Ah @ Ah) + b / kappa * Ah) + a * I
+        if Q is None:
+            Q = _bf16(Pm) if end else _f16(Pm)
+            P = Q
+        else:
+            P = _f16(Pm)
+            Q = (_bf16 if end else _f16)(P @ Q)
+        if not end:
+            R = _f16(P @ Ah)
+            Ah = _f16(P @ R)
+    O = _bf16(f * _f32(Q @ X))
+    return O.T if tr else O

@@ -77,7 +77,7 @@ def _fake_batch(mn, n, r, c, **kw):
         v.dtype = kw.get(f + "_dt", _capi.MUON_BF16)
     b.sumsq = 0x7F0000100000
     b.variance = 0x7F0000200000
-    b.lr_scale = 1.0
+    b.fan_out, b.fan_in = r, c
     return b
 
 
@@ -232,17 +232,114 @@ def test_workspace_holds_the_transposed_copy_of_tall_small_slices(mn):
     for which in (1, 2):
         tall = size(_fake_batch(mn, n, r, c), which)
         # the same buffers without the copy: m x m ones of the same m, plus
-        # (standard) the X-sized buffer of a rows x cols slice
+        # the X-sized buffer of a rows x cols slice (standard: the iterate;
+        # Gram: the iterate a restart forms)
         m = c
         mm = n * ((m + 63) // 64 * 64) * m * 2
         base = 256 + 2 * 256                   # error word, norm partials and sums (rounded up)
+        xbuf = n * r * ((c + 63) // 64 * 64) * 2
         if which == 1:
-            base_bufs = 2 * mm + n * r * ((c + 63) // 64 * 64) * 2
+            base_bufs = 2 * mm + xbuf
         else:
-            base_bufs = 5 * mm
+            base_bufs = 5 * mm + xbuf
         assert tall >= base_bufs + copy
         assert tall - copy < base_bufs + base + 5 * 256 + 8 * n * ((r * c + 8191) // 8192) + 64
     # wide twin and a tall slice with a long side past 4096: no copy
     assert size(_fake_batch(mn, n, c, r), 1) < size(_fake_batch(mn, n, r, c), 1)
     t_big = size(_fake_batch(mn, 1, 5000, 96), 2)
-    assert t_big < 5 * ((96 + 63) // 64 * 64) * 96 * 2 + 256 * 8 + 4 * ((5000 * 96 + 8191) // 8192) + 4096
+    assert t_big < (5 * ((96 + 63) // 64 * 64) * 96 * 2 + 5000 * 128 * 2 + 256 * 8 + 4 * ((5000 * 96 + 8191) // 8192)
+                    + 4096)
+
+
+# ----------------------------------------------------------------- update scale (host code)
+
+@pytest.mark.parametrize("shape,mode,extra", [((4096, 4096), "spectral", 1.0), ((1024, 4096), "spectral", 1.0),
+                                              ((8192, 4096), "spectral", 1.0), ((14336, 4096), "spectral", 1.0),
+                                              ((4096, 14336), "spectral", 2.5), ((4096, 4096), "rms_norm", 1.0),
+                                              ((14336, 4096), "rms_norm", 1.0), ((64, 576), "rms_norm", 0.5),
+                                              ((1, 1), "rms_norm", 1.0), ((7168, 2048), "spectral", 0.3)])
+def test_update_scale_through_the_c_abi_matches_the_oracle(mn, shape, mode, extra):
+    import numpy as np
+    import oracle
+    got = mn.update_scale(*shape, mode=mode, extra=extra)
+    # the ABI takes extra as a float32; the scale is computed in double and rounded once to float32
+    want = oracle.update_scale(*shape, mode=mode, extra=float(np.float32(extra)))
+    assert got == float(np.float32(want))
+
+
+def test_update_scale_closed_values(mn):
+    import math
+    assert mn.update_scale(4096, 4096) == 1.0
+    assert mn.update_scale(1024, 4096) == 1.0
+    assert abs(mn.update_scale(8192, 4096) - math.sqrt(2)) < 1e-7
+    assert abs(mn.update_scale(14336, 4096) - math.sqrt(3.5)) < 1e-7
+    assert abs(mn.update_scale(4096, 4096, "rms_norm") - 12.8) < 1e-5
+    assert abs(mn.update_scale(1024, 4096, "rms_norm", 0.5) - 6.4) < 1e-5
+
+
+def test_update_scale_rejects_bad_arguments(mn):
+    from newton_schulz_ns_b200 import _capi
+    out = ctypes.c_float(0.0)
+    for args in [(0, 4, 0, 1.0), (4, 0, 0, 1.0), (-3, 4, 0, 1.0), (4, 4, 2, 1.0), (4, 4, -1, 1.0),
+                 (4, 4, 0, float("nan")), (4, 4, 1, float("inf"))]:
+        assert _capi.lib.muon_update_scale(*args, ctypes.byref(out)) == 1, args
+    assert _capi.lib.muon_update_scale(4, 4, 0, 1.0, None) == 1
+
+
+@no_device
+def test_update_rejects_missing_fans_and_unknown_modes(mn):
+    good = _fake_batch(mn, 2, 64, 576)
+    nofan = _fake_batch(mn, 2, 64, 576)
+    nofan.fan_out = 0
+    assert _call(mn, "normuon_update", [nofan], 0x7F0000300000, 1 << 30) == 1
+    neg = _fake_batch(mn, 2, 64, 576)
+    neg.fan_in = -5
+    assert _call(mn, "normuon_update", [neg], 0x7F0000300000, 1 << 30) == 1
+    hp = mn.Hparams()
+    h, keep = hp.to_c()
+    from newton_schulz_ns_b200 import _capi
+    arr = (_capi.MuonBatch * 1)(good)
+    h.scale_mode = 5
+    assert _capi.lib.normuon_update(arr, 1, ctypes.byref(h), 1, 0x7F0000300000, 1 << 30, None) == 1
+    h.scale_mode = 0
+    h.extra_scale_factor = float("nan")
+    assert _capi.lib.normuon_update(arr, 1, ctypes.byref(h), 1, 0x7F0000300000, 1 << 30, None) == 1
+    # every call validates the hyperparameters, the restart period included
+    for fn in ("muon_momentum_norm", "muon_ns_batched", "muon_gram_ns_batched"):
+        assert _call(mn, fn, [good], 0x7F0000300000, 1 << 30, gram_restart=-1) == 1
+        assert _call(mn, fn, [good], 0x7F0000300000, 1 << 30, gram_restart=17) == 1
+        assert _call(mn, fn, [good], 0x7F0000300000, 1 << 30, scale_mode="spectral", extra_scale_factor=float("inf")) == 1
+
+
+def test_testing_options_round_trip_and_range_checks(mn):
+    from newton_schulz_ns_b200 import _capi
+    prev = _capi.MuonTestingOptions()
+    assert _capi.lib.muon_testing_set_options(None, ctypes.byref(prev)) == 0
+    assert (prev.fused_small, prev.max_waves, prev.max_problems, prev.pdl) == (1, 32, 1, 1)
+    with mn.testing_options(fused_small=0, max_waves=4, pdl=0):
+        cur = _capi.MuonTestingOptions()
+        _capi.lib.muon_testing_set_options(None, ctypes.byref(cur))
+        assert (cur.fused_small, cur.max_waves, cur.max_problems, cur.pdl) == (0, 4, 1, 0)
+    cur = _capi.MuonTestingOptions()
+    _capi.lib.muon_testing_set_options(None, ctypes.byref(cur))
+    assert (cur.fused_small, cur.max_waves, cur.max_problems, cur.pdl) == (1, 32, 1, 1)
+    for bad in [(2, 32, 1, 1), (1, -1, 1, 1), (1, 32, 0, 1), (1, 32, 9, 1), (1, 32, 1, 3)]:
+        o = _capi.MuonTestingOptions(*bad)
+        assert _capi.lib.muon_testing_set_options(ctypes.byref(o), None) == 1
+    _capi.lib.muon_testing_set_options(None, ctypes.byref(cur))
+    assert (cur.fused_small, cur.max_waves, cur.max_problems, cur.pdl) == (1, 32, 1, 1)
+
+
+def test_row_sum_partials_take_workspace_only_when_requested(mn):
+    from newton_schulz_ns_b200 import _capi
+    n, r, c = 3, 300, 520
+    plain = _fake_batch(mn, n, r, c)
+    asked = _fake_batch(mn, n, r, c)
+    asked.row_sumsq = 0x7F0000400000
+    for which in (1, 2):
+        a = _capi.lib.muon_workspace_size((_capi.MuonBatch * 1)(plain), 1, which)
+        b = _capi.lib.muon_workspace_size((_capi.MuonBatch * 1)(asked), 1, which)
+        # one float per output row and per 256-column tile (at least 16 per row: the fused path's
+        # CTA halves), rounded up to the 256-byte alignment
+        per_row = max((c + 255) // 256, 16)
+        assert b - a == (4 * n * per_row * r + 255) // 256 * 256

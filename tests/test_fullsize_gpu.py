@@ -14,6 +14,7 @@ import pytest
 import torch
 
 import bench
+import float32_model
 import oracle
 import workloads
 
@@ -33,23 +34,28 @@ def rel(a, b):
     return float(np.linalg.norm(a - b) / np.linalg.norm(b))
 
 
-def _bf16_within_one_ulp(got, want, terms=None):
-    """At most one bf16 ulp from the oracle, >= 99.9% identical.
+def _bf16_within_one_ulp(got, want, slack=0.0):
+    """At most one bf16 ulp (+ slack) from the oracle, >= 99.99% identical.
 
-    ``terms``: magnitude of the quantities the device adds in float32 to form
-    the value; where they nearly cancel, their float32 rounding (a few 2^-24
-    of each) may exceed the bf16 ulp of the small result, and that much more
-    is allowed.
+    ``slack``: the float32 update's rounding error beyond its final rounding
+    (see update_slack), which can exceed a bf16 ulp where W_new is much
+    smaller than W.  The 99.99% bar is what float32 arithmetic of the stated
+    formulas achieves on these distributions (a float32 model of the kernels,
+    tests/float32_model.py, counts a few 1e-5 of flipped roundings).
     """
-    ulp = np.abs(oracle.bf16_round(np.abs(want) * (1 + 2.0 ** -7)) - oracle.bf16_round(np.abs(want)))
-    ulp = np.maximum(ulp, 2.0 ** -133)
-    slack = 0.0 if terms is None else 4 * 2.0 ** -24 * terms
+    ulp = float32_model.bf16_ulp(want)
     bad = np.abs(got - want) > ulp * 1.0001 + slack
     if np.any(bad):
         i = np.flatnonzero(bad)[:5]
         raise AssertionError(f"{int(bad.sum())} elements beyond one ulp: got {got.flat[i]}, want {want.flat[i]}, "
-                             f"ulp {ulp.flat[i]}, terms {None if terms is None else terms.flat[i]}")
-    assert np.mean(got == want) >= 0.999
+                             f"ulp {ulp.flat[i]}")
+    assert np.mean(got == want) >= 0.9999, float(np.mean(got == want))
+
+
+def update_slack(W0, W_new, dW):
+    """float32 rounding of W*keep and of the fused multiply-add (2^-24 of |W| and |W_new|), plus the
+    coefficient's relative error, which the fp32-stage parity bar holds below 1e-5 of |dW|."""
+    return 2.0 ** -24 * (np.abs(W0) + np.abs(W_new)) + 1e-5 * np.abs(dW)
 
 
 def _run_full_step(key, variant, samples):
@@ -77,7 +83,7 @@ def _run_full_step(key, variant, samples):
                                       mu=h32(wl.momentum), nesterov=wl.nesterov, variant=variant,
                                       normuon=wl.normuon, beta2=h32(wl.beta2), nor_eps=h32(wl.nor_eps),
                                       lr=h32(wl.lr), weight_decay=h32(wl.weight_decay),
-                                      lr_scale=h32(b.lr_scale), mom_store=mstore, w_store="f64")
+                                      lr_scale=h32(oracle.update_scale(b.fan_out, b.fan_in)), mom_store=mstore, w_store="f64")
         err = rel(O[0], ref["O"][0])
         assert err < 3e-2, (g.name, si, err)
         _bf16_within_one_ulp(f64(b.momentum[si]), ref["M"][0])
@@ -86,20 +92,19 @@ def _run_full_step(key, variant, samples):
                                        st["v"][None] if st["v"] is not None else None,
                                        mu=h32(wl.momentum), nesterov=wl.nesterov, normuon=wl.normuon,
                                        beta2=h32(wl.beta2), nor_eps=h32(wl.nor_eps), lr=h32(wl.lr),
-                                       weight_decay=h32(wl.weight_decay), lr_scale=h32(b.lr_scale),
+                                       weight_decay=h32(wl.weight_decay), lr_scale=h32(oracle.update_scale(b.fan_out, b.fan_in)),
                                        mom_store=mstore, w_store="f64", O_override=O)
         if wl.normuon:
             assert rel(f64(b.variance.view(b.n, b.rows)[si]), ref2["v"][0]) < 1e-5
+        slack = update_slack(st["W"], ref2["W"][0], ref2["W"][0] - st["W"])
         if wl.weight_dtype == torch.float32:
             dW = f64(b.weight[si]) - st["W"]
             assert rel(dW, ref2["W"][0] - st["W"]) < 1e-5
-            terms = np.abs(st["W"]) + np.abs(ref2["W"][0] - st["W"])
             if b.weight_copy is not None:
                 _bf16_within_one_ulp(f64(b.weight_copy[si]), oracle.bf16_round(oracle.fp32_round(ref2["W"][0])),
-                                     terms)
+                                     slack)
         else:
-            terms = np.abs(st["W"]) + np.abs(ref2["W"][0] - st["W"])
-            _bf16_within_one_ulp(f64(b.weight[si]), oracle.bf16_round(ref2["W"][0]), terms)
+            _bf16_within_one_ulp(f64(b.weight[si]), oracle.bf16_round(ref2["W"][0]), slack)
     del groups, ws
     torch.cuda.empty_cache()
 

@@ -282,6 +282,40 @@ def test_spectral_scale_values(shape, scale):
     assert orc.spectral_scale(*shape) == pytest.approx(scale, rel=1e-15)
 
 
+def _orthogonal(r, c, seed):
+    """An exactly orthogonal r x c matrix: orthonormal rows (r <= c) or columns (r > c)."""
+    rng = np.random.default_rng(seed)
+    q, _ = np.linalg.qr(rng.standard_normal((max(r, c), min(r, c))))
+    return q.T if r <= c else q
+
+
+@pytest.mark.parametrize("shape", [(64, 576), (576, 64), (256, 256), (128, 4096), (1024, 512), (1, 7)])
+@pytest.mark.parametrize("extra", [1.0, 0.5])
+def test_rms_norm_scale_gives_orthogonal_updates_rms_two_tenths(shape, extra):
+    # The rms_norm mode's defining property: an orthogonalized update scaled
+    # by it has element RMS 0.2 (times extra) whatever the shape.
+    O = _orthogonal(*shape, seed=shape[0] + shape[1])
+    U = orc.rms_norm_scale(*shape, extra) * O
+    assert math.sqrt(float(np.mean(U * U))) == pytest.approx(0.2 * extra, rel=1e-12)
+    assert orc.update_scale(*shape, mode="rms_norm", extra=extra) == orc.rms_norm_scale(*shape, extra)
+
+
+@pytest.mark.parametrize("shape", [(576, 64), (256, 256), (1024, 512), (14336, 4096), (7, 1)])
+def test_spectral_scale_gives_unit_rms_operator_norm_when_fan_out_ge_fan_in(shape):
+    # ||s O||_{RMS->RMS} = sqrt(fan_in / fan_out) * ||s O||_2 = 1 for an orthogonal O.
+    r, c = shape
+    O = _orthogonal(r, c, seed=r + 2 * c)
+    s = orc.update_scale(r, c, mode="spectral")
+    assert math.sqrt(c / r) * s * np.linalg.norm(O, 2) == pytest.approx(1.0, rel=1e-12)
+
+
+def test_update_scale_rejects_unknown_modes_and_empty_shapes():
+    with pytest.raises(ValueError):
+        orc.update_scale(4, 4, mode="shape")
+    with pytest.raises(ValueError):
+        orc.update_scale(0, 4)
+
+
 def test_weight_update_closed_forms():
     rng = np.random.default_rng(16)
     Oh = rng.standard_normal((4, 5))
@@ -316,6 +350,22 @@ def test_ns_flops_closed_forms():
     tri = orc.ns_flops(m, m, "standard", triangle=True)
     assert full == 30 * m ** 3 and tri == 20 * m ** 3          # one triangle: a third off, square case
     assert orc.ns_flops(256, 1024, "gram") == 256 ** 2 * 1024 * 3 + 17 * 256 ** 3
+    # one restart (before step 3 of 5): Q X and X X^T again; no P Q at step 3, no P A P at step 2
+    assert orc.ns_flops(256, 1024, "gram", restart=3) == 256 ** 2 * 1024 * 6 + 14 * 256 ** 3
+
+
+@pytest.mark.parametrize("shape", [(64, 576), (300, 200), (128, 128), (5, 3)])
+@pytest.mark.parametrize("restart,steps", [(1, 5), (2, 5), (3, 5), (3, 16), (4, 16)])
+def test_gram_with_restarts_equals_standard(shape, restart, steps):
+    # A restart re-forms X = Q X and A = X X^T and resets Q: in exact
+    # arithmetic nothing changes, with any per-step schedule.
+    rng = np.random.default_rng(shape[0] * 7 + restart)
+    U = rng.standard_normal(shape)
+    sched = [(3.4445 - 0.03 * k, -4.7750 + 0.05 * k, 2.0315 - 0.02 * k) for k in range(steps)]
+    ref = orc.newton_schulz(U, steps=steps, abc=sched)
+    got = orc.gram_newton_schulz(U, steps=steps, abc=sched, restart=restart)
+    assert np.max(np.abs(got - ref)) <= 1e-10 * max(1.0, np.max(np.abs(ref)))
+    assert np.array_equal(orc.ns_batched(U[None], "gram", steps, abc=sched, restart=restart)[0], got)
 
 
 # ----------------------------------------------------------------- Polar Express schedule (LP oracle)

@@ -18,6 +18,13 @@ import torch
 DEV = "cuda"
 
 
+def _cuda_device_present() -> bool:
+    try:
+        return torch.cuda.is_available()
+    except Exception:  # noqa: BLE001
+        return False
+
+
 @pytest.fixture(scope="module")
 def mn():
     import newton_schulz_ns_b200 as m
@@ -66,6 +73,30 @@ def test_noalloc_matches_workspace_call_twice_in_a_row(mn):
             assert bool(torch.all(torch.isfinite(b.sumsq)))
 
 
+@pytest.mark.gpu
+def test_noalloc_many_batches_match_workspace_call(mn):
+    # More batches than one elementwise launch takes (16): the call is split
+    # into several launches, each with its own stretch of the shared scratch.
+    shapes = [(1 + k % 3, 16 + 8 * k, 40 + 24 * (k % 5), torch.bfloat16, torch.bfloat16 if k % 2 else torch.float32)
+              for k in range(37)]
+    base = _state(shapes, 2)
+    ref = _batches(mn, [(G.clone(), M.clone()) for G, M in base])
+    new = _batches(mn, [(G.clone(), M.clone()) for G, M in base])
+    hp = mn.Hparams(mu=0.9, nesterov=True)
+    ws = mn.allocate_workspace(ref, 0)
+    for call in range(2):
+        mn.muon_momentum_norm(ref, hp, ws)
+        mn.muon_momentum_norm_noalloc(new, hp)
+        torch.cuda.synchronize()
+        for a, b in zip(ref, new):
+            assert torch.equal(a.momentum, b.momentum), call
+            assert torch.equal(a.ns_in, b.ns_in), call
+            assert torch.equal(a.sumsq, b.sumsq), call
+
+
+# The call below passes fake device addresses that host-side validation must
+# reject; like the other fake-address checks it never runs where a GPU is.
+@pytest.mark.skipif(_cuda_device_present(), reason="passes fake device addresses: host-only check")
 def test_noalloc_rejects_calls_beyond_its_scratch(mn):
     from newton_schulz_ns_b200 import _capi
     b = _capi.MuonBatch()
