@@ -412,7 +412,14 @@ struct ProblemSpec {
   int64_t out_ld, out_bs;
   int out_f16;
   float* row_ss;
+  int mirror;                // tri: write the upper triangle too
+  int a_sym, b_sym;          // symmetric operands stored as their lower 256-blocks
 };
+
+// m x m matrices with m >= 256 are computed by the 2-CTA kernel and stored
+// as their lower 256 x 256 blocks only; every consumer reads them as
+// symmetric operands.  Smaller ones are stored whole (mirrored).
+inline bool sym_compact(int64_t m) { return m >= 256; }
 
 // Builds every launch of `specs` (at most MAX_PROBLEMS problems each) and
 // then enqueues them, so that an encoding error enqueues nothing.
@@ -446,6 +453,9 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
     if (cta_pair == 1 || pair_units <= 0) return 1;
     return s.M >= 256 ? 2 : 1;
   };
+  // Symmetric-operand reads need the pair kernel's stage geometry.
+  for (const ProblemSpec& s : specs)
+    if ((s.a_sym || s.b_sym) && s.slices > 0 && s.M > 0 && s.N > 0 && pick_cg(s) != 2) return MUON_BAD_SHAPE;
   auto tiles_per_slice = [](const ProblemSpec& s, int cg) {
     const int tm = BM * cg;
     const int mt = static_cast<int>(cdiv(s.M, tm)), nt = static_cast<int>(cdiv(s.N, BN));
@@ -532,6 +542,9 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
       g.nt = static_cast<int>(cdiv(s.N, BN));
       g.kt = static_cast<int>(cdiv(s.K, cg == 2 ? GemmCfg<2>::KB : GemmCfg<1>::KB));
       g.tri = s.tri;
+      g.mirror = s.mirror;
+      g.a_sym = s.a_sym;
+      g.b_sym = s.b_sym;
       if (s.tri) {
         int cnt = 0;
         for (int j = 0; j < g.nt; ++j) cnt += std::max(0, g.mt - step * j);
@@ -884,11 +897,12 @@ ProblemSpec syrk_spec(const muon_batch& b, const Mat& x, void* out, int64_t ldm,
   s.out_ld = ldm;
   s.out_bs = bsm;
   s.out_f16 = out_f16;
+  s.mirror = sym_compact(m) ? 0 : 1;
   return s;
 }
 
-// Symmetric m x m product out = f * (alpha * P S + beta * D) + gamma I (lower + mirror);
-// both factors are symmetric, so both are read K-major.
+// Symmetric m x m product out = f * (alpha * P S + beta * D) + gamma I (lower triangle,
+// mirrored when m < 256); both factors are symmetric and read as such.
 ProblemSpec sym_spec(int m, int slices, const Mat& p, const Mat& q, void* out, int64_t ldm, int64_t bsm, int out_f16,
                      float alpha, float beta, const void* add, int add_f16, float gamma) {
   ProblemSpec s{};
@@ -914,6 +928,8 @@ ProblemSpec sym_spec(int m, int slices, const Mat& p, const Mat& q, void* out, i
   s.out_ld = ldm;
   s.out_bs = bsm;
   s.out_f16 = out_f16;
+  s.mirror = sym_compact(m) ? 0 : 1;
+  s.a_sym = s.b_sym = sym_compact(m) ? 1 : 0;
   return s;
 }
 
@@ -934,6 +950,7 @@ ProblemSpec apply_spec(const muon_batch& b, const Mat& f, const Mat& x, void* ou
     s.K = m;
     s.a = f;
     s.a_mn = 0;
+    s.a_sym = sym_compact(m) ? 1 : 0;
     s.b = x;
     s.b_mn = 1;
   } else {
@@ -944,6 +961,7 @@ ProblemSpec apply_spec(const muon_batch& b, const Mat& f, const Mat& x, void* ou
     s.a_mn = 0;
     s.b = f;
     s.b_mn = 0;
+    s.b_sym = sym_compact(m) ? 1 : 0;
   }
   s.alpha = 1.0f;
   s.beta = beta;
@@ -1579,6 +1597,7 @@ muon_status muon_testing_gemm(int M, int N, int K, int slices, int tri, int in_d
   s.out_bs = bsc;
   s.out_f16 = out_dtype == MUON_F16;
   s.row_ss = tri ? nullptr : row_ss;
+  s.mirror = 1;
   std::vector<ProblemSpec> v{s};
   return launch_gemms(v, sms, reinterpret_cast<int*>(workspace), stream, cta_pair, raster_group);
 }

@@ -20,8 +20,14 @@
 // triangle, so A = X X^T and B = b*A + c*A^2 cost about half of a full
 // product (the one-triangle products of the Megatron-Core
 // layer_sharded_muon docs, use_syrk).  The tiles of each 256 x 256 diagonal
-// block are written as computed; every tile below them is written twice, as
-// computed and transposed into the upper triangle.
+// block are written as computed.  Every tile below them is either written
+// twice, as computed and transposed into the upper triangle ("mirror"), or
+// once, when every consumer reads the matrix as symmetric: an operand
+// flagged a_sym / b_sym takes each 128-wide K stage that lies above the
+// 256 x 256 diagonal blocks from the stored lower triangle, transposed
+// (S[rows][k] = S[k][rows]: the same tensor map read MN-major), so the
+// upper triangle is never written nor read.  (That read uses the pair
+// kernel's stage geometry: K stages and row halves of 128.)
 //
 // The epilogue stages each warp's 32 x 32 piece of the tile in shared
 // memory (double-buffered) and writes it, and its transpose for mirrored
@@ -88,9 +94,11 @@ struct GemmProblem {
   int tiles_per_slice;
   int tile_begin;           // first linear tile of this problem in the launch
   int group_m;              // non-symmetric problems: row tiles per raster band
-  int tri;                  // symmetric output: lower-triangle tiles + mirror
+  int tri;                  // symmetric output: lower-triangle tiles (+ mirror)
+  int mirror;               // tri: also write the transposed tiles into the upper triangle
   int a_mn, b_mn;           // operand majors (1 = MN-major)
-  uint32_t idesc;           // tcgen05 instruction descriptor
+  int a_sym, b_sym;         // operand is a symmetric matrix stored as its lower 256-blocks (pair kernel)
+  uint32_t idesc;           // tcgen05 instruction descriptor (a_mn, b_mn majors)
   float alpha, beta, gamma, f0;
   int s_pow;                // exponent of the per-slice normalization factor
   float eps;
@@ -249,6 +257,7 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
         const GemmProblem& pr = P.prob[tc.p];
         const int arow = tc.tm * Cfg::TILE_M + static_cast<int>(rank) * BM;      // this CTA's A rows
         const int brow = tc.tn * BN + static_cast<int>(rank) * Cfg::B_ROWS;      // this CTA's B rows
+        const int a256 = (tc.tm * Cfg::TILE_M) >> 8, b256 = tc.tn;                // 256-blocks of those rows
         for (int kb = 0; kb < pr.kt; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit)) {
             record_error(P.err, abort_flag, kErrProducer);
@@ -259,22 +268,25 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
           uint8_t* a_dst = sA + stage * Cfg::A_STAGE_BYTES;
           uint8_t* b_dst = sB + stage * Cfg::B_STAGE_BYTES;
           const int k0 = kb * Cfg::KB;
-          // K-major: KSUB boxes [rows][64]; MN-major: blocks [KB][64] along M (or N).
+          // K-major: KSUB boxes [rows][64]; MN-major: blocks [KB][64] along M (or N).  A
+          // symmetric operand's stages above the diagonal blocks are read transposed (MN-major).
+          const bool amn = pr.a_mn || (pr.a_sym && (k0 >> 8) > a256);
+          const bool bmn = pr.b_mn || (pr.b_sym && (k0 >> 8) > b256);
 #pragma unroll
-          for (int j = 0; j < (pr.a_mn ? BM / 64 : Cfg::KSUB); ++j) {
-            const int x = pr.a_mn ? arow + 64 * j : k0 + 64 * j;
-            const int y = pr.a_mn ? k0 : arow;
-            uint8_t* dst = a_dst + j * (pr.a_mn ? Cfg::MN_BLOCK_BYTES : BM * BK * 2);
+          for (int j = 0; j < (amn ? BM / 64 : Cfg::KSUB); ++j) {
+            const int x = amn ? arow + 64 * j : k0 + 64 * j;
+            const int y = amn ? k0 : arow;
+            uint8_t* dst = a_dst + j * (amn ? Cfg::MN_BLOCK_BYTES : BM * BK * 2);
             if (CG == 2)
               tma_load_3d_pair(dst, &P.mapA[tc.p], &full[stage], x, y, tc.slice);
             else
               tma_load_3d(dst, &P.mapA[tc.p], &full[stage], x, y, tc.slice);
           }
 #pragma unroll
-          for (int j = 0; j < (pr.b_mn ? Cfg::B_ROWS / 64 : Cfg::KSUB); ++j) {
-            const int x = pr.b_mn ? brow + 64 * j : k0 + 64 * j;
-            const int y = pr.b_mn ? k0 : brow;
-            uint8_t* dst = b_dst + j * (pr.b_mn ? Cfg::MN_BLOCK_BYTES : Cfg::B_ROWS * BK * 2);
+          for (int j = 0; j < (bmn ? Cfg::B_ROWS / 64 : Cfg::KSUB); ++j) {
+            const int x = bmn ? brow + 64 * j : k0 + 64 * j;
+            const int y = bmn ? k0 : brow;
+            uint8_t* dst = b_dst + j * (bmn ? Cfg::MN_BLOCK_BYTES : Cfg::B_ROWS * BK * 2);
             if (CG == 2)
               tma_load_3d_pair(dst, &P.mapB[tc.p], &full[stage], x, y, tc.slice);
             else
@@ -322,12 +334,11 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
         // K-major: the next 16 K elements are 32 bytes along the swizzled row,
         // and every 64 K the next box; MN-major: the next 16 K rows are two
         // 8-row groups, 2048 bytes.
-        const uint64_t a_desc0 = pr.a_mn ? smem_desc_sw128(smem_u32(sA), Cfg::MN_BLOCK_BYTES, 1024)
-                                         : smem_desc_sw128(smem_u32(sA), 16, 1024);
-        const uint64_t b_desc0 = pr.b_mn ? smem_desc_sw128(smem_u32(sB), Cfg::MN_BLOCK_BYTES, 1024)
-                                         : smem_desc_sw128(smem_u32(sB), 16, 1024);
-        const bool a_mn = pr.a_mn != 0, b_mn = pr.b_mn != 0;
-        const uint32_t idesc = pr.idesc;
+        const uint64_t mn_desc0 = smem_desc_sw128(smem_u32(sA), Cfg::MN_BLOCK_BYTES, 1024);
+        const uint64_t k_desc0 = smem_desc_sw128(smem_u32(sA), 16, 1024);
+        const uint64_t mn_bdesc0 = smem_desc_sw128(smem_u32(sB), Cfg::MN_BLOCK_BYTES, 1024);
+        const uint64_t k_bdesc0 = smem_desc_sw128(smem_u32(sB), 16, 1024);
+        const int a256 = (tc.tm * Cfg::TILE_M) >> 8, b256 = tc.tn;
         const int kt = pr.kt;
         for (int kb = 0; kb < kt; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, limit)) {
@@ -336,6 +347,13 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
             break;
           }
           tc_fence_after();
+          // The producer's choice of major for this stage (see its loads).
+          const int k256 = (kb * Cfg::KB) >> 8;
+          const bool a_mn = pr.a_mn || (pr.a_sym && k256 > a256);
+          const bool b_mn = pr.b_mn || (pr.b_sym && k256 > b256);
+          const uint32_t idesc = pr.idesc | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
+          const uint64_t a_desc0 = a_mn ? mn_desc0 : k_desc0;
+          const uint64_t b_desc0 = b_mn ? mn_bdesc0 : k_bdesc0;
           const uint64_t ad = a_desc0 + static_cast<uint64_t>((stage * Cfg::A_STAGE_BYTES) >> 4);
           const uint64_t bd = b_desc0 + static_cast<uint64_t>((stage * Cfg::B_STAGE_BYTES) >> 4);
 #pragma unroll
@@ -396,7 +414,7 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
       const int row = row0 + lane;
       const bool row_ok = row < pr.M;
       // Mirrored tiles: strictly below the 256 x 256 diagonal blocks.
-      const bool mirror = pr.tri && tc.tm * Cfg::TILE_M >= (tc.tn + 1) * BN;
+      const bool mirror = pr.tri && pr.mirror && tc.tm * Cfg::TILE_M >= (tc.tn + 1) * BN;
       float f = pr.f0;
       if (pr.s_pow > 0) {
         const float s = 1.0f / (sqrtf(pr.sumsq[tc.slice]) + pr.eps);
@@ -405,15 +423,30 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
       const long long add_slice = static_cast<long long>(tc.slice) * pr.add_bs;
       const bool use_add = pr.beta != 0.0f && pr.addend != nullptr;
       float rss = 0.0f;
+      // The addend of a whole 32-column chunk (64 bytes of this row) is loaded
+      // one chunk ahead, so its global-memory latency overlaps the previous
+      // chunk's work instead of stalling every chunk.
+      uint4 add_cur[4], add_nxt[4];
+      auto load_addend = [&](int c, uint4 (&dst)[4]) {
+        const int col0 = tc.tn * BN + c * 32;
+        if (use_add && row_ok && col0 + 32 <= pr.N) {
+          const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(pr.addend) + add_slice +
+                                                            static_cast<long long>(row) * pr.add_ld + col0);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) dst[w] = src[w];
+        }
+      };
+      load_addend(0, add_cur);
 
       for (int c = 0; c < BN / 32; ++c) {
+        if (c + 1 < BN / 32) load_addend(c + 1, add_nxt);
         uint32_t r[32];
         __syncwarp();
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + c * 32),
                            r);
         tmem_ld_wait();
         const int col0 = tc.tn * BN + c * 32;
-        if (col0 >= pr.N) continue;                       // warp-uniform
+        if (col0 >= pr.N) continue;                       // warp-uniform (every later chunk too)
         const bool full_chunk = col0 + 32 <= pr.N;
         float v[32];
 #pragma unroll
@@ -421,11 +454,9 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
         if (use_add && row_ok) {
           const long long aoff = add_slice + static_cast<long long>(row) * pr.add_ld + col0;
           if (full_chunk) {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                reinterpret_cast<const uint16_t*>(pr.addend) + aoff);
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
-              uint4 u = src[w];
+              uint4 u = add_cur[w];
               const uint32_t words[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
               for (int h = 0; h < 4; ++h) {
@@ -516,6 +547,8 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
           for (int j = 0; j < 32 && col0 + j < pr.N; ++j)
             out16[out_slice + static_cast<long long>(col0 + j) * pr.out_ld + row] = h16[j];
         }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) add_cur[w] = add_nxt[w];
       }
       if (pr.row_ss != nullptr && row_ok)
         pr.row_ss[(static_cast<long long>(tc.slice) * pr.nt + tc.tn) * pr.M + row] = rss;
