@@ -48,7 +48,11 @@ def minimax_quintic_lp(lo: float, hi: float, points: int = 4001) -> Tuple[Tuple[
 
     k = np.arange(points)
     x = 0.5 * (lo + hi) - 0.5 * (hi - lo) * np.cos(np.pi * k / (points - 1))
-    V = np.stack([x, x ** 3, x ** 5], axis=1)
+    # Solved in the variable t = x / hi (coefficients a hi, b hi^3, c hi^5):
+    # the same problem, but with columns t, t^3, t^5 of comparable size on any
+    # interval, which keeps the solver's tolerance small next to E.
+    t = x / hi
+    V = np.stack([t, t ** 3, t ** 5], axis=1)
     ones = np.ones((points, 1))
     # 1 - p(x) <= E  ->  -V z - E <= -1 ;   p(x) - 1 <= E  ->  V z - E <= 1
     A_ub = np.vstack([np.hstack([-V, -ones]), np.hstack([V, -ones])])
@@ -57,7 +61,7 @@ def minimax_quintic_lp(lo: float, hi: float, points: int = 4001) -> Tuple[Tuple[
     if not res.success:
         raise RuntimeError(f"linear program failed: {res.message}")
     a, b, c, E = res.x
-    return (float(a), float(b), float(c)), float(E)
+    return (float(a / hi), float(b / hi ** 3), float(c / hi ** 5)), float(E)
 
 
 def quintic_image(coef, lo: float, hi: float) -> Tuple[float, float]:
