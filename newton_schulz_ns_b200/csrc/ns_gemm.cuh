@@ -257,7 +257,10 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
         const GemmProblem& pr = P.prob[tc.p];
         const int arow = tc.tm * Cfg::TILE_M + static_cast<int>(rank) * BM;      // this CTA's A rows
         const int brow = tc.tn * BN + static_cast<int>(rank) * Cfg::B_ROWS;      // this CTA's B rows
-        const int a256 = (tc.tm * Cfg::TILE_M) >> 8, b256 = tc.tn;                // 256-blocks of those rows
+        // First K stage read transposed (above the diagonal 256-blocks), per symmetric operand.
+        const int kbA = pr.a_sym ? (((tc.tm * Cfg::TILE_M) >> 8) + 1) * (256 / Cfg::KB) : 0x7FFFFFFF;
+        const int kbB = pr.b_sym ? (tc.tn + 1) * (256 / Cfg::KB) : 0x7FFFFFFF;
+        const bool a_mn0 = pr.a_mn != 0, b_mn0 = pr.b_mn != 0;
         for (int kb = 0; kb < pr.kt; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit)) {
             record_error(P.err, abort_flag, kErrProducer);
@@ -270,8 +273,8 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
           const int k0 = kb * Cfg::KB;
           // K-major: KSUB boxes [rows][64]; MN-major: blocks [KB][64] along M (or N).  A
           // symmetric operand's stages above the diagonal blocks are read transposed (MN-major).
-          const bool amn = pr.a_mn || (pr.a_sym && (k0 >> 8) > a256);
-          const bool bmn = pr.b_mn || (pr.b_sym && (k0 >> 8) > b256);
+          const bool amn = a_mn0 || kb >= kbA;
+          const bool bmn = b_mn0 || kb >= kbB;
 #pragma unroll
           for (int j = 0; j < (amn ? BM / 64 : Cfg::KSUB); ++j) {
             const int x = amn ? arow + 64 * j : k0 + 64 * j;
@@ -338,7 +341,10 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
         const uint64_t k_desc0 = smem_desc_sw128(smem_u32(sA), 16, 1024);
         const uint64_t mn_bdesc0 = smem_desc_sw128(smem_u32(sB), Cfg::MN_BLOCK_BYTES, 1024);
         const uint64_t k_bdesc0 = smem_desc_sw128(smem_u32(sB), 16, 1024);
-        const int a256 = (tc.tm * Cfg::TILE_M) >> 8, b256 = tc.tn;
+        const int kbA = pr.a_sym ? (((tc.tm * Cfg::TILE_M) >> 8) + 1) * (256 / Cfg::KB) : 0x7FFFFFFF;
+        const int kbB = pr.b_sym ? (tc.tn + 1) * (256 / Cfg::KB) : 0x7FFFFFFF;
+        const bool a_mn0 = pr.a_mn != 0, b_mn0 = pr.b_mn != 0;
+        const uint32_t idesc0 = pr.idesc;
         const int kt = pr.kt;
         for (int kb = 0; kb < kt; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, limit)) {
@@ -348,10 +354,9 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
           }
           tc_fence_after();
           // The producer's choice of major for this stage (see its loads).
-          const int k256 = (kb * Cfg::KB) >> 8;
-          const bool a_mn = pr.a_mn || (pr.a_sym && k256 > a256);
-          const bool b_mn = pr.b_mn || (pr.b_sym && k256 > b256);
-          const uint32_t idesc = pr.idesc | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
+          const bool a_mn = a_mn0 || kb >= kbA;
+          const bool b_mn = b_mn0 || kb >= kbB;
+          const uint32_t idesc = idesc0 | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
           const uint64_t a_desc0 = a_mn ? mn_desc0 : k_desc0;
           const uint64_t b_desc0 = b_mn ? mn_bdesc0 : k_bdesc0;
           const uint64_t ad = a_desc0 + static_cast<uint64_t>((stage * Cfg::A_STAGE_BYTES) >> 4);

@@ -17,11 +17,12 @@
 //   * A = sum_r X_r X_r^T: each CTA multiplies its own columns on the tensor
 //     core (fp32 in TMEM) and pushes the lower triangle of each row of its
 //     partial to the CTA that owns the row's 8-row block, with distributed-
-//     shared-memory stores; after a cluster barrier each owner sums its rows
-//     over the C partials in rank order (deterministic), scales and rounds
-//     them to bf16 and pushes them into every CTA's copy of A; after a
-//     second barrier each CTA fills A's upper triangle from the lower one
-//     (A is exactly symmetric, as on the GEMM path);
+//     shared-memory stores that count their bytes on the owner's mbarrier;
+//     once all C partials of its rows have arrived each owner sums them in
+//     rank order (deterministic), scales and rounds them to bf16 and pushes
+//     them into every CTA's copy of A the same way; once all of A's lower
+//     triangle has arrived each CTA fills the upper triangle from it (A is
+//     exactly symmetric, as on the GEMM path);
 //   * each CTA forms B = b A + c A^2 over its copy of A (128^3, redundantly;
 //     cheaper than another exchange) and its own columns of a X + B X, which
 //     need no other CTA's data, and writes them back over X;
@@ -45,7 +46,7 @@
 // 32 (w % 4) .. + 31 (one row per thread) and half w / 4 of the columns.
 // Every mbarrier wait is bounded; a CTA that gives up records an error,
 // stops issuing work and still takes every cluster barrier, so its peers
-// finish too.
+// finish too (their bounded waits for its data run out).
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -65,7 +66,7 @@ constexpr int SMALL_A_BYTES = 2 * SMALL_BLK;                  // A (then B in pl
 constexpr int SMALL_RECV_BYTES = 128 * 512;                   // C slots of fp32 partial rows
 constexpr int SMALL_SMEM_BYTES = 1024 + SMALL_X_BYTES + SMALL_A_BYTES + SMALL_RECV_BYTES + 64;
 
-enum SmallError : int { kSmallErrLoad = 5, kSmallErrMma = 6 };
+enum SmallError : int { kSmallErrLoad = 5, kSmallErrMma = 6, kSmallErrExchange = 7 };
 
 struct __align__(64) SmallParams {
   CUtensorMap map_in;        // ns_in  [slices][m][n] bf16, box {64, 128, 1}, 128-B swizzle
@@ -303,8 +304,9 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
   uint8_t* Xs = smem;
   uint8_t* As = Xs + SMALL_X_BYTES;   // A, overwritten in place by B = b A + c A^2
   uint8_t* Rv = As + SMALL_A_BYTES;   // partial rows pushed here by every CTA of the cluster
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Rv + SMALL_RECV_BYTES);   // [0] load, [1] MMA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  // [0] load, [1] MMA, [2] partial rows received (owner), [3] A received
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Rv + SMALL_RECV_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x;
@@ -340,6 +342,8 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
     *abort_flag = 0;
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
+    mbar_init(&bars[2], 1);
+    mbar_init(&bars[3], 1);
     fence_barrier_init();
     tma_prefetch_desc(&P.map_in);
     tma_prefetch_desc(&P.map_out);
@@ -390,11 +394,30 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
   const uint32_t rv0 = smem_u32(Rv);
   const uint32_t a0 = smem_u32(As);
 
+  // Bytes one exchange delivers to this CTA: as an owner, the partial rows of
+  // its blocks from every CTA (16 bytes per 4 columns up to the diagonal);
+  // and A's lower triangle in 8 x 8 blocks from all owners.
+  uint32_t recv_bytes = 0;
+  for (int lb = 0; lb < kb && static_cast<int>(rank) * kb + lb < G; ++lb) {
+    const int b = unfold(static_cast<int>(rank) * kb + lb);
+    for (int r8 = 0; r8 < 8; ++r8) recv_bytes += 16u * static_cast<uint32_t>(((8 * b + r8) >> 2) + 1);
+  }
+  recv_bytes *= static_cast<uint32_t>(C);
+  const uint32_t a_bytes = 64u * static_cast<uint32_t>(G * (G + 1));
+  uint32_t xphase = 0;        // completed exchanges (parity of the receive barriers)
+
   // ---- A = fA * X X^T over the cluster, into every CTA's As (bf16; fp16 in
-  //      the Gram form), upper triangle mirrored.  Every CTA takes both
-  //      cluster barriers whether or not it is still working, so a CTA that
-  //      gave up never strands its peers.
+  //      the Gram form), upper triangle mirrored.  Partial rows and A's rows
+  //      travel as st.async stores that complete bytes on the receiver's
+  //      mbarrier, so each CTA waits only for the data it needs, not for the
+  //      whole cluster.  (Every CTA's next exchange starts after it holds this
+  //      exchange's A, which needs every owner to have finished reading its
+  //      receive slots: the slots and barriers are never overwritten early.)
   auto exchange = [&](float fA) {
+    if (ok && tid == 0) {
+      mbar_arrive_expect_tx(&bars[2], recv_bytes);
+      mbar_arrive_expect_tx(&bars[3], a_bytes);
+    }
     // partial X_r X_r^T -> TMEM columns [0, 128)
     if (ok) {
       if (tid == 0) {
@@ -420,21 +443,26 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
         const int owner = p / kb;
         const int t = static_cast<int>(rank) * Rm + (p - owner * kb) * 8 + (row & 7);   // slot `rank`
         const int jn = min(16, (row >> 2) + 1 - half * 16);                             // chunks to send
+        const uint32_t rbar = mapa_shared(smem_u32(&bars[2]), static_cast<uint32_t>(owner));
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           if (j < jn) {
             const uint32_t dst = mapa_shared(rv0 + recv_chunk(t, half * 16 + j), static_cast<uint32_t>(owner));
-            st_cluster_v4(dst, make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+            st_async_v4(dst, make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]), rbar);
           }
         }
       }
     }
-    tc_fence_before();
-    cluster_sync();           // every partial row has reached its owner
-
-    // owner: for its row blocks b, A[8b .. 8b+7][0 .. 8b+7] = fA * sum over
-    // the slots in rank order, pushed to every CTA (the diagonal block's
-    // upper half carries unsent entries; the mirror below replaces it)
+    tc_fence_before();        // the TMEM reads above precede the next product's writes
+    // owner: wait for its slots, then for its row blocks b,
+    // A[8b .. 8b+7][0 .. 8b+7] = fA * sum over the slots in rank order,
+    // pushed to every CTA (the diagonal block's upper half carries unsent
+    // entries; the mirror below replaces it)
+    if (ok) {
+      const bool got = mbar_wait_cluster_bounded(&bars[2], xphase & 1u, abort_flag, P.timeout_ns);
+      ok = __syncthreads_and(got) != 0;
+      if (!ok && tid == 0) small_record_error(P.err, abort_flag, kSmallErrExchange);
+    }
     if (ok) {
       int items = 0;
       for (int lb = 0; lb < kb && rank * kb + lb < G; ++lb) items += 8 * (unfold(rank * kb + lb) + 1);
@@ -470,13 +498,20 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
         for (int e = 0; e < 8; ++e) acc[e] *= fA;
         const uint4 pk = GRAM ? pack_f16x8(acc) : pack_bf16x8(acc);
         const uint32_t dst = a0 + sw128_chunk(8 * b + r8, g);
-        for (int q = 0; q < C; ++q) st_cluster_v4(mapa_shared(dst, static_cast<uint32_t>(q)), pk);
+        const uint32_t abar = smem_u32(&bars[3]);
+        for (int q = 0; q < C; ++q)
+          st_async_v4(mapa_shared(dst, static_cast<uint32_t>(q)), pk, mapa_shared(abar, static_cast<uint32_t>(q)));
       }
-      fence_proxy_async_cluster();
     }
-    cluster_sync();           // every CTA holds the lower triangle of A; the receive slots are free again
+    // every CTA: wait for all of A's lower triangle
+    if (ok) {
+      const bool got = mbar_wait_cluster_bounded(&bars[3], xphase & 1u, abort_flag, P.timeout_ns);
+      ok = __syncthreads_and(got) != 0;
+      if (!ok && tid == 0) small_record_error(P.err, abort_flag, kSmallErrExchange);
+    }
+    ++xphase;
 
-    // upper triangle of A from the lower one (local)
+    // upper triangle of A from the lower one (local; ends with the async-proxy fence)
     if (ok) mirror_upper(As, G, tid);
     __syncthreads();
   };

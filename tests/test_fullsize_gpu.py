@@ -118,3 +118,32 @@ def test_llama8b_full_step_standard_sampled():
 def test_moe_full_step_gram_sampled():
     # w1 of experts 0 and 37 (wide), w2 of experts 5 and 63 (tall).
     _run_full_step("moe", "gram", [(0, 0), (0, 37), (1, 5), (1, 63)])
+
+
+def test_gram_rank_deficient_moe_slices_stay_in_band():
+    # Expert-sized slices (2048 x 7168 and its transpose) of rank 1 and 64,
+    # Gram form with the default restarts, through the GEMM path: the top
+    # singular value stays in the quintic's band and the result is as close
+    # to the exact one as a numpy model of the storage precisions.
+    import newton_schulz_ns_b200 as mn
+    from precision_model import ns_gram_f16
+    for shape, rank in [((2048, 7168), 1), ((7168, 2048), 64)]:
+        r, c = shape
+        g = torch.Generator().manual_seed(rank + r)
+        x = (torch.randn(r, rank, generator=g) @ torch.randn(rank, c, generator=g)).to(torch.bfloat16)
+        U = x.to(DEV)[None]
+        out = torch.empty_like(U)
+        b = mn.Batch(1, r, c, ns_in=U, ns_out=out)
+        ws = mn.allocate_workspace([b], 2)
+        mn.muon_gram_ns_batched([b], mn.Hparams(), ws)
+        torch.cuda.synchronize()
+        assert mn.workspace_error(ws) == 0
+        got, u = f64(out[0]), f64(U[0])
+        assert np.all(np.isfinite(got))
+        smax = float(np.linalg.norm(got, 2))
+        assert smax <= 1.25, (shape, rank, smax)
+        ref = oracle.gram_newton_schulz(u, restart=3)
+        model = ns_gram_f16(u, restart=3)
+        assert rel(got, ref) <= max(3 * rel(model, ref), 3e-2), (shape, rank, rel(got, ref), rel(model, ref))
+        del ws
+        torch.cuda.empty_cache()

@@ -300,7 +300,7 @@ def test_rms_norm_scale_gives_orthogonal_updates_rms_two_tenths(shape, extra):
     assert orc.update_scale(*shape, mode="rms_norm", extra=extra) == orc.rms_norm_scale(*shape, extra)
 
 
-@pytest.mark.parametrize("shape", [(576, 64), (256, 256), (1024, 512), (14336, 4096), (7, 1)])
+@pytest.mark.parametrize("shape", [(576, 64), (256, 256), (1024, 512), (3584, 1024), (7, 1)])
 def test_spectral_scale_gives_unit_rms_operator_norm_when_fan_out_ge_fan_in(shape):
     # ||s O||_{RMS->RMS} = sqrt(fan_in / fan_out) * ||s O||_2 = 1 for an orthogonal O.
     r, c = shape
