@@ -132,18 +132,20 @@ def kernel_source_hash():
 
 
 def measured_traffic(key, variant):
-    """DRAM bytes of one Newton-Schulz call from the committed ncu summary, or None.
+    """DRAM bytes of one Newton-Schulz call, scaled from the committed ncu summary, or None.
 
-    The summary records the hash of the kernel sources it was captured with;
-    a different hash (the kernel changed since) gives None.
+    The summary holds per-launch captures of a one-layer case (a few launches
+    per ncu run) and their scaling to one call of the full workload; it
+    records the hash of the kernel sources it was captured with, and a
+    different hash (the kernel changed since) gives None.
     """
     import re
-    path = os.path.join(ROOT, "profiles", f"ns_gemm_{key}_{variant}_traffic.md")
+    path = os.path.join(ROOT, "profiles", f"ns_gemm_{key}_{variant}_traffic_scaled.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
-    m_bytes = re.search(r"dram_bytes_per_ns_call:\s*([0-9.eE+]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_ns_call_scaled:\s*([0-9.eE+]+)", text)
     if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
         return None
     return float(m_bytes.group(1))
@@ -572,7 +574,9 @@ def run_ours(args, wl, variant, rank, world, local_rank):
                      "frac": round(achieved / peak_s, 4), "frac_of_burst": round(achieved / peak_b, 4),
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a long step)",
                      "traffic": measured_traffic(wl.key, variant) if args.scale_down == 1 else None,
-                     "traffic_unit": "bytes per Newton-Schulz call (ncu dram__bytes_read.sum + write.sum)"},
+                     "traffic_unit": "bytes per Newton-Schulz call: ncu dram__bytes_read.sum + write.sum of "
+                                     "one-layer launches, scaled by the slices and steps of one call "
+                                     f"(profiles/ns_gemm_{wl.key}_{variant}_traffic_scaled.md)"},
         "gpu_launches": int(launches),
         "clocks": clk,
     }

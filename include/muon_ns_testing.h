@@ -15,7 +15,8 @@
  * add_dtype (MUON_BF16 | MUON_F16) the types of C and D.  D may be NULL
  * when beta == 0.  All pointers are device memory; ld/bs are in elements.
  * row_ss (device, may be NULL; non-tri only) receives, per slice, per
- * 256-column block and per row, the sum of squares of the stored C values.
+ * 128-column block and per row, the sum of squares of the stored C values
+ * ([slices][ceil(N / 128) rounded up to even][M]).
  * cta_pair: 0 lets the library choose the tile kernel, 1 forces single-CTA
  * 128 x 256 tiles, 2 forces 2-CTA (cta_group::2) 256 x 256 tiles.
  * raster_group: row tiles per raster band of a non-symmetric problem

@@ -293,10 +293,10 @@ struct NsBatchWs {
 };
 
 // Partial row sums per output row that the last product leaves: one per
-// 256-column tile on the GEMM path, one per CTA and column half on the fused
-// path (clusters of at most SMALL_MAX_CLUSTER CTAs).
+// 128-column half of a 256-column tile on the GEMM path, one per CTA and
+// column half on the fused path (clusters of at most SMALL_MAX_CLUSTER CTAs).
 inline int row_partials_per_row(int64_t cols) {
-  return static_cast<int>(std::max<int64_t>((cols + BN - 1) / BN, 2 * SMALL_MAX_CLUSTER));
+  return static_cast<int>(std::max<int64_t>(2 * ((cols + BN - 1) / BN), 2 * SMALL_MAX_CLUSTER));
 }
 
 bool small_shape_ok(int64_t rows, int64_t cols);
@@ -501,7 +501,7 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
       if (c.addend) c.addend = static_cast<const uint16_t*>(s.addend) + static_cast<int64_t>(s0) * s.add_bs;
       c.out = static_cast<uint16_t*>(s.out) + static_cast<int64_t>(s0) * s.out_bs;
       if (c.sumsq) c.sumsq = s.sumsq + s0;
-      if (c.row_ss) c.row_ss = s.row_ss + static_cast<int64_t>(s0) * cdiv(s.N, BN) * s.M;
+      if (c.row_ss) c.row_ss = s.row_ss + static_cast<int64_t>(s0) * 2 * cdiv(s.N, BN) * s.M;
       chunks.push_back(c);
       chunk_cg.push_back(cg);
     }
@@ -580,16 +580,23 @@ muon_status launch_gemms(const std::vector<ProblemSpec>& specs, int sms, int* er
       const int kb_rows = cg == 2 ? GemmCfg<2>::KB : GemmCfg<1>::KB;
       if (!encode_map(&P.mapA[np], s.a, 64, s.a_mn ? kb_rows : BM)) return MUON_CUDA_ERROR;
       if (!encode_map(&P.mapB[np], s.b, 64, s.b_mn ? kb_rows : b_rows)) return MUON_CUDA_ERROR;
-      // Output: 32 x 32 boxes, swizzled for the direct staging layout, plain for the transposed one.
+      // Output: 32 x 32 boxes, swizzled for the staging layout.
       const Mat c{s.out, s.M, s.N, s.out_ld, s.out_bs, s.slices, s.out_f16};
       if (!encode_map(&P.mapC[np], c, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return MUON_CUDA_ERROR;
-      if (!encode_map(&P.mapCT[np], c, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) return MUON_CUDA_ERROR;
       tiles += static_cast<long long>(g.tiles_per_slice) * s.slices;
       if (tiles > INT32_MAX) return MUON_BAD_SHAPE;
       ++np;
     }
     P.num_problems = np;
     P.total_tiles = static_cast<int>(tiles);
+    // Split each tile's epilogue over two warps per lane quadrant where it
+    // would not hide behind the next tile's main loop: short K (<= 2048) or
+    // at most one wave of tiles (each CTA's epilogue is then on the critical
+    // path).  Long-K launches keep one warp per quadrant (measured: splitting
+    // them cost the power-capped Llama-8B call about 1%).
+    bool short_k = false;
+    for (int k = 0; k < np; ++k) short_k |= P.prob[k].K <= 2048;
+    P.epi_split = (short_k || tiles <= units) ? 1 : 0;
   }
   // Programmatic dependent launch: each GEMM may start its prologue (barrier
   // setup, TMEM allocation) on idle SMs while the previous kernel drains; the
@@ -1237,7 +1244,7 @@ muon_status finalize_gemm_row_sums(const muon_batch* batches, int nb, const Layo
     const muon_batch& b = batches[i];
     if (batch_empty(b) || fused[i] || !b.row_sumsq) continue;
     const muon_status st = launch_row_finalize(reinterpret_cast<const float*>(ws + L.nsb[i].rs_off),
-                                               static_cast<int>(cdiv(b.cols, BN)), b.rows, b.n, b.row_sumsq, sms,
+                                               static_cast<int>(2 * cdiv(b.cols, BN)), b.rows, b.n, b.row_sumsq, sms,
                                                stream);
     if (st != MUON_OK) return st;
   }

@@ -30,18 +30,23 @@
 // kernel's stage geometry: K stages and row halves of 128.)
 //
 // The epilogue stages each warp's 32 x 32 piece of the tile in shared
-// memory (double-buffered) and writes it, and its transpose for mirrored
-// tiles, with TMA bulk tensor stores, which clip at the slice's bounds.
+// memory (double-buffered) and writes it with TMA bulk tensor stores, which
+// clip at the slice's bounds; the transposed copy of a mirrored tile goes
+// straight to global memory (64 contiguous bytes per column and warp).
 //
-// Roles (192 threads, one CTA per SM, persistent over a static tile stride):
+// Roles (320 threads, one CTA per SM, persistent over a static tile stride):
 //   warp 0 lane 0 : TMA producer over a STAGES-deep shared-memory ring (in a
 //                   pair, both CTAs load their halves; the leader's barrier
 //                   counts the bytes of both)
 //   warp 1        : TMEM allocation; lane 0 issues the MMAs (the leader only
 //                   in a pair; its commits reach both CTAs' barriers)
-//   warps 2..5    : epilogue, one TMEM lane (= output row) per thread;
-//                   two 256-column accumulators let the epilogue of one
-//                   tile overlap the main loop of the next.
+//   warps 2..9    : epilogue, one TMEM lane (= output row) per thread; in
+//                   launches whose tiles have a short main loop (K <= 2048)
+//                   or that hold at most one wave of tiles, two warps per
+//                   lane quadrant split a tile's 256 columns (its epilogue
+//                   then takes half as long), otherwise warps 2..5 take whole
+//                   tiles; two 256-column accumulators let the epilogue of
+//                   one tile overlap the main loop of the next.
 // Every wait is bounded (see mbar_wait_bounded); a role that gives up
 // records an error code in *err, raises the CTA's abort flag and leaves;
 // in-flight TMA loads and MMAs are waited for (bounded) before TMEM is freed.
@@ -58,11 +63,12 @@ constexpr int BM = 128;                          // rows of A (and of the accumu
 constexpr int BN = 256;                          // columns of a tile
 constexpr int BK = 64;                           // K of one TMA box (one 128-byte swizzled row of bf16)
 constexpr uint32_t TMEM_COLS = 2 * BN;           // two accumulators
-constexpr int GEMM_THREADS = 192;
 constexpr int MAX_PROBLEMS = 8;
-constexpr int EPI_WARPS = 4;
+constexpr int EPI_WARPS = 8;                                // two per TMEM lane quadrant, one per column half
+constexpr int GEMM_THREADS = 64 + 32 * EPI_WARPS;
+constexpr int EPI_CHUNKS = BN / 32 / 2;                     // 32-column chunks per epilogue warp and tile
 constexpr int STG_BYTES = 32 * 32 * 2;                      // one 32 x 32 box of 16-bit values
-constexpr int STG_PER_WARP = 2 /*buffers*/ * 2 /*direct, mirror*/ * STG_BYTES;
+constexpr int STG_PER_WARP = 2 /*buffers*/ * STG_BYTES;
 
 // A stage holds KB = 64 * KSUB elements of K.  K-major operands are KSUB
 // boxes of [rows][64] (one 128-byte swizzled row each); MN-major operands are
@@ -109,17 +115,18 @@ struct GemmProblem {
   long long out_ld, out_bs;
   int out_f16;              // 1: C is fp16, 0: bf16
   int add_f16;              // 1: D is fp16, 0: bf16
-  float* row_ss;            // optional [slices][nt][M]: sum over the tile's columns of bf16(C)^2
+  float* row_ss;            // optional [slices][2 nt][M]: per 128-column half of a tile, sum of bf16(C)^2
 };
 
 struct __align__(64) GemmParams {
   CUtensorMap mapA[MAX_PROBLEMS];
   CUtensorMap mapB[MAX_PROBLEMS];
-  CUtensorMap mapC[MAX_PROBLEMS];     // output, 32 x 32 boxes, 64-byte swizzle (direct tiles)
-  CUtensorMap mapCT[MAX_PROBLEMS];    // output, 32 x 32 boxes, no swizzle (mirrored tiles)
+  CUtensorMap mapC[MAX_PROBLEMS];     // output, 32 x 32 boxes, 64-byte swizzle
   GemmProblem prob[MAX_PROBLEMS];
   int num_problems;
   int total_tiles;
+  int epi_split;                      // 1: two epilogue warps per lane quadrant, one per column half;
+                                      // 0: warps 2..5 take whole tiles and warps 6..9 stay idle
   int* err;
   unsigned long long timeout_ns;
 };
@@ -206,7 +213,7 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128 * CG);     // every epilogue thread of the pair
+      mbar_init(&tempty[a], 32 * (P.epi_split ? EPI_WARPS : EPI_WARPS / 2) * CG);   // every working epilogue thread of the pair
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -217,7 +224,6 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
       tma_prefetch_desc(&P.mapA[p]);
       tma_prefetch_desc(&P.mapB[p]);
       tma_prefetch_desc(&P.mapC[p]);
-      tma_prefetch_desc(&P.mapCT[p]);
     }
   }
   if (warp == 1) {
@@ -398,11 +404,21 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
     }
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    // Warps 2..9: warp & 3 is the TMEM lane quadrant a warp may access (rows
+    // 32q .. 32q + 31 of the CTA's accumulator).  With epi_split the two
+    // warps of a quadrant take one 128-column half of the tile each (launches
+    // whose main loop per tile is short, where the epilogue would be exposed);
+    // otherwise warps 2..5 take whole tiles, which hide behind long main loops.
+    const int q = warp & 3;
+    const int ch = (warp - 2) >> 2;
+    const bool split = P.epi_split != 0;
+    const int c_begin = split ? ch * EPI_CHUNKS : 0;
+    const int c_end = split ? c_begin + EPI_CHUNKS : 2 * EPI_CHUNKS;
     uint8_t* stg = sStg + (warp - 2) * STG_PER_WARP;
+    const bool idle = !split && ch == 1;
     int iter = 0;
     uint32_t stores = 0;     // bulk groups this warp has committed (selects the staging buffer)
-    for (int t = unit; t < P.total_tiles; t += units, ++iter) {
+    for (int t = unit; t < P.total_tiles && !idle; t += units, ++iter) {
       const TileCoord tc = decode_tile<CG>(P, t);
       const GemmProblem& pr = P.prob[tc.p];
       const int acc = iter & 1;
@@ -427,7 +443,7 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
       }
       const long long add_slice = static_cast<long long>(tc.slice) * pr.add_bs;
       const bool use_add = pr.beta != 0.0f && pr.addend != nullptr;
-      float rss = 0.0f;
+      float rss0 = 0.0f, rss1 = 0.0f;   // sums of squares of the tile's two 128-column halves
       // The addend of a whole 32-column chunk (64 bytes of this row) is loaded
       // one chunk ahead, so its global-memory latency overlaps the previous
       // chunk's work instead of stalling every chunk.
@@ -441,10 +457,10 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
           for (int w = 0; w < 4; ++w) dst[w] = src[w];
         }
       };
-      load_addend(0, add_cur);
+      load_addend(c_begin, add_cur);
 
-      for (int c = 0; c < BN / 32; ++c) {
-        if (c + 1 < BN / 32) load_addend(c + 1, add_nxt);
+      for (int c = c_begin; c < c_end; ++c) {
+        if (c + 1 < c_end) load_addend(c + 1, add_nxt);
         uint32_t r[32];
         __syncwarp();
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + c * 32),
@@ -486,6 +502,7 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
         }
         // Round to the output type once; these are the values stored.
         uint16_t h16[32];
+        float css = 0.0f;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           float x = v[j] * f;
@@ -500,63 +517,63 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
             h16[j] = __bfloat16_as_ushort(hv);
             xr = __bfloat162float(hv);
           }
-          if (row_ok && col0 + j < pr.N) rss += xr * xr;
+          if (row_ok && col0 + j < pr.N) css += xr * xr;
         }
+        if (c < EPI_CHUNKS)
+          rss0 += css;
+        else
+          rss1 += css;
         // Boxes whose innermost extent lies fully inside the slice go out by
-        // TMA; the ragged last chunk of a row (and of a mirrored column) is
-        // written element by element, so nothing past the slice's last column
-        // is ever touched.
+        // TMA; the ragged last chunk of a row is written element by element,
+        // so nothing past the slice's last column is ever touched.  Mirrored
+        // columns go straight to global memory: for each column j the warp's
+        // 32 rows are 64 contiguous bytes of output row col0 + j.
         const bool st_d = full_chunk;
-        const bool st_m = mirror && row0 + 32 <= pr.M;
         const long long out_slice = static_cast<long long>(tc.slice) * pr.out_bs;
         uint16_t* out16 = reinterpret_cast<uint16_t*>(pr.out);
-        if (st_d || st_m) {
+        if (st_d) {
           // The staging buffer used two stores ago must have been read out.
-          const uint32_t buf = stores & 1u;
-          uint8_t* sd = stg + buf * (2 * STG_BYTES);
-          uint8_t* sm = sd + STG_BYTES;
+          uint8_t* sd = stg + (stores & 1u) * STG_BYTES;
           if (lane == 0 && stores >= 2) bulk_wait_group_read<1>();
           __syncwarp();
-          if (st_d) {
-            // Row `lane`, 64 bytes, 16-byte chunks placed by the 64-byte swizzle.
+          // Row `lane`, 64 bytes, 16-byte chunks placed by the 64-byte swizzle.
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const uint4 val = make_uint4(
-                  static_cast<uint32_t>(h16[8 * w + 0]) | (static_cast<uint32_t>(h16[8 * w + 1]) << 16),
-                  static_cast<uint32_t>(h16[8 * w + 2]) | (static_cast<uint32_t>(h16[8 * w + 3]) << 16),
-                  static_cast<uint32_t>(h16[8 * w + 4]) | (static_cast<uint32_t>(h16[8 * w + 5]) << 16),
-                  static_cast<uint32_t>(h16[8 * w + 6]) | (static_cast<uint32_t>(h16[8 * w + 7]) << 16));
-              *reinterpret_cast<uint4*>(sd + lane * 64 + ((w ^ ((lane >> 1) & 3)) << 4)) = val;
-            }
-          }
-          if (st_m) {
-            // Transposed box: row j holds column j of this warp's 32 rows.
-            uint16_t* mt = reinterpret_cast<uint16_t*>(sm);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) mt[j * 32 + lane] = h16[j];
+          for (int w = 0; w < 4; ++w) {
+            const uint4 val = make_uint4(
+                static_cast<uint32_t>(h16[8 * w + 0]) | (static_cast<uint32_t>(h16[8 * w + 1]) << 16),
+                static_cast<uint32_t>(h16[8 * w + 2]) | (static_cast<uint32_t>(h16[8 * w + 3]) << 16),
+                static_cast<uint32_t>(h16[8 * w + 4]) | (static_cast<uint32_t>(h16[8 * w + 5]) << 16),
+                static_cast<uint32_t>(h16[8 * w + 6]) | (static_cast<uint32_t>(h16[8 * w + 7]) << 16));
+            *reinterpret_cast<uint4*>(sd + lane * 64 + ((w ^ ((lane >> 1) & 3)) << 4)) = val;
           }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (st_d) tma_store_3d(&P.mapC[tc.p], sd, col0, row0, tc.slice);
-            if (st_m) tma_store_3d(&P.mapCT[tc.p], sm, row0, col0, tc.slice);
+            tma_store_3d(&P.mapC[tc.p], sd, col0, row0, tc.slice);
             bulk_commit_group();
           }
           ++stores;
-        }
-        if (!st_d && row_ok) {
+        } else if (row_ok) {
           for (int j = 0; j < 32 && col0 + j < pr.N; ++j)
             out16[out_slice + static_cast<long long>(row) * pr.out_ld + col0 + j] = h16[j];
         }
-        if (mirror && !st_m && row_ok) {
-          for (int j = 0; j < 32 && col0 + j < pr.N; ++j)
-            out16[out_slice + static_cast<long long>(col0 + j) * pr.out_ld + row] = h16[j];
+        if (mirror && row_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col0 + j < pr.N) out16[out_slice + static_cast<long long>(col0 + j) * pr.out_ld + row] = h16[j];
         }
 #pragma unroll
         for (int w = 0; w < 4; ++w) add_cur[w] = add_nxt[w];
       }
-      if (pr.row_ss != nullptr && row_ok)
-        pr.row_ss[(static_cast<long long>(tc.slice) * pr.nt + tc.tn) * pr.M + row] = rss;
+      if (pr.row_ss != nullptr && row_ok) {
+        float* rs = pr.row_ss + (static_cast<long long>(tc.slice) * 2 * pr.nt + 2 * tc.tn) * pr.M + row;
+        if (split) {
+          rs[static_cast<long long>(ch) * pr.M] = ch == 0 ? rss0 : rss1;
+        } else {
+          rs[0] = rss0;
+          rs[pr.M] = rss1;
+        }
+      }
       tc_fence_before();
       if (CG == 2)
         mbar_arrive_leader(&tempty[acc]);

@@ -332,14 +332,14 @@ def test_testing_options_round_trip_and_range_checks(mn):
 
 def test_row_sum_partials_take_workspace_only_when_requested(mn):
     from newton_schulz_ns_b200 import _capi
-    n, r, c = 3, 300, 520
+    n, r, c = 3, 300, 2100
     plain = _fake_batch(mn, n, r, c)
     asked = _fake_batch(mn, n, r, c)
     asked.row_sumsq = 0x7F0000400000
     for which in (1, 2):
         a = _capi.lib.muon_workspace_size((_capi.MuonBatch * 1)(plain), 1, which)
         b = _capi.lib.muon_workspace_size((_capi.MuonBatch * 1)(asked), 1, which)
-        # one float per output row and per 256-column tile (at least 16 per row: the fused path's
-        # CTA halves), rounded up to the 256-byte alignment
-        per_row = max((c + 255) // 256, 16)
+        # one float per output row and per 128-column half of a 256-column tile (at least 16 per
+        # row: the fused path's CTA halves), rounded up to the 256-byte alignment
+        per_row = max(2 * ((c + 255) // 256), 16)
         assert b - a == (4 * n * per_row * r + 255) // 256 * 256

@@ -137,14 +137,14 @@ def test_row_sums_of_squares(mn, cta_pair):
     A = _rnd((S, M, K), torch.bfloat16, 7)
     B = _rnd((S, K, N), torch.bfloat16, 8)
     C = _empty((S, M, N), torch.bfloat16)
-    nt = (N + 255) // 256
-    rss = torch.full((S, nt, M), float("nan"), device=DEV)
+    nh = 2 * ((N + 255) // 256)                 # one partial per 128-column half of a 256-column tile
+    rss = torch.full((S, nh, M), float("nan"), device=DEV)
     ws = _ws()
     mn.testing_gemm(A, False, B, True, C, K=K, row_ss=rss, cta_pair=cta_pair, workspace=ws)
     torch.cuda.synchronize()
     c = _f64(C)
-    for t in range(nt):
-        ref = np.sum(c[:, :, 256 * t:256 * (t + 1)] ** 2, axis=2)
+    for t in range(nh):
+        ref = np.sum(c[:, :, 128 * t:128 * (t + 1)] ** 2, axis=2)
         assert np.allclose(_f64(rss)[:, t], ref, rtol=1e-5)
 
 
@@ -197,3 +197,30 @@ def test_bounded_wait_times_out_and_context_survives(mn):
     torch.cuda.synchronize()
     assert mn.workspace_error(ws) == 0
     _check(C, _f64(A) @ np.swapaxes(_f64(B), 1, 2))
+
+
+@pytest.mark.parametrize("cta_pair", PAIRS)
+def test_long_k_launch_with_several_waves(mn, cta_pair):
+    # K > 2048 and more tiles than one wave: the launch keeps one epilogue
+    # warp per TMEM lane quadrant (short-K or single-wave launches split each
+    # tile's columns over two).  Addend, per-slice factor and row sums, as
+    # the Newton-Schulz apply phase uses them.
+    S, M, N, K = 2, 2048, 2600, 2304
+    A = _rnd((S, M, K), torch.bfloat16, 21, 0.05)
+    B = _rnd((S, K, N), torch.bfloat16, 22, 0.05)
+    D = _rnd((S, M, N), torch.bfloat16, 23)
+    C = _empty((S, M, N), torch.bfloat16)
+    ss = torch.tensor([4.0, 9.0], device=DEV)
+    nh = 2 * ((N + 255) // 256)
+    rss = torch.full((S, nh, M), float("nan"), device=DEV)
+    ws = _ws()
+    mn.testing_gemm(A, False, B, True, C, K=K, D=D, alpha=1.0, beta=0.75, f0=1.0, s_pow=1, sumsq=ss, eps=0.0,
+                    row_ss=rss, cta_pair=cta_pair, workspace=ws)
+    torch.cuda.synchronize()
+    f = np.array([1 / 2.0, 1 / 3.0])[:, None, None]
+    ref = f * (_f64(A) @ _f64(B) + 0.75 * _f64(D))
+    _check(C, ref)
+    c = _f64(C)
+    for t in range(nh):
+        want = np.sum(c[:, :, 128 * t:128 * (t + 1)] ** 2, axis=2)
+        assert np.allclose(_f64(rss)[:, t], want, rtol=1e-5)
