@@ -156,7 +156,11 @@ muon_status device_setup(int* sms_out, int* pair_units_out = nullptr) {
           cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SMALL_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(ns_small_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SMALL_SMEM_BYTES) != cudaSuccess) {
+                               SMALL_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(ns_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               STREAM_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(ns_stream_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               STREAM_SMEM_BYTES) != cudaSuccess) {
         d.ready = false;
         return MUON_CUDA_ERROR;
       }
@@ -744,16 +748,36 @@ SmallSplit small_split(int64_t n) {
   return SmallSplit{C, 64 * static_cast<int>(cdiv(blocks, C))};
 }
 
-// A wide slice (rows <= cols) the fused kernel takes: rows <= 128 and
-// cols <= 8 * 512.
-bool small_shape_ok(int64_t rows, int64_t cols) {
-  if (rows > cols || rows > SMALL_MAX_M) return false;
+// How a wide slice (rows <= cols) with at most 128 rows runs the whole
+// iteration in one clustered launch: with its columns resident in the
+// cluster's shared memory when they fit on 4 CTAs (cols <= 2048), streamed
+// through 4-CTA clusters otherwise (cols a multiple of 8, at most
+// STREAM_MAX_N: the 4-CTA clusters fill the device, where 8-CTA resident
+// clusters fit only 15 at once), resident on 8 CTAs for the remaining
+// cols <= 4096; larger slices take the GEMM path.  Shape only, so a slice's
+// result never depends on the batch.
+enum class SmallPath { kGemm, kResident, kStream };
+
+SmallPath small_path(int64_t rows, int64_t cols) {
+  if (rows > cols || rows > SMALL_MAX_M || rows < 1) return SmallPath::kGemm;
   const SmallSplit sp = small_split(cols);
-  return sp.C <= SMALL_MAX_CLUSTER && sp.w <= SMALL_MAX_W;
+  if (sp.C <= 4 && sp.w <= SMALL_MAX_W) return SmallPath::kResident;
+  if (cols % 8 == 0 && cols <= STREAM_MAX_N) return SmallPath::kStream;
+  if (sp.C <= SMALL_MAX_CLUSTER && sp.w <= SMALL_MAX_W) return SmallPath::kResident;
+  return SmallPath::kGemm;
 }
 
-// Slices whose short side is at most 128 and long side at most 8 * 512 run
-// the whole iteration in one clustered launch (ns_small.cuh); tall ones
+bool small_shape_ok(int64_t rows, int64_t cols) { return small_path(rows, cols) != SmallPath::kGemm; }
+
+// Cluster split of a fused slice: C CTAs of w columns (a multiple of 64).
+SmallSplit fused_split(int64_t rows, int64_t cols) {
+  if (small_path(rows, cols) == SmallPath::kStream)     // pairs of 64-column blocks per CTA
+    return SmallSplit{STREAM_CLUSTER, 128 * static_cast<int>(cdiv(cdiv(cols, 128), STREAM_CLUSTER))};
+  return small_split(cols);
+}
+
+// Slices whose short side is at most 128 run the whole iteration in one
+// clustered launch when small_path allows (ns_small.cuh); tall ones
 // (rows > cols) are transposed into the workspace first and back after.
 // The choice depends on the shape only, so a slice's result never depends
 // on the rest of the batch (tests can send them through the GEMM path,
@@ -786,7 +810,8 @@ muon_status launch_rows_sumsq(const muon_batch& b, int sms, cudaStream_t stream)
 
 muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const float* sumsq, int* err, bool gram,
                          float* row_partials, cudaStream_t stream) {
-  const SmallSplit sp = small_split(b.cols);
+  const bool streamed = small_path(b.rows, b.cols) == SmallPath::kStream;
+  const SmallSplit sp = fused_split(b.rows, b.cols);
   SmallParams P;
   std::memset(&P, 0, sizeof(P));
   P.row_ss = row_partials;
@@ -818,7 +843,7 @@ muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const floa
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(sp.C), static_cast<unsigned>(std::min(kMaxGridY, b.n - s0)), 1);
     cfg.blockDim = dim3(SMALL_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = SMALL_SMEM_BYTES;
+    cfg.dynamicSmemBytes = streamed ? STREAM_SMEM_BYTES : SMALL_SMEM_BYTES;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -829,7 +854,9 @@ muon_status launch_small(const muon_batch& b, const muon_hparams* hp, const floa
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 2 : 1;
-    if (cudaLaunchKernelEx(&cfg, gram ? ns_small_gram_kernel : ns_small_kernel, P) != cudaSuccess) {
+    auto kernel = streamed ? (gram ? ns_stream_gram_kernel : ns_stream_kernel)
+                           : (gram ? ns_small_gram_kernel : ns_small_kernel);
+    if (cudaLaunchKernelEx(&cfg, kernel, P) != cudaSuccess) {
       (void)cudaGetLastError();
       return MUON_CUDA_ERROR;
     }
@@ -858,7 +885,7 @@ muon_status run_small(const muon_batch& b, const NsBatchWs& w, uint8_t* ws, cons
     float* part = b.row_sumsq ? reinterpret_cast<float*>(ws + w.rs_off) : nullptr;
     muon_status st = launch_small(b, hp, sumsq, err, gram, part, stream);
     if (st != MUON_OK || part == nullptr) return st;
-    return launch_row_finalize(part, 2 * small_split(b.cols).C, b.rows, b.n, b.row_sumsq, sms, stream);
+    return launch_row_finalize(part, 2 * fused_split(b.rows, b.cols).C, b.rows, b.n, b.row_sumsq, sms, stream);
   }
   void* T = ws + w.t_off;
   const int64_t in_bs = b.n > 1 ? b.ns_in.batch_stride : b.rows * b.ns_in.ld;

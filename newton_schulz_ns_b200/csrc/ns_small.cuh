@@ -296,140 +296,94 @@ __device__ __forceinline__ void epi_columns(uint32_t taddr, int row, int half, i
   fence_proxy_async_smem();
 }
 
-template <bool GRAM>
-__device__ __forceinline__ void ns_small_body(const SmallParams& P) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem =
-      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* Xs = smem;
-  uint8_t* As = Xs + SMALL_X_BYTES;   // A, overwritten in place by B = b A + c A^2
-  uint8_t* Rv = As + SMALL_A_BYTES;   // partial rows pushed here by every CTA of the cluster
-  // [0] load, [1] MMA, [2] partial rows received (owner), [3] A received
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Rv + SMALL_RECV_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+// ---------------------------------------------------------------------------
+// Per-CTA state shared by the two clustered kernels (resident and streaming)
+// and the steps they have in common: the bounded wait on the MMA barrier and
+// the cluster exchange that turns each CTA's partial X_r X_r^T (fp32, TMEM
+// columns [0, 128)) into the full A = fA * X X^T in every CTA's As.
+// ---------------------------------------------------------------------------
+struct SmallCta {
+  int tid, warp, quarter, half, row;
+  uint32_t tlane, rank;
+  int C, m, m8, G, kb, Rm;
+  uint32_t tmem;
+  uint8_t* As;               // A (B = b A + c A^2 in place), K-major SW128, 128 x 128
+  uint8_t* Rv;               // receive slots; Gram: P and Q after the first exchange
+  uint32_t a0, rv0;
+  uint64_t* mma_bar;
+  uint64_t* recv_bar;        // owner: partial rows of its blocks received
+  uint64_t* a_bar;           // A's lower triangle received
+  uint32_t mph = 0;          // completed phases of the MMA barrier
+  uint32_t xphase = 0;       // completed exchanges
+  uint32_t recv_bytes = 0, a_bytes = 0;
+  bool ok = true;
+  bool pending = false;      // an MMA commit whose wait gave up
+  volatile int* abort_flag;
+  int* err;
+  unsigned long long timeout;
 
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int quarter = warp & 3;                     // TMEM lanes 32 quarter .. + 31
-  const int half = warp >> 2;                       // column half handled in the epilogues
-  const int row = quarter * 32 + (tid & 31);        // TMEM lane = row of the 128-row tiles
-  const uint32_t tlane = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t rank = cluster_ctarank();
-  const int C = static_cast<int>(gridDim.x);        // the cluster spans gridDim.x
-  const int slice = P.slice0 + static_cast<int>(blockIdx.y);
-  const int w = P.w;
-  const int nblk = w >> 6;
-  const int m8 = (P.m + 7) & ~7;                    // rows / columns of A that can be nonzero
   // Row blocks of 8 are dealt to the C CTAs in the order 0, G-1, 1, G-2, ...
   // in runs of kb, so that every CTA reduces about the same share of the
   // lower triangle; a receive slot holds the kb blocks of one owner.
-  const int G = m8 >> 3;
-  const int kb = (G + C - 1) / C;
-  const int Rm = kb * 8;                            // rows per receive slot (C * Rm <= 128)
-  auto fold = [G](int b) {
+  __device__ __forceinline__ int fold(int b) const {
     const int lo = min(b, G - 1 - b);
     return 2 * lo + (b > G - 1 - b ? 1 : 0);
-  };
-  auto unfold = [G](int p) { return (p & 1) ? G - 1 - (p >> 1) : (p >> 1); };
-  const uint32_t ncols = w > 256 ? 512u : 256u;     // P and A^2 take 256 columns; a X + B X takes w
-  // This thread's slot for its row's partial sum of squares of the output.
-  float* row_slot = P.row_ss == nullptr ? nullptr
-                                        : P.row_ss + (static_cast<long long>(slice) * (2 * C) + 2 * static_cast<int>(rank) + half) *
-                                                         P.m + row;
-
-  if (tid == 0) {
-    *abort_flag = 0;
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    mbar_init(&bars[2], 1);
-    mbar_init(&bars[3], 1);
-    fence_barrier_init();
-    tma_prefetch_desc(&P.map_in);
-    tma_prefetch_desc(&P.map_out);
   }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, ncols);
-    tmem_relinquish();
+  __device__ __forceinline__ int unfold(int p) const { return (p & 1) ? G - 1 - (p >> 1) : (p >> 1); }
+
+  __device__ __forceinline__ void init(int m_, volatile int* abort_, int* err_, unsigned long long timeout_) {
+    tid = threadIdx.x;
+    warp = tid >> 5;
+    quarter = warp & 3;                       // TMEM lanes 32 quarter .. + 31
+    half = warp >> 2;                         // column half handled in the epilogues
+    row = quarter * 32 + (tid & 31);          // TMEM lane = row of the 128-row tiles
+    tlane = static_cast<uint32_t>(quarter * 32) << 16;
+    rank = cluster_ctarank();
+    C = static_cast<int>(gridDim.x);          // the cluster spans gridDim.x
+    m = m_;
+    m8 = (m + 7) & ~7;                        // rows / columns of A that can be nonzero
+    G = m8 >> 3;
+    kb = (G + C - 1) / C;
+    Rm = kb * 8;                              // rows per receive slot (C * Rm <= 128)
+    abort_flag = abort_;
+    err = err_;
+    timeout = timeout_;
+    // Bytes one exchange delivers to this CTA: as an owner, the partial rows
+    // of its blocks from every CTA (16 bytes per 4 columns up to the
+    // diagonal); and A's lower triangle in 8 x 8 blocks from all owners.
+    recv_bytes = 0;
+    for (int lb = 0; lb < kb && static_cast<int>(rank) * kb + lb < G; ++lb) {
+      const int b = unfold(static_cast<int>(rank) * kb + lb);
+      for (int r8 = 0; r8 < 8; ++r8) recv_bytes += 16u * static_cast<uint32_t>(((8 * b + r8) >> 2) + 1);
+    }
+    recv_bytes *= static_cast<uint32_t>(C);
+    a_bytes = 64u * static_cast<uint32_t>(G * (G + 1));
   }
-  // A outside its m8 x m8 corner is never written by the exchange: zero it once.
-  for (int i = tid; i < SMALL_A_BYTES / 16; i += SMALL_THREADS)
-    reinterpret_cast<uint4*>(As)[i] = make_uint4(0u, 0u, 0u, 0u);
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
 
-  // Nothing above touched global memory: let the next kernel of the stream
-  // start its prologue, then wait for the previous one's results.
-  pdl_launch_dependents();
-  pdl_wait_prerequisites();
-
-  // ---- resident columns of the slice (zero outside it)
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bars[0], static_cast<uint32_t>(nblk * SMALL_BLK));
-    for (int j = 0; j < nblk; ++j)
-      tma_load_3d(Xs + j * SMALL_BLK, &P.map_in, &bars[0], static_cast<int>(rank) * w + 64 * j, 0, slice);
-  }
-  bool ok = __syncthreads_and(mbar_wait_bounded(&bars[0], 0, abort_flag, P.timeout_ns)) != 0;
-  if (!ok && tid == 0) small_record_error(P.err, abort_flag, kSmallErrLoad);
-  cluster_sync();             // every CTA of the cluster runs before its shared memory is addressed remotely
-
-  const float s = 1.0f / (sqrtf(P.sumsq[slice]) + P.eps);
-  uint32_t mph = 0;          // completed phases of the MMA barrier
-  bool pending = false;      // an MMA commit whose wait gave up
-  auto wait_mma = [&]() {
-    const bool got = mbar_wait_bounded(&bars[1], mph & 1u, abort_flag, P.timeout_ns);
+  // Waits (all threads) for the MMA barrier's next phase.
+  __device__ __forceinline__ bool wait_mma() {
+    const bool got = mbar_wait_bounded(mma_bar, mph & 1u, abort_flag, timeout);
     const bool all = __syncthreads_and(got) != 0;
     if (!all) {
       pending = true;
-      if (tid == 0) small_record_error(P.err, abort_flag, kSmallErrMma);
+      if (tid == 0) small_record_error(err, abort_flag, kSmallErrMma);
     }
     ++mph;
     return all;
-  };
-
-  const uint32_t idesc_sq = mma_idesc_f16(1, 0, 0, 128, 128);
-  const uint32_t rv0 = smem_u32(Rv);
-  const uint32_t a0 = smem_u32(As);
-
-  // Bytes one exchange delivers to this CTA: as an owner, the partial rows of
-  // its blocks from every CTA (16 bytes per 4 columns up to the diagonal);
-  // and A's lower triangle in 8 x 8 blocks from all owners.
-  uint32_t recv_bytes = 0;
-  for (int lb = 0; lb < kb && static_cast<int>(rank) * kb + lb < G; ++lb) {
-    const int b = unfold(static_cast<int>(rank) * kb + lb);
-    for (int r8 = 0; r8 < 8; ++r8) recv_bytes += 16u * static_cast<uint32_t>(((8 * b + r8) >> 2) + 1);
   }
-  recv_bytes *= static_cast<uint32_t>(C);
-  const uint32_t a_bytes = 64u * static_cast<uint32_t>(G * (G + 1));
-  uint32_t xphase = 0;        // completed exchanges (parity of the receive barriers)
 
-  // ---- A = fA * X X^T over the cluster, into every CTA's As (bf16; fp16 in
-  //      the Gram form), upper triangle mirrored.  Partial rows and A's rows
-  //      travel as st.async stores that complete bytes on the receiver's
-  //      mbarrier, so each CTA waits only for the data it needs, not for the
-  //      whole cluster.  (Every CTA's next exchange starts after it holds this
-  //      exchange's A, which needs every owner to have finished reading its
-  //      receive slots: the slots and barriers are never overwritten early.)
-  auto exchange = [&](float fA) {
+  // A = fA * (sum over the cluster of the partials in TMEM [0, 128)), into
+  // every CTA's As (bf16; fp16 in the Gram form), upper triangle mirrored.
+  // Partial rows and A's rows travel as st.async stores that complete bytes
+  // on the receiver's mbarrier, so each CTA waits only for the data it needs.
+  // (Every CTA's next exchange starts after it holds this exchange's A,
+  // which needs every owner to have finished reading its receive slots: the
+  // slots and barriers are never overwritten early.)
+  template <bool GRAM>
+  __device__ __forceinline__ void exchange(float fA) {
     if (ok && tid == 0) {
-      mbar_arrive_expect_tx(&bars[2], recv_bytes);
-      mbar_arrive_expect_tx(&bars[3], a_bytes);
-    }
-    // partial X_r X_r^T -> TMEM columns [0, 128)
-    if (ok) {
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t x0 = smem_u32(Xs);
-        for (int kk = 0; kk < w / 16; ++kk) {
-          const uint64_t d = smem_desc_sw128(x0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
-          tc_mma_f16(tmem, d, d, idesc_sq, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bars[1]);
-      }
-      ok = wait_mma();
+      mbar_arrive_expect_tx(recv_bar, recv_bytes);
+      mbar_arrive_expect_tx(a_bar, a_bytes);
     }
     // push row `row` of the partial, its lower triangle (4-column chunks up
     // to the diagonal) within columns [64 half, 64 half + 64), to the CTA
@@ -443,7 +397,7 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
         const int owner = p / kb;
         const int t = static_cast<int>(rank) * Rm + (p - owner * kb) * 8 + (row & 7);   // slot `rank`
         const int jn = min(16, (row >> 2) + 1 - half * 16);                             // chunks to send
-        const uint32_t rbar = mapa_shared(smem_u32(&bars[2]), static_cast<uint32_t>(owner));
+        const uint32_t rbar = mapa_shared(smem_u32(recv_bar), static_cast<uint32_t>(owner));
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           if (j < jn) {
@@ -459,19 +413,20 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
     // pushed to every CTA (the diagonal block's upper half carries unsent
     // entries; the mirror below replaces it)
     if (ok) {
-      const bool got = mbar_wait_cluster_bounded(&bars[2], xphase & 1u, abort_flag, P.timeout_ns);
+      const bool got = mbar_wait_cluster_bounded(recv_bar, xphase & 1u, abort_flag, timeout);
       ok = __syncthreads_and(got) != 0;
-      if (!ok && tid == 0) small_record_error(P.err, abort_flag, kSmallErrExchange);
+      if (!ok && tid == 0) small_record_error(err, abort_flag, kSmallErrExchange);
     }
     if (ok) {
       int items = 0;
-      for (int lb = 0; lb < kb && rank * kb + lb < G; ++lb) items += 8 * (unfold(rank * kb + lb) + 1);
+      for (int lb = 0; lb < kb && static_cast<int>(rank) * kb + lb < G; ++lb)
+        items += 8 * (unfold(static_cast<int>(rank) * kb + lb) + 1);
       for (int it = tid; it < items; it += SMALL_THREADS) {
-        int lb = 0, rest = it, b = unfold(rank * kb);
+        int lb = 0, rest = it, b = unfold(static_cast<int>(rank) * kb);
         while (rest >= 8 * (b + 1)) {
           rest -= 8 * (b + 1);
           ++lb;
-          b = unfold(rank * kb + lb);
+          b = unfold(static_cast<int>(rank) * kb + lb);
         }
         const int r8 = rest / (b + 1);
         const int g = rest - r8 * (b + 1);
@@ -498,29 +453,187 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
         for (int e = 0; e < 8; ++e) acc[e] *= fA;
         const uint4 pk = GRAM ? pack_f16x8(acc) : pack_bf16x8(acc);
         const uint32_t dst = a0 + sw128_chunk(8 * b + r8, g);
-        const uint32_t abar = smem_u32(&bars[3]);
+        const uint32_t abar = smem_u32(a_bar);
         for (int q = 0; q < C; ++q)
           st_async_v4(mapa_shared(dst, static_cast<uint32_t>(q)), pk, mapa_shared(abar, static_cast<uint32_t>(q)));
       }
     }
     // every CTA: wait for all of A's lower triangle
     if (ok) {
-      const bool got = mbar_wait_cluster_bounded(&bars[3], xphase & 1u, abort_flag, P.timeout_ns);
+      const bool got = mbar_wait_cluster_bounded(a_bar, xphase & 1u, abort_flag, timeout);
       ok = __syncthreads_and(got) != 0;
-      if (!ok && tid == 0) small_record_error(P.err, abort_flag, kSmallErrExchange);
+      if (!ok && tid == 0) small_record_error(err, abort_flag, kSmallErrExchange);
     }
     ++xphase;
-
     // upper triangle of A from the lower one (local; ends with the async-proxy fence)
     if (ok) mirror_upper(As, G, tid);
     __syncthreads();
-  };
+  }
 
-  // ---- (B, X) <- (Q, X) product on the resident columns: TMEM [0, w) = F X
-  //      with F a 128 x 128 bf16 K-major matrix in shared memory
-  auto left_product = [&](uint32_t f0) {
+  // A^2 -> TMEM columns [128, 256), then B = c A^2 + b A in place over A.
+  __device__ __forceinline__ void form_b(float cb, float cc) {
+    const uint32_t idesc_sq = mma_idesc_f16(1, 0, 0, 128, 128);
     if (ok) {
       if (tid == 0) {
+        fence_proxy_async_smem();
+        tc_fence_after();
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t d = smem_desc_sw128(a0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+          tc_mma_f16(tmem + 128, d, d, idesc_sq, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(mma_bar);
+      }
+      ok = wait_mma();
+    }
+    if (ok) {
+      tc_fence_after();
+      epi_square(tmem + tlane + 128u, row, half, m8, m, cc, cb, As, false, 0.0f, As, false);
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+};
+
+// The whole iteration, for a kernel whose columns `X` provide
+//   partial(c, k)          : TMEM [0, 128) = this CTA's X_r X_r^T before step k (the
+//                            input's at k = 0; the streaming kernel accumulates the later
+//                            ones during its passes, so it only does k = 0)
+//   apply(c, F, a, f, rss, next) : X_r <- f (F X_r + a X_r) with F a 128 x 128 bf16
+//                            K-major matrix in shared memory; rss (or null): this
+//                            thread's row sum of squares of the stored values; next:
+//                            a later exchange will need this X's partial
+// Standard form: per step exchange, B, apply.  Gram form: one exchange of
+// kappa s^2 X0 X0^T, the m x m iteration on P and Q (fp16, kappa-scaled A,
+// every CTA alike), restarts every P.restart steps (X <- xf Q X, A again
+// from an exchange, Q = I), and O = xf Q X.
+template <bool GRAM, class Cols>
+__device__ __forceinline__ void small_iterate(SmallCta& c, Cols& X, const SmallParams& P, float s, float* row_slot) {
+  if (!GRAM) {
+    for (int k = 0; k < P.steps; ++k) {
+      X.partial(c, k);
+      c.template exchange<false>((k == 0) ? s * s : 1.0f);
+      c.form_b(P.b[k], P.c[k]);
+      const bool last = k == P.steps - 1;
+      X.apply(c, c.a0, P.a[k], (k == 0) ? s : 1.0f, (last && P.row_ss != nullptr) ? row_slot : nullptr, !last);
+    }
+    return;
+  }
+  X.partial(c, 0);
+  c.template exchange<true>(P.kappa * (s * s));
+  uint8_t* Pb = c.Rv;                             // P (and, at a segment's start, the first Q)
+  uint8_t* Qb = c.Rv + SMALL_A_BYTES;             // Q
+  const int tid = c.tid;
+  auto clear_pq = [&]() {
+    for (int i = tid; i < 2 * SMALL_A_BYTES / 16; i += SMALL_THREADS)
+      reinterpret_cast<uint4*>(c.Rv)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+    __syncthreads();
+  };
+  clear_pq();
+  const uint32_t idesc_h = mma_idesc_f16(0, 0, 0, 128, 128);
+  const float kap = P.kappa;
+  const int R = P.restart;
+  auto restart_at = [&](int k) { return R > 0 && k > 0 && k < P.steps && k % R == 0; };
+  float xf = s;                                   // X's factor: s while X is the input
+  int seg_start = 0;
+  for (int k = 0; k < P.steps; ++k) {
+    if (restart_at(k)) {
+      // X <- xf Q X (Q in bf16)
+      X.apply(c, smem_u32(Qb), 0.0f, xf, nullptr, true);
+      xf = 1.0f;
+      X.partial(c, k);
+      tc_fence_before();
+      __syncthreads();
+      cluster_sync();       // no CTA still reads its Q when peers push partial rows over it
+      c.template exchange<true>(kap);
+      clear_pq();
+      seg_start = k;
+    }
+    const bool first = k == seg_start;
+    const bool end = k == P.steps - 1 || restart_at(k + 1);
+    uint8_t* Pd = first ? Qb : Pb;               // Q = P at a segment's start
+    // P = a I + (b / kappa) A + (c / kappa^2) A^2; bf16 when it is the segment's final Q
+    if (c.ok) {
+      if (tid == 0) issue_square(c.tmem, c.a0, c.a0, idesc_h, c.mma_bar);
+      c.ok = c.wait_mma();
+    }
+    if (c.ok) {
+      tc_fence_after();
+      epi_square(c.tmem + c.tlane, c.row, c.half, c.m8, c.m, P.c[k] / (kap * kap), P.b[k] / kap, c.As, true, P.a[k],
+                 Pd, !(first && end));
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (c.ok) mirror_upper(Pd, c.G, tid);
+    __syncthreads();
+    if (!first) {
+      // Q <- P Q, bf16 when the segment ends
+      if (c.ok) {
+        if (tid == 0) issue_square(c.tmem, smem_u32(Pb), smem_u32(Qb), idesc_h, c.mma_bar);
+        c.ok = c.wait_mma();
+      }
+      if (c.ok) {
+        tc_fence_after();
+        epi_square(c.tmem + c.tlane, c.row, c.half, c.m8, c.m, 1.0f, 0.0f, nullptr, false, 0.0f, Qb, !end);
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (c.ok) mirror_upper(Qb, c.G, tid);
+      __syncthreads();
+    }
+    if (!end) {
+      // R = P A, then A <- P R (fp16, each over A in place once its product is done)
+      for (int h = 0; h < 2; ++h) {
+        if (c.ok) {
+          if (tid == 0) issue_square(c.tmem, smem_u32(Pd), c.a0, idesc_h, c.mma_bar);
+          c.ok = c.wait_mma();
+        }
+        if (c.ok) {
+          tc_fence_after();
+          epi_square(c.tmem + c.tlane, c.row, c.half, c.m8, c.m, 1.0f, 0.0f, nullptr, false, 0.0f, c.As, true);
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (c.ok) mirror_upper(c.As, c.G, tid);
+        __syncthreads();
+      }
+    }
+  }
+  // O = xf Q X (Q in bf16)
+  X.apply(c, smem_u32(Qb), 0.0f, xf, P.row_ss != nullptr ? row_slot : nullptr, false);
+}
+
+// ---------------------------------------------------------------------------
+// Resident columns: CTA r keeps X[:, r w, (r+1) w) in shared memory (w <= 512).
+// ---------------------------------------------------------------------------
+struct ResidentCols {
+  uint8_t* Xs;
+  int w;
+
+  __device__ __forceinline__ void partial(SmallCta& c, int) {
+    if (!c.ok) return;
+    const uint32_t idesc_sq = mma_idesc_f16(1, 0, 0, 128, 128);
+    if (c.tid == 0) {
+      fence_proxy_async_smem();
+      tc_fence_after();
+      const uint32_t x0 = smem_u32(Xs);
+      for (int kk = 0; kk < w / 16; ++kk) {
+        const uint64_t d = smem_desc_sw128(x0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+        tc_mma_f16(c.tmem, d, d, idesc_sq, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(c.mma_bar);
+    }
+    c.ok = c.wait_mma();
+  }
+
+  __device__ __forceinline__ void apply(SmallCta& c, uint32_t f0, float a, float f, float* rss, bool) {
+    // F X_r -> TMEM [0, w)
+    if (c.ok) {
+      if (c.tid == 0) {
         fence_proxy_async_smem();
         tc_fence_after();
         const uint32_t x0 = smem_u32(Xs);
@@ -530,156 +643,98 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t ad = smem_desc_sw128(f0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = smem_desc_sw128(x0 + (nc >> 6) * SMALL_BLK + kk * 16 * 128, SMALL_BLK, 1024);
-            tc_mma_f16(tmem + static_cast<uint32_t>(nc), ad, bd, idesc, kk > 0 ? 1u : 0u);
+            tc_mma_f16(c.tmem + static_cast<uint32_t>(nc), ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
         }
-        tc_commit(&bars[1]);
+        tc_commit(c.mma_bar);
       }
-      ok = wait_mma();
+      c.ok = c.wait_mma();
     }
-  };
-
-  if (!GRAM) {
-    for (int k = 0; k < P.steps; ++k) {
-      const float ca = P.a[k], cb = P.b[k], cc = P.c[k];
-      exchange((k == 0) ? s * s : 1.0f);
-
-      // ---- A^2 -> TMEM columns [128, 256)
-      if (ok) {
-        if (tid == 0) {
-          fence_proxy_async_smem();
-          tc_fence_after();
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t d = smem_desc_sw128(a0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
-            tc_mma_f16(tmem + 128, d, d, idesc_sq, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&bars[1]);
-        }
-        ok = wait_mma();
-      }
-      // ---- B = c A^2 + b A, in place over A
-      if (ok) {
-        tc_fence_after();
-        epi_square(tmem + tlane + 128u, row, half, m8, P.m, cc, cb, As, false, 0.0f, As, false);
-        fence_proxy_async_smem();
-      }
-      tc_fence_before();
-      __syncthreads();
-
-      // ---- B X_r -> TMEM columns [0, w)
-      left_product(a0);
-      // ---- X <- f * (B X + a X), in place (the last step also leaves row sums of squares)
-      if (ok) {
-        tc_fence_after();
-        float* rss = (P.row_ss != nullptr && k == P.steps - 1) ? row_slot : nullptr;
-        epi_columns(tmem + tlane, row, half, w, m8, ca, (k == 0) ? s : 1.0f, Xs, rss, P.m);
-      }
-      tc_fence_before();
-      __syncthreads();
-    }
-  } else {
-    // ---- G = kappa s^2 X0 X0^T, then the m x m iteration (fp16, kappa-scaled
-    //      A), every CTA of the cluster alike.  Restarts (every P.restart
-    //      iterations): X <- f Q X on the resident columns, A = kappa X X^T
-    //      over the cluster again, Q = I.
-    exchange(P.kappa * (s * s));
-    uint8_t* Pb = Rv;                               // P (and, at a segment's start, the first Q)
-    uint8_t* Qb = Rv + SMALL_A_BYTES;               // Q
-    auto clear_pq = [&]() {
-      for (int i = tid; i < 2 * SMALL_A_BYTES / 16; i += SMALL_THREADS)
-        reinterpret_cast<uint4*>(Rv)[i] = make_uint4(0u, 0u, 0u, 0u);
-      fence_proxy_async_smem();
-      __syncthreads();
-    };
-    clear_pq();
-    const uint32_t idesc_h = mma_idesc_f16(0, 0, 0, 128, 128);
-    const float kap = P.kappa;
-    const int R = P.restart;
-    auto restart_at = [&](int k) { return R > 0 && k > 0 && k < P.steps && k % R == 0; };
-    float xf = s;                                   // X's factor: s while X is the input
-    int seg_start = 0;
-    for (int k = 0; k < P.steps; ++k) {
-      if (restart_at(k)) {
-        // X <- xf Q X (Q in bf16), in place
-        left_product(smem_u32(Qb));
-        if (ok) {
-          tc_fence_after();
-          epi_columns(tmem + tlane, row, half, w, m8, 0.0f, xf, Xs);
-        }
-        xf = 1.0f;
-        tc_fence_before();
-        __syncthreads();
-        cluster_sync();       // no CTA still reads its Q when peers push partial rows over it
-        exchange(kap);
-        clear_pq();
-        seg_start = k;
-      }
-      const bool first = k == seg_start;
-      const bool end = k == P.steps - 1 || restart_at(k + 1);
-      uint8_t* Pd = first ? Qb : Pb;               // Q = P at a segment's start
-      // P = a I + (b / kappa) A + (c / kappa^2) A^2; bf16 when it is the segment's final Q
-      if (ok) {
-        if (tid == 0) issue_square(tmem, a0, a0, idesc_h, &bars[1]);
-        ok = wait_mma();
-      }
-      if (ok) {
-        tc_fence_after();
-        epi_square(tmem + tlane, row, half, m8, P.m, P.c[k] / (kap * kap), P.b[k] / kap, As, true, P.a[k], Pd,
-                   !(first && end));
-        fence_proxy_async_smem();
-      }
-      tc_fence_before();
-      __syncthreads();
-      if (ok) mirror_upper(Pd, G, tid);
-      __syncthreads();
-      if (!first) {
-        // Q <- P Q, bf16 when the segment ends
-        if (ok) {
-          if (tid == 0) issue_square(tmem, smem_u32(Pb), smem_u32(Qb), idesc_h, &bars[1]);
-          ok = wait_mma();
-        }
-        if (ok) {
-          tc_fence_after();
-          epi_square(tmem + tlane, row, half, m8, P.m, 1.0f, 0.0f, nullptr, false, 0.0f, Qb, !end);
-          fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (ok) mirror_upper(Qb, G, tid);
-        __syncthreads();
-      }
-      if (!end) {
-        // R = P A, then A <- P R (fp16, each over A in place once its product is done)
-        for (int h = 0; h < 2; ++h) {
-          if (ok) {
-            if (tid == 0) issue_square(tmem, smem_u32(Pd), a0, idesc_h, &bars[1]);
-            ok = wait_mma();
-          }
-          if (ok) {
-            tc_fence_after();
-            epi_square(tmem + tlane, row, half, m8, P.m, 1.0f, 0.0f, nullptr, false, 0.0f, As, true);
-            fence_proxy_async_smem();
-          }
-          tc_fence_before();
-          __syncthreads();
-          if (ok) mirror_upper(As, G, tid);
-          __syncthreads();
-        }
-      }
-    }
-    // ---- O = xf Q X on the resident columns (Q in bf16)
-    left_product(smem_u32(Qb));
-    if (ok) {
+    // X <- f (F X + a X), in place
+    if (c.ok) {
       tc_fence_after();
-      epi_columns(tmem + tlane, row, half, w, m8, 0.0f, xf, Xs, P.row_ss != nullptr ? row_slot : nullptr, P.m);
+      epi_columns(c.tmem + c.tlane, c.row, c.half, w, c.m8, a, f, Xs, rss, c.m);
     }
     tc_fence_before();
     __syncthreads();
   }
+};
+
+template <bool GRAM>
+__device__ __forceinline__ void ns_small_body(const SmallParams& P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* Xs = smem;
+  uint8_t* As = Xs + SMALL_X_BYTES;   // A, overwritten in place by B = b A + c A^2
+  uint8_t* Rv = As + SMALL_A_BYTES;   // partial rows pushed here by every CTA of the cluster
+  // [0] load, [1] MMA, [2] partial rows received (owner), [3] A received
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Rv + SMALL_RECV_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  SmallCta c;
+  c.init(P.m, abort_flag, P.err, P.timeout_ns);
+  const int tid = c.tid;
+  const int slice = P.slice0 + static_cast<int>(blockIdx.y);
+  const int w = P.w;
+  const int nblk = w >> 6;
+  const uint32_t ncols = w > 256 ? 512u : 256u;     // P and A^2 take 256 columns; a X + B X takes w
+  // This thread's slot for its row's partial sum of squares of the output.
+  float* row_slot = P.row_ss == nullptr
+                        ? nullptr
+                        : P.row_ss + (static_cast<long long>(slice) * (2 * c.C) + 2 * static_cast<int>(c.rank) + c.half) *
+                                         P.m + c.row;
+
+  if (tid == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&P.map_in);
+    tma_prefetch_desc(&P.map_out);
+  }
+  if (c.warp == 0) {
+    tmem_alloc(tmem_slot, ncols);
+    tmem_relinquish();
+  }
+  // A outside its m8 x m8 corner is never written by the exchange: zero it once.
+  for (int i = tid; i < SMALL_A_BYTES / 16; i += SMALL_THREADS)
+    reinterpret_cast<uint4*>(As)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  c.tmem = *tmem_slot;
+  c.As = As;
+  c.Rv = Rv;
+  c.a0 = smem_u32(As);
+  c.rv0 = smem_u32(Rv);
+  c.mma_bar = &bars[1];
+  c.recv_bar = &bars[2];
+  c.a_bar = &bars[3];
+
+  // Nothing above touched global memory: let the next kernel of the stream
+  // start its prologue, then wait for the previous one's results.
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
+
+  // ---- resident columns of the slice (zero outside it)
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], static_cast<uint32_t>(nblk * SMALL_BLK));
+    for (int j = 0; j < nblk; ++j)
+      tma_load_3d(Xs + j * SMALL_BLK, &P.map_in, &bars[0], static_cast<int>(c.rank) * w + 64 * j, 0, slice);
+  }
+  c.ok = __syncthreads_and(mbar_wait_bounded(&bars[0], 0, abort_flag, P.timeout_ns)) != 0;
+  if (!c.ok && tid == 0) small_record_error(P.err, abort_flag, kSmallErrLoad);
+  cluster_sync();             // every CTA of the cluster runs before its shared memory is addressed remotely
+
+  const float s = 1.0f / (sqrtf(P.sumsq[slice]) + P.eps);
+  ResidentCols X{Xs, w};
+  small_iterate<GRAM>(c, X, P, s, row_slot);
 
   // ---- resident columns -> ns_out (rows < m, columns < n)
-  if (ok) {
-    const int col_base = static_cast<int>(rank) * w;
+  if (c.ok) {
+    const int col_base = static_cast<int>(c.rank) * w;
     if (P.tma_store) {
       if (tid == 0) {
         for (int j = 0; j < nblk && col_base + 64 * j < P.n; ++j)
@@ -709,14 +764,14 @@ __device__ __forceinline__ void ns_small_body(const SmallParams& P) {
 
   // A commit whose wait gave up may still be running: give it one more
   // bounded wait before its TMEM is released.
-  if (pending && tid == 0) {
+  if (c.pending && tid == 0) {
     volatile int never = 0;
-    (void)mbar_wait_bounded(&bars[1], (mph - 1u) & 1u, &never, P.timeout_ns);
+    (void)mbar_wait_bounded(&bars[1], (c.mph - 1u) & 1u, &never, P.timeout_ns);
   }
   tc_fence_before();
   __syncthreads();
   cluster_sync();             // no CTA leaves while a peer may still address its shared memory
-  if (warp == 0) tmem_dealloc(tmem, ncols);
+  if (c.warp == 0) tmem_dealloc(c.tmem, ncols);
 }
 
 __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid_constant__ SmallParams P) {
@@ -725,6 +780,258 @@ __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_kernel(const __grid
 
 __global__ void __launch_bounds__(SMALL_THREADS, 1) ns_small_gram_kernel(const __grid_constant__ SmallParams P) {
   ns_small_body<true>(P);
+}
+
+// ---------------------------------------------------------------------------
+// Streaming columns: for slices too long to keep resident on a 4-CTA cluster
+// (n > 2048), CTA r owns columns [r w, (r+1) w) of X (w = 128 * npair, any
+// length) in global memory (ns_out after the first pass; the slice's 1 MB at
+// 128 x 4096 stays in L2) and streams them through shared memory in pairs of
+// 64-column blocks every step.  One pass computes, per pair p,
+//   F X_p on the tensor core (TMEM [256, 384)),
+//   X_p' = f (F X_p + a X_p) (bf16, staged in shared memory),
+//   the next exchange's partial += X_p' X_p'^T (TMEM [0, 128)),
+//   and stores X_p' back by TMA;
+// a first pass over the input forms its partial only.  With 4-CTA clusters
+// the B200 runs 37 clusters at once, so a 32-head batch takes one wave where
+// the resident kernel's 8-CTA clusters take three.
+// ---------------------------------------------------------------------------
+constexpr int STREAM_PAIR = 2 * SMALL_BLK;          // two 64-column blocks [128 rows][64], 32 KB
+constexpr int STREAM_STAGES = 2;                   // block pairs in flight
+constexpr int STREAM_CLUSTER = 4;
+constexpr int STREAM_MAX_N = 16384;
+constexpr int STREAM_SMEM_BYTES = 1024 + SMALL_A_BYTES + SMALL_RECV_BYTES + STREAM_STAGES * STREAM_PAIR +
+                                  2 * STREAM_PAIR + 128;
+
+struct StreamCols {
+  const CUtensorMap* map_in;
+  const CUtensorMap* map_out;
+  uint8_t* ring;             // STREAM_STAGES block pairs, SW128
+  uint8_t* Xo;               // two block pairs: X_p' (MMA operand and TMA store source)
+  uint64_t* ld_bar;          // one per ring stage
+  int npair, col0, slice, n;
+  uint32_t loads = 0;        // pairs loaded so far over all passes: stage g % STAGES, parity (g / STAGES) & 1
+  bool src_out = false;      // X lives in ns_out (after the first pass that stored it)
+
+  __device__ __forceinline__ void issue_load(const CUtensorMap* src, int p, uint32_t g) {
+    const int st = static_cast<int>(g % STREAM_STAGES);
+    uint8_t* dst = ring + st * STREAM_PAIR;
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(&ld_bar[st], static_cast<uint32_t>(STREAM_PAIR));
+    tma_load_3d(dst, src, &ld_bar[st], col0 + 128 * p, 0, slice);
+    tma_load_3d(dst + SMALL_BLK, src, &ld_bar[st], col0 + 128 * p + 64, 0, slice);
+  }
+
+  __device__ __forceinline__ bool wait_load(SmallCta& c, uint32_t g) {
+    const bool got =
+        mbar_wait_bounded(&ld_bar[g % STREAM_STAGES], (g / STREAM_STAGES) & 1u, c.abort_flag, c.timeout);
+    const bool all = __syncthreads_and(got) != 0;
+    if (!all && c.tid == 0) small_record_error(c.err, c.abort_flag, kSmallErrLoad);
+    return all;
+  }
+
+  // One pass over this CTA's block pairs.  product = false: partial X X^T of
+  // the input only.  product = true: X <- f (F X + a X) pair by pair, stored
+  // to ns_out, with the next partial when `next` and row sums when rss != null.
+  __device__ __forceinline__ void pass(SmallCta& c, bool product, uint32_t f0, float a, float f, float* rss,
+                                       bool next) {
+    const CUtensorMap* src = src_out ? map_out : map_in;
+    const uint32_t base = loads;
+    const uint32_t idesc_sq = mma_idesc_f16(1, 0, 0, 128, 128);
+    const uint32_t idesc_fx = mma_idesc_f16(1, 0, 1, 128, 128);
+    if (c.ok && c.tid == 0)
+      for (int p = 0; p < min(STREAM_STAGES, npair); ++p) issue_load(src, p, base + static_cast<uint32_t>(p));
+    float ss = 0.0f;
+    for (int p = 0; p < npair; ++p) {
+      const uint32_t g = base + static_cast<uint32_t>(p);
+      if (c.ok) c.ok = wait_load(c, g);
+      uint8_t* xp = ring + (g % STREAM_STAGES) * STREAM_PAIR;
+      const uint32_t xp0 = smem_u32(xp);
+      if (!product) {
+        if (c.ok) {
+          if (c.tid == 0) {
+            tc_fence_after();
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t d = smem_desc_sw128(xp0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+              tc_mma_f16(c.tmem, d, d, idesc_sq, (p | kk) != 0 ? 1u : 0u);
+            }
+            tc_commit(c.mma_bar);
+          }
+          c.ok = c.wait_mma();
+        }
+      } else {
+        uint8_t* xo = Xo + (p & 1) * STREAM_PAIR;
+        // F X_p -> TMEM [256, 384); its commit also covers the previous pair's partial product
+        if (c.ok) {
+          if (c.tid == 0) {
+            bulk_wait_group_read<1>();              // the stores from xo two pairs ago have read it
+            tc_fence_after();
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t ad = smem_desc_sw128(f0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(xp0 + kk * 16 * 128, SMALL_BLK, 1024);
+              tc_mma_f16(c.tmem + 256u, ad, bd, idesc_fx, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(c.mma_bar);
+          }
+          c.ok = c.wait_mma();
+        }
+        // X_p' = f (F X_p + a X_p): row `row`, columns [64 half, 64 half + 64) of the pair
+        if (c.ok) {
+          tc_fence_after();
+          uint32_t v[64];
+          tmem_ld_64(c.tmem + c.tlane + 256u + static_cast<uint32_t>(c.half * 64), v);
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            const uint32_t off = sw128_chunk(c.row, c.half * 8 + h);
+            float xf[8], o[8];
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(xp + off), xf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[e] = (__uint_as_float(v[h * 8 + e]) + a * xf[e]) * f;
+            const uint4 pk = pack_bf16x8(o);
+            *reinterpret_cast<uint4*>(xo + off) = pk;
+            if (rss != nullptr) {
+              float st[8];
+              unpack_bf16x8(pk, st);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) ss += st[e] * st[e];
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (c.ok && c.tid == 0) {
+          if (next) {
+            tc_fence_after();
+            const uint32_t xo0 = smem_u32(xo);
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t d = smem_desc_sw128(xo0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+              tc_mma_f16(c.tmem, d, d, idesc_sq, (p | kk) != 0 ? 1u : 0u);
+            }
+          }
+          for (int b = 0; b < 2; ++b)
+            if (col0 + 128 * p + 64 * b < n) tma_store_3d(map_out, xo + b * SMALL_BLK, col0 + 128 * p + 64 * b, 0, slice);
+          bulk_commit_group();
+        }
+      }
+      // The stage's pair has been read by its product and by the epilogue
+      // (before the barrier above): load the pair STAGES ahead into it.
+      if (c.ok && c.tid == 0 && p + STREAM_STAGES < npair)
+        issue_load(src, p + STREAM_STAGES, g + static_cast<uint32_t>(STREAM_STAGES));
+    }
+    loads = base + static_cast<uint32_t>(npair);
+    if (product) {
+      // the last partial product, and every store, complete before the next pass or exchange
+      if (c.ok) {
+        if (c.tid == 0) tc_commit(c.mma_bar);
+        c.ok = c.wait_mma();
+      }
+      if (c.tid == 0) bulk_wait_group_all();
+      src_out = true;
+      if (rss != nullptr && c.row < c.m) *rss = ss;
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  __device__ __forceinline__ void partial(SmallCta& c, int k) {
+    if (k == 0) pass(c, false, 0u, 0.0f, 1.0f, nullptr, false);   // later partials come from the passes
+  }
+
+  __device__ __forceinline__ void apply(SmallCta& c, uint32_t f0, float a, float f, float* rss, bool next) {
+    pass(c, true, f0, a, f, rss, next);
+  }
+};
+
+template <bool GRAM>
+__device__ __forceinline__ void ns_stream_body(const SmallParams& P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* As = smem;
+  uint8_t* Rv = As + SMALL_A_BYTES;
+  uint8_t* ring = Rv + SMALL_RECV_BYTES;
+  uint8_t* Xo = ring + STREAM_STAGES * STREAM_PAIR;
+  // [0, STAGES) ring loads, then MMA, partial rows received (owner), A received
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Xo + 2 * STREAM_PAIR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + STREAM_STAGES + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  SmallCta c;
+  c.init(P.m, abort_flag, P.err, P.timeout_ns);
+  const int tid = c.tid;
+  const int slice = P.slice0 + static_cast<int>(blockIdx.y);
+  constexpr uint32_t ncols = 512;                  // partial [0,128), products [128,256), F X_p [256,384)
+  float* row_slot = P.row_ss == nullptr
+                        ? nullptr
+                        : P.row_ss + (static_cast<long long>(slice) * (2 * c.C) + 2 * static_cast<int>(c.rank) + c.half) *
+                                         P.m + c.row;
+
+  if (tid == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < STREAM_STAGES + 3; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&P.map_in);
+    tma_prefetch_desc(&P.map_out);
+  }
+  if (c.warp == 0) {
+    tmem_alloc(tmem_slot, ncols);
+    tmem_relinquish();
+  }
+  // A outside its m8 x m8 corner is never written by the exchange: zero it once.
+  for (int i = tid; i < SMALL_A_BYTES / 16; i += SMALL_THREADS)
+    reinterpret_cast<uint4*>(As)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  c.tmem = *tmem_slot;
+  c.As = As;
+  c.Rv = Rv;
+  c.a0 = smem_u32(As);
+  c.rv0 = smem_u32(Rv);
+  c.mma_bar = &bars[STREAM_STAGES];
+  c.recv_bar = &bars[STREAM_STAGES + 1];
+  c.a_bar = &bars[STREAM_STAGES + 2];
+  cluster_sync();             // every CTA's barriers exist before peers address them
+
+  // Nothing above touched global memory: let the next kernel of the stream
+  // start its prologue, then wait for the previous one's results.
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
+
+  const float s = 1.0f / (sqrtf(P.sumsq[slice]) + P.eps);
+  StreamCols X;
+  X.map_in = &P.map_in;
+  X.map_out = &P.map_out;
+  X.ring = ring;
+  X.Xo = Xo;
+  X.ld_bar = bars;
+  X.npair = P.w >> 7;
+  X.col0 = static_cast<int>(c.rank) * P.w;
+  X.slice = slice;
+  X.n = P.n;
+  small_iterate<GRAM>(c, X, P, s, row_slot);
+
+  // A product whose wait gave up may still be running: one more commit tracks
+  // every product issued so far; give it a bounded wait before TMEM is released.
+  if (c.pending && tid == 0) {
+    volatile int never = 0;
+    tc_commit(c.mma_bar);
+    (void)mbar_wait_bounded(c.mma_bar, c.mph & 1u, &never, P.timeout_ns);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();             // no CTA leaves while a peer may still address its shared memory
+  if (c.warp == 0) tmem_dealloc(c.tmem, ncols);
+}
+
+__global__ void __launch_bounds__(SMALL_THREADS, 1) ns_stream_kernel(const __grid_constant__ SmallParams P) {
+  ns_stream_body<false>(P);
+}
+
+__global__ void __launch_bounds__(SMALL_THREADS, 1) ns_stream_gram_kernel(const __grid_constant__ SmallParams P) {
+  ns_stream_body<true>(P);
 }
 
 }  // namespace muon

@@ -218,10 +218,10 @@ def test_polar_express_schedule_safety_and_arguments(mn):
 
 
 def test_workspace_holds_the_transposed_copy_of_tall_small_slices(mn):
-    # A tall slice with a short side <= 128 and a long side <= 4096 runs the
-    # fused kernel on a transposed copy [n][cols][rows] (rows rounded to 64)
-    # in the workspace of both Newton-Schulz forms; a wide slice, and a tall
-    # one outside those limits, needs none.
+    # A tall slice with a short side <= 128 that a fused kernel takes runs it
+    # on a transposed copy [n][cols][rows] (rows rounded to 64) in the
+    # workspace of both Newton-Schulz forms; a wide slice, and a tall one
+    # outside those limits, needs none.
     from newton_schulz_ns_b200 import _capi
 
     def size(b, which):
@@ -244,11 +244,16 @@ def test_workspace_holds_the_transposed_copy_of_tall_small_slices(mn):
             base_bufs = 5 * mm + xbuf
         assert tall >= base_bufs + copy
         assert tall - copy < base_bufs + base + 5 * 256 + 8 * n * ((r * c + 8191) // 8192) + 64
-    # wide twin and a tall slice with a long side past 4096: no copy
+    # wide twin, and tall slices the fused kernels do not take (long side past
+    # 4096 and not a multiple of 8, or past 16384): no copy
     assert size(_fake_batch(mn, n, c, r), 1) < size(_fake_batch(mn, n, r, c), 1)
-    t_big = size(_fake_batch(mn, 1, 5000, 96), 2)
-    assert t_big < (5 * ((96 + 63) // 64 * 64) * 96 * 2 + 5000 * 128 * 2 + 256 * 8 + 4 * ((5000 * 96 + 8191) // 8192)
-                    + 4096)
+    for rows in (5001, 16392):
+        t_big = size(_fake_batch(mn, 1, rows, 96), 2)
+        assert t_big < (5 * ((96 + 63) // 64 * 64) * 96 * 2 + rows * 128 * 2 + 256 * 8
+                        + 4 * ((rows * 96 + 8191) // 8192) + 4096)
+    # a tall slice the streaming kernel takes (long side a multiple of 8, past 4096) gets the copy
+    t_stream = size(_fake_batch(mn, 1, 5000, 96), 2)
+    assert t_stream >= 96 * ((5000 + 63) // 64 * 64) * 2
 
 
 # ----------------------------------------------------------------- update scale (host code)

@@ -1,17 +1,21 @@
 """Parity of the fused small-side Newton-Schulz kernel with the fp64 oracle.
 
-Slices with rows <= cols, rows <= 128 and cols <= 4096 (the per-head
-[32, 128, 4096] batch, the conv megabatch [16, 64, 576]) run the whole
-iteration in one clustered launch: each CTA keeps a column block of X in
-shared memory and the cluster sums X X^T over distributed shared memory.
-Both forms: the standard one exchanges X X^T at every step; the Gram one
-exchanges X0 X0^T once and iterates on the m x m side in every CTA.  Tall
-slices (rows > cols, cols <= 128) take the same kernel on a transposed copy.
-The shapes below cover every cluster split the planner picks (1 to 8 CTAs,
-64 to 512 columns each), ragged last blocks, CTAs that hold only padding,
-and short sides from 1 to 128.  Bars: 3e-2 relative Frobenius error against
-the oracle per slice; bitwise batch invariance and run-to-run determinism;
-nothing written outside the slice.
+Slices with rows <= cols and rows <= 128 (the per-head [32, 128, 4096]
+batch, the conv megabatch [16, 64, 576]) run the whole iteration in one
+clustered launch and the cluster sums X X^T over distributed shared memory.
+Up to 2048 columns each CTA keeps its column block of X resident in shared
+memory; longer slices (columns a multiple of 8, up to 16384) stream their
+column blocks through 4-CTA clusters from L2 at every step; the remaining
+ones up to 4096 columns stay resident on 8 CTAs.  Both forms: the standard
+one exchanges X X^T at every step; the Gram one exchanges X0 X0^T once (and
+at each restart) and iterates on the m x m side in every CTA.  Tall slices
+(rows > cols, cols <= 128) take the same kernels on a transposed copy.  The
+shapes below cover every cluster split the planner picks (1 to 8 resident
+CTAs of 64 to 512 columns, 4 streaming CTAs of 768 to 4096 columns), ragged
+last blocks, CTAs that hold only padding, and short sides from 1 to 128.
+Bars: 3e-2 relative Frobenius error against the oracle per slice; bitwise
+batch invariance and run-to-run determinism; nothing written outside the
+slice.
 """
 import numpy as np
 import pytest
@@ -68,25 +72,34 @@ def _ns(mn, U, hp=None, fused=True, variant="standard"):
     return base, out, launches
 
 
-# (rows, cols): cluster split (CTAs x columns each) the planner picks
+# (rows, cols): cluster split (CTAs x columns each) the planner picks.
+# Columns resident in shared memory when they fit on 4 CTAs (cols <= 2048);
+# longer slices (cols a multiple of 8, up to 16384) stream their columns
+# through 4-CTA clusters in 64-column blocks; the rest up to 4096 columns
+# stay resident on 8 CTAs.
 SHAPES = [
-    (64, 576),     # conv megabatch slice: 4 x 192, the last CTA partly padding
-    (128, 4096),   # attention head: 8 x 512
-    (128, 2000),   # 4 x 512, ragged last block
-    (100, 1000),   # 4 x 256, ragged
-    (128, 128),    # 2 x 64
-    (3, 5),        # 1 x 64, element stores (cols not a multiple of 8)
-    (1, 4096),     # one row: each CTA owns one row of A
-    (128, 4040),   # 8 x 512, last CTA mostly padding
-    (65, 3000),    # 8 x 384, 9 rows of A per CTA
-    (33, 200),     # 4 x 64, 10 rows of A per CTA, one CTA only padding
-    (50, 1001),    # 4 x 256, 14 rows of A per CTA, element stores
+    (64, 576),     # conv megabatch slice: resident 4 x 192, the last CTA partly padding
+    (128, 4096),   # attention head: streamed 4 x 1024 (16 blocks per CTA)
+    (128, 2000),   # resident 4 x 512, ragged last block
+    (100, 1000),   # resident 4 x 256, ragged
+    (128, 128),    # resident 2 x 64
+    (3, 5),        # resident 1 x 64, element stores (cols not a multiple of 8)
+    (1, 4096),     # streamed; one row: one owner, three CTAs own no block of A
+    (128, 4040),   # streamed 4 x 1024, last CTA's last blocks partly padding
+    (65, 3000),    # streamed 4 x 768, 9 row blocks of A
+    (33, 200),     # resident 4 x 64, 10 rows of A per CTA, one CTA only padding
+    (50, 1001),    # resident 4 x 256, 14 rows of A per CTA, element stores
+    (50, 4001),    # resident 8 x 512 (cols not a multiple of 8: not streamed)
+    (128, 8192),   # streamed 4 x 2048 (past the resident limit)
+    (96, 16384),   # streamed 4 x 4096, the longest fused slice
+    (17, 5000),    # streamed 4 x 1280, ragged
     # tall slices: transposed into the workspace, fused, transposed back
     (576, 64),     # a channel-expanding conv slice
-    (4096, 128),
+    (4096, 128),   # streamed on the transposed copy
     (1000, 100),
     (5, 3),
-    (3001, 65),    # element stores on the transposed copy
+    (3001, 65),    # resident 8 x 384, element stores on the transposed copy
+    (12288, 80),   # streamed on the transposed copy
 ]
 
 
