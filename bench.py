@@ -63,6 +63,10 @@ def parse():
                          "minimax schedule for singular values in [--pe-lower, 1]")
     ap.add_argument("--pe-lower", type=float, default=1e-3)
     ap.add_argument("--pe-safety", type=float, default=1.01)
+    ap.add_argument("--schedule", choices=["serial", "two-stream"], default="serial",
+                    help="serial: one call per stage over every shape; two-stream: per-shape calls, each shape's "
+                         "Newton-Schulz on the main stream while the momentum of the next shape and the update of "
+                         "the previous one run on a second stream (TwoStreamStep)")
     ap.add_argument("--graph", choices=["on", "off"], default="on",
                     help="on: the timed steps replay a CUDA graph of one whole step (the per-stage split "
                          "comes from eager steps after it); off: eager calls")
@@ -409,8 +413,14 @@ def run_ours(args, wl, variant, rank, world, local_rank):
     ns_flop = sum(b.n * ns_flops(b.rows, b.cols, variant, wl.ns_steps) for b in groups)
     slices = sum(b.n for b in groups)
 
+    two_stream = mn.TwoStreamStep(groups, hp, variant, wl.normuon, AUTO_GRAM_RATIO, dev) \
+        if args.schedule == "two-stream" else None
+
     def step(ev=None):
         st = torch.cuda.current_stream()            # the capture stream while a graph is recorded
+        if ev is None and two_stream is not None:
+            two_stream(st)
+            return
         if ev is not None:
             ev[0].record(st)
         mn.muon_momentum_norm(groups, hp, ws, st)
@@ -431,6 +441,8 @@ def run_ours(args, wl, variant, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     assert mn.workspace_error(ws) == 0, "device-side wait timed out"
+    if two_stream is not None:
+        assert two_stream.workspace_errors() == 0, "device-side wait timed out"
 
     # ---- device-resident timing
     gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[local_rank] \
@@ -561,6 +573,10 @@ def run_ours(args, wl, variant, rank, world, local_rank):
         "config": dict(workload_config(args, wl, variant), parallelism=f"replicas x{world} (no exchange)"),
         "launch": ("CUDA graph of one whole step, replayed for each timed step" if args.graph == "on"
                    else "eager calls"),
+        "schedule": ("two streams: per-shape calls, each shape's Newton-Schulz overlapping the next shape's "
+                     "momentum and the previous shape's NorMuon + update (TwoStreamStep); the per-stage split "
+                     "in ms_breakdown comes from serial eager steps" if two_stream is not None
+                     else "serial: one call per stage over every shape"),
         "pct_bf16_peak": round(100 * value / world / peak_s, 2),
         "pct_bf16_peak_burst": round(100 * value / world / peak_b, 2),
         "matrices_per_s": round(world * slices * args.steps / sec, 2),

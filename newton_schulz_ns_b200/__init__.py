@@ -21,7 +21,8 @@ from ._capi import MUON_BF16, MUON_F16, MUON_F32, MuonError  # noqa: F401
 __all__ = ["Batch", "Hparams", "muon_workspace_size", "muon_momentum_norm", "muon_ns_batched",
            "muon_gram_ns_batched", "normuon_update", "workspace_error", "testing_gemm", "update_scale",
            "ns_flops", "version", "kernel_launches", "muon_momentum_norm_noalloc", "muon_ns_auto_batched",
-           "polar_express_schedule", "allocate_workspace", "testing_options", "MuonError", "LIB_PATH"]
+           "polar_express_schedule", "allocate_workspace", "testing_options", "TwoStreamStep", "MuonError",
+           "LIB_PATH"]
 
 LIB_PATH = _capi.LIB_PATH
 
@@ -221,9 +222,14 @@ def muon_workspace_size(batches: Sequence[Batch], which: int = -1) -> int:
 
 
 def allocate_workspace(batches: Sequence[Batch], which: int = -1, device=None) -> torch.Tensor:
-    """A uint8 CUDA tensor of muon_workspace_size bytes (torch's allocator aligns it to 512 B)."""
-    return torch.empty(max(256, muon_workspace_size(batches, which)), dtype=torch.uint8,
-                       device=device or "cuda")
+    """A uint8 CUDA tensor of muon_workspace_size bytes (torch's allocator aligns it to 512 B).
+
+    Its error word (the first 256 bytes) starts cleared, so workspace_error
+    reads 0 for a workspace that no Newton-Schulz call has used yet.
+    """
+    ws = torch.empty(max(256, muon_workspace_size(batches, which)), dtype=torch.uint8, device=device or "cuda")
+    ws[:256].zero_()
+    return ws
 
 
 def muon_momentum_norm(batches: Sequence[Batch], hp: Hparams, workspace: torch.Tensor, stream=None) -> None:
@@ -280,6 +286,88 @@ def normuon_update(batches: Sequence[Batch], hp: Hparams, use_normuon: bool, wor
     p, nbytes = _ws(workspace)
     _capi.check(_capi.lib.normuon_update(arr, nb, ctypes.byref(h), int(bool(use_normuon)), p, nbytes,
                                          _stream_ptr(stream)), "normuon_update")
+
+
+class TwoStreamStep:
+    """One optimizer step over several batches, scheduled on two streams.
+
+    Scheduling only (every operation is one of the C-ABI calls above): the
+    Newton-Schulz call of batch i runs on the caller's stream while the
+    momentum of batch i + 1 and the NorMuon + update of batch i - 1 run on a
+    second stream, so the tensor-core-bound and the HBM-bound kernels of the
+    step overlap.  Calls on different streams must not share a workspace:
+    each stream gets its own, sized for the largest batch.  Batch i's
+    Newton-Schulz call waits for its momentum and its update waits for its
+    Newton-Schulz call (events).  The two smallest batches go first and
+    last, where their kernels cannot overlap anything.  Results are those of
+    the serial calls: every slice's result is independent of the batch it
+    is in.
+
+    ``variant``: "standard", "gram" or "auto" (``gram_min_ratio`` as in
+    ``muon_ns_auto_batched``).  Call it with the stream to enqueue on (the
+    current stream by default); it can be captured in a CUDA graph after one
+    eager call.
+    """
+
+    def __init__(self, batches: Sequence[Batch], hp: Hparams, variant: str = "standard", use_normuon: bool = True,
+                 gram_min_ratio: float = 1.25, device=None):
+        if not batches:
+            raise ValueError("no batches")
+        sizes = [b.n * b.rows * b.cols for b in batches]
+        by_size = sorted(range(len(batches)), key=lambda i: (sizes[i], i))
+        if len(batches) > 2:
+            middle = sorted(by_size[2:], key=lambda i: (-sizes[i], i))
+            self.order = [by_size[0]] + middle + [by_size[1]]
+        else:
+            self.order = by_size
+        self.batches = [batches[i] for i in self.order]
+        self.hp = hp
+        self.variant = variant
+        self.use_normuon = bool(use_normuon)
+        self.gram_min_ratio = float(gram_min_ratio)
+        which_ns = {"standard": 1, "gram": 2, "auto": -1}[variant]
+        dev = device or "cuda"
+        ns_bytes = max(muon_workspace_size([b], which_ns) for b in self.batches)
+        ew_bytes = max(max(muon_workspace_size([b], 0), muon_workspace_size([b], 3)) for b in self.batches)
+        self.ws_ns = torch.zeros(max(256, ns_bytes), dtype=torch.uint8, device=dev)
+        self.ws_ew = torch.zeros(max(256, ew_bytes), dtype=torch.uint8, device=dev)
+        self.ew_stream = torch.cuda.Stream(device=dev)
+        self.ev_mom = [torch.cuda.Event() for _ in self.batches]
+        self.ev_ns = [torch.cuda.Event() for _ in self.batches]
+
+    def _ns(self, b, stream):
+        if self.variant == "standard":
+            muon_ns_batched([b], self.hp, self.ws_ns, stream)
+        elif self.variant == "gram":
+            muon_gram_ns_batched([b], self.hp, self.ws_ns, stream)
+        else:
+            muon_ns_auto_batched([b], self.hp, self.ws_ns, self.gram_min_ratio, stream)
+
+    def __call__(self, stream=None) -> None:
+        main = stream if stream is not None else torch.cuda.current_stream()
+        side = self.ew_stream
+        side.wait_stream(main)
+        bs = self.batches
+        for i, b in enumerate(bs):
+            muon_momentum_norm([b], self.hp, self.ws_ew, side)
+            self.ev_mom[i].record(side)
+            main.wait_event(self.ev_mom[i])
+            self._ns(b, main)
+            self.ev_ns[i].record(main)
+            if i > 0:
+                side.wait_event(self.ev_ns[i - 1])
+                normuon_update([bs[i - 1]], self.hp, self.use_normuon, self.ws_ew, side)
+        side.wait_event(self.ev_ns[-1])
+        normuon_update([bs[-1]], self.hp, self.use_normuon, self.ws_ew, side)
+        main.wait_stream(side)
+
+    def workspace_errors(self) -> int:
+        """The Newton-Schulz workspace's error word (0: no device-side wait ran out).
+
+        Each Newton-Schulz call clears the word when it starts, so this is the
+        last call's status; the momentum and update kernels have no waits.
+        """
+        return workspace_error(self.ws_ns)
 
 
 def workspace_error(workspace: torch.Tensor, stream=None) -> int:

@@ -547,3 +547,53 @@ def test_ns_polar_express_schedule(mn, variant, shape):
         # the exact result lies in [1 - E_5, 1 + E_5]; bf16 adds a little.
         s_out = np.linalg.svd(got[i], compute_uv=False)
         assert np.all(np.abs(s_out - 1.0) <= errs[-1] + 0.05), (s_out.min(), s_out.max(), errs[-1])
+
+
+@pytest.mark.parametrize("variant", ["standard", "gram", "auto"])
+def test_two_stream_step_equals_serial_calls(mn, variant):
+    # TwoStreamStep only schedules the same C-ABI calls per batch on two
+    # streams (Newton-Schulz of one batch overlapping the momentum of the
+    # next and the update of the previous) with a workspace per stream; the
+    # results must equal the serial calls over all batches bit for bit, also
+    # when the step is captured in a CUDA graph and replayed.
+    shapes = [(2, 300, 520), (3, 64, 576), (1, 256, 256), (2, 520, 300), (4, 128, 4096), (2, 640, 100)]
+
+    def state():
+        bs = []
+        for k, (n, r, c) in enumerate(shapes):
+            d = dict(grad=_seeded(n, r, c, 600 + k, torch.bfloat16), momentum=_aligned(n, r, c, torch.bfloat16),
+                     ns_in=_aligned(n, r, c, torch.bfloat16), ns_out=_aligned(n, r, c, torch.bfloat16),
+                     weight=_seeded(n, r, c, 650 + k, torch.float32, std=0.02),
+                     weight_copy=_aligned(n, r, c, torch.bfloat16), sumsq=torch.zeros(n, device=DEV),
+                     variance=torch.zeros(n * r, device=DEV), row_sumsq=torch.zeros(n * r, device=DEV))
+            bs.append(mn.Batch(n, r, c, fan_out=r, fan_in=c, **d))
+        return bs
+
+    hp = mn.Hparams(lr=0.02, weight_decay=0.01)
+    serial, two, graphed = state(), state(), state()
+    ws = mn.allocate_workspace(serial, -1)
+    for _ in range(2):
+        mn.muon_momentum_norm(serial, hp, ws)
+        if variant == "standard":
+            mn.muon_ns_batched(serial, hp, ws)
+        elif variant == "gram":
+            mn.muon_gram_ns_batched(serial, hp, ws)
+        else:
+            mn.muon_ns_auto_batched(serial, hp, ws, gram_min_ratio=1.25)
+        mn.normuon_update(serial, hp, True, ws)
+    step = mn.TwoStreamStep(two, hp, variant, True)
+    for _ in range(2):
+        step()
+    gstep = mn.TwoStreamStep(graphed, hp, variant, True)
+    gstep()                                             # eager first call (per-device set-up)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        gstep()
+    g.replay()                                          # second step of the graphed state
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0 and step.workspace_errors() == 0 and gstep.workspace_errors() == 0
+    for a, b, c in zip(serial, two, graphed):
+        for name in ("momentum", "ns_out", "weight", "weight_copy", "variance", "row_sumsq"):
+            assert torch.equal(getattr(a, name), getattr(b, name)), (name, a.rows, a.cols)
+            assert torch.equal(getattr(a, name), getattr(c, name)), ("graph", name, a.rows, a.cols)
