@@ -205,7 +205,8 @@ def test_gram_rank_deficient_stays_in_band(mn, shape, rank):
 
 
 @pytest.mark.parametrize("restart", [0, 1, 2, 3])
-@pytest.mark.parametrize("shape,steps", [((128, 1024), 5), ((300, 200), 5), ((256, 768), 7), ((96, 700), 16)])
+@pytest.mark.parametrize("shape,steps", [((128, 1024), 5), ((300, 200), 5), ((256, 768), 7), ((96, 700), 16),
+                                         ((128, 4096), 5), ((96, 6000), 7)])
 def test_gram_restart_periods_match_oracle(mn, restart, shape, steps):
     r, c = shape
     U = _seeded(2, r, c, 140 + r, torch.bfloat16)
