@@ -177,11 +177,18 @@ MUON_API muon_status muon_momentum_norm(const muon_batch* batches, int nb, const
  * rows > cols is iterated transposed; the result O is in the slice's own
  * orientation.  X0 = U / (sqrt(sumsq) + ns_eps), with sumsq from
  * muon_momentum_norm when batch.sumsq is non-NULL, else computed here.
- * Batches whose slices have rows <= cols, rows <= 128 and cols <= 4096 run
- * every iteration in one launch (a thread-block cluster per slice, the slice
- * held in shared memory, X X^T summed across the cluster in a fixed order);
- * the choice depends on the shape only, so a slice's result does not depend
- * on the rest of the batch.
+ * Batches whose slices have a short side <= 128 run every iteration in one
+ * launch (a thread-block cluster per slice, X X^T summed across the cluster
+ * in a fixed order): long side <= 2048 (or <= 4096 when not a multiple of 8)
+ * with the slice held in shared memory, long side 2049..16384 and a multiple
+ * of 8 with its columns streamed from L2 each iteration; tall slices go
+ * through a transposed copy in the workspace.  The choice depends on the
+ * shape only, so a slice's result does not depend on the rest of the batch.
+ * When a call has both such batches and others, the fused batches run on a
+ * second stream owned by the calling thread, forked from `stream` after the
+ * call's first work and joined back into it before the call returns (event
+ * record and wait: legal under stream capture); work enqueued on `stream`
+ * afterwards is ordered after all of the call's work.
  * Reads ns_in (left unchanged), sumsq; writes ns_out, and row_sumsq when it
  * is non-NULL (per output row, the sum of squares of the stored bf16 values,
  * summed in a fixed order: tile partials from the last product's epilogue).

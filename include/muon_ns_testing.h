@@ -56,11 +56,17 @@ MUON_API muon_status muon_testing_bounded_wait(uint64_t limit_ns, void* workspac
 /*
  * Kernel-selection switches for tests and experiments, process-wide (all
  * devices, all threads); production callers never need them.  Defaults:
- *   fused_small   1: slices with short side <= 128 and long side <= 4096 run
- *                    the fused clustered kernel; 0: the GEMM path
+ *   fused_small   1: slices with short side <= 128 run the fused clustered
+ *                    kernels (long side <= 2048, or <= 4096 when not a
+ *                    multiple of 8: columns resident in shared memory; long
+ *                    side 2049..16384 and a multiple of 8: columns streamed
+ *                    from L2); 0: every slice takes the GEMM path
  *   max_waves    32: waves of tiles per GEMM launch (0: no cap)
  *   max_problems  1: problems that share a GEMM launch beyond one wave (1..8)
  *   pdl           1: programmatic dependent launch; 0: plain launches
+ *   overlap       1: a call with both fused and GEMM-path slices runs the
+ *                    fused ones on a second stream of the calling thread,
+ *                    joined back before the call's later work; 0: one stream
  * Sets *opts when non-NULL (after range checks: MUON_INVALID_ARG and no
  * change when a value is out of range) and returns the previous switches in
  * *previous when non-NULL.  Not to be called while another thread enqueues
@@ -71,6 +77,7 @@ typedef struct {
   int32_t max_waves;
   int32_t max_problems;
   int32_t pdl;
+  int32_t overlap;
 } muon_testing_options;
 
 MUON_API muon_status muon_testing_set_options(const muon_testing_options* opts, muon_testing_options* previous);

@@ -381,12 +381,12 @@ def workspace_error(workspace: torch.Tensor, stream=None) -> int:
 def testing_options(**switches):
     """Temporarily sets the library's kernel-selection switches (include/muon_ns_testing.h).
 
-    Keys: fused_small, max_waves, max_problems, pdl.  For tests and
+    Keys: fused_small, max_waves, max_problems, pdl, overlap.  For tests and
     experiments; production calls use the defaults.
     """
     prev = _capi.MuonTestingOptions()
     _capi.check(_capi.lib.muon_testing_set_options(None, ctypes.byref(prev)), "muon_testing_set_options")
-    new = _capi.MuonTestingOptions(prev.fused_small, prev.max_waves, prev.max_problems, prev.pdl)
+    new = _capi.MuonTestingOptions(prev.fused_small, prev.max_waves, prev.max_problems, prev.pdl, prev.overlap)
     for k, v in switches.items():
         if not hasattr(new, k):
             raise KeyError(k)

@@ -51,7 +51,7 @@ class MuonHparams(ctypes.Structure):
 
 class MuonTestingOptions(ctypes.Structure):
     _fields_ = [("fused_small", ctypes.c_int32), ("max_waves", ctypes.c_int32), ("max_problems", ctypes.c_int32),
-                ("pdl", ctypes.c_int32)]
+                ("pdl", ctypes.c_int32), ("overlap", ctypes.c_int32)]
 
 
 MUON_SCALE_SPECTRAL, MUON_SCALE_RMS_NORM = 0, 1

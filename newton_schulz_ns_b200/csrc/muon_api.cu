@@ -58,6 +58,7 @@ struct Options {
   std::atomic<int> max_waves{32};
   std::atomic<int> max_problems{1};
   std::atomic<int> pdl{1};
+  std::atomic<int> overlap{1};
 };
 Options g_opt;
 
@@ -192,6 +193,87 @@ muon_status device_setup(int* sms_out, int* pair_units_out = nullptr) {
   if (pair_units_out) *pair_units_out = d.pair_units;
   return MUON_OK;
 }
+
+// ------------------------------------------------------------ second stream
+// A call whose batches take both the fused small-side kernels and the GEMM
+// path runs the fused slices on a second stream beside the GEMM launches:
+// the two touch disjoint workspace regions and outputs, and the fused
+// kernel holds one cluster per slice for the whole iteration while the GEMM
+// chain of the other slices is a series of short launches that leave most
+// SMs idle.  The second stream (highest priority, so the fused clusters are
+// placed first when both are waiting) and its two events belong to the
+// calling thread and device, and are made again when the device's context
+// changes.  Fork and join are an event record plus a wait on each side, a
+// pattern that stream capture accepts; the join is issued on every return
+// path once the fork was made.
+struct SideStream {
+  unsigned long long ctx = 0;
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+thread_local SideStream t_side[kMaxDevices];
+
+class SideFork {
+ public:
+  SideFork() = default;
+  SideFork(const SideFork&) = delete;
+  SideFork& operator=(const SideFork&) = delete;
+  ~SideFork() { (void)close(); }
+
+  // *work receives the stream the fused slices go to: the second stream
+  // when `want`, else `main` itself.
+  muon_status open(cudaStream_t main, bool want, cudaStream_t* work) {
+    *work = main;
+    if (!want) return MUON_OK;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MUON_CUDA_ERROR;
+    SideStream& t = t_side[dev];
+    const unsigned long long ctx = current_ctx_id();
+    if (t.s == nullptr || ctx != t.ctx) {   // first use on this thread, or a new context (old handles are gone)
+      // Creating a stream or an event enqueues nothing; relaxed capture mode
+      // lets a first call made under stream capture do it.
+      cudaStreamCaptureMode mode = cudaStreamCaptureModeRelaxed;
+      (void)cudaThreadExchangeStreamCaptureMode(&mode);
+      int lo = 0, hi = 0;
+      const bool ok = cudaDeviceGetStreamPriorityRange(&lo, &hi) == cudaSuccess &&
+                      cudaStreamCreateWithPriority(&t.s, cudaStreamNonBlocking, hi) == cudaSuccess &&
+                      cudaEventCreateWithFlags(&t.fork, cudaEventDisableTiming) == cudaSuccess &&
+                      cudaEventCreateWithFlags(&t.join, cudaEventDisableTiming) == cudaSuccess;
+      (void)cudaThreadExchangeStreamCaptureMode(&mode);
+      if (!ok) {
+        (void)cudaGetLastError();
+        t = SideStream{};
+        return MUON_CUDA_ERROR;
+      }
+      t.ctx = ctx;
+    }
+    if (cudaEventRecord(t.fork, main) != cudaSuccess || cudaStreamWaitEvent(t.s, t.fork, 0) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return MUON_CUDA_ERROR;
+    }
+    main_ = main;
+    side_ = t.s;
+    join_ = t.join;
+    *work = side_;
+    return MUON_OK;
+  }
+
+  // Makes `main` wait for everything enqueued on the second stream.
+  muon_status close() {
+    if (side_ == nullptr) return MUON_OK;
+    const cudaStream_t s = side_;
+    side_ = nullptr;
+    if (cudaEventRecord(join_, s) != cudaSuccess || cudaStreamWaitEvent(main_, join_, 0) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return MUON_CUDA_ERROR;
+    }
+    return MUON_OK;
+  }
+
+ private:
+  cudaStream_t main_ = nullptr, side_ = nullptr;
+  cudaEvent_t join_ = nullptr;
+};
 
 // ---------------------------------------------------------------- validation
 inline bool dtype_is(int32_t dt, std::initializer_list<int> allowed) {
@@ -1144,9 +1226,11 @@ muon_status muon_testing_set_options(const muon_testing_options* opts, muon_test
   cur.max_waves = g_opt.max_waves.load();
   cur.max_problems = g_opt.max_problems.load();
   cur.pdl = g_opt.pdl.load();
+  cur.overlap = g_opt.overlap.load();
   if (opts) {
     if ((opts->fused_small != 0 && opts->fused_small != 1) || opts->max_waves < 0 || opts->max_waves > 1000000 ||
-        opts->max_problems < 1 || opts->max_problems > MAX_PROBLEMS || (opts->pdl != 0 && opts->pdl != 1))
+        opts->max_problems < 1 || opts->max_problems > MAX_PROBLEMS || (opts->pdl != 0 && opts->pdl != 1) ||
+        (opts->overlap != 0 && opts->overlap != 1))
       return MUON_INVALID_ARG;
   }
   if (previous) *previous = cur;
@@ -1155,6 +1239,7 @@ muon_status muon_testing_set_options(const muon_testing_options* opts, muon_test
     g_opt.max_waves.store(opts->max_waves);
     g_opt.max_problems.store(opts->max_problems);
     g_opt.pdl.store(opts->pdl);
+    g_opt.overlap.store(opts->overlap);
   }
   return MUON_OK;
 }
@@ -1278,6 +1363,27 @@ muon_status finalize_gemm_row_sums(const muon_batch* batches, int nb, const Layo
   return MUON_OK;
 }
 
+// Marks the batches that take the fused small-side kernels and enqueues
+// them: on a second stream when the call also has GEMM-path batches (and
+// the overlap switch is on), else on the call's stream.
+muon_status start_fused(const muon_batch* batches, int nb, const Layout& L, uint8_t* ws, const muon_hparams* hp,
+                        const std::vector<const float*>& sumsq, int* err, bool gram, int sms, cudaStream_t stream,
+                        std::vector<char>& fused, SideFork& side, cudaStream_t& fstream) {
+  fused.assign(nb, 0);
+  bool any_fused = false, any_gemm = false;
+  for (int i = 0; i < nb; ++i) {
+    if (batch_empty(batches[i])) continue;
+    fused[i] = small_eligible(batches[i]) ? 1 : 0;
+    if (fused[i]) any_fused = true;
+    else any_gemm = true;
+  }
+  const bool fork = any_fused && any_gemm && g_opt.overlap.load(std::memory_order_relaxed) != 0;
+  muon_status st = side.open(stream, fork, &fstream);
+  for (int i = 0; i < nb && st == MUON_OK; ++i)
+    if (fused[i]) st = run_small(batches[i], L.nsb[i], ws, hp, sumsq[i], err, gram, sms, fstream);
+  return st;
+}
+
 muon_status ns_standard_impl(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
                              size_t workspace_bytes, cudaStream_t stream, bool clear_err) {
   muon_status st = validate_ns(batches, nb, hp);
@@ -1294,12 +1400,11 @@ muon_status ns_standard_impl(const muon_batch* batches, int nb, const muon_hpara
   if ((st = prepare_norms(batches, nb, L, ws, sms, stream, sumsq, clear_err)) != MUON_OK) return st;
   int* err = reinterpret_cast<int*>(ws);
 
-  std::vector<char> fused(nb, 0);
-  for (int i = 0; i < nb; ++i) {
-    if (batch_empty(batches[i]) || !small_eligible(batches[i])) continue;
-    fused[i] = 1;
-    if ((st = run_small(batches[i], L.nsb[i], ws, hp, sumsq[i], err, false, sms, stream)) != MUON_OK) return st;
-  }
+  std::vector<char> fused;
+  SideFork side;
+  cudaStream_t fstream = stream;
+  if ((st = start_fused(batches, nb, L, ws, hp, sumsq, err, false, sms, stream, fused, side, fstream)) != MUON_OK)
+    return st;
   const int S = hp->ns_steps;
   for (int it = 0; it < S; ++it) {
     const Coefs cf = coefs_at(hp, it);
@@ -1331,7 +1436,8 @@ muon_status ns_standard_impl(const muon_batch* batches, int nb, const muon_hpara
     if ((st = launch_gemms(poly, sms, err, stream)) != MUON_OK) return st;
     if ((st = launch_gemms(apply, sms, err, stream)) != MUON_OK) return st;
   }
-  return finalize_gemm_row_sums(batches, nb, L, ws, fused, sms, stream);
+  if ((st = finalize_gemm_row_sums(batches, nb, L, ws, fused, sms, stream)) != MUON_OK) return st;
+  return side.close();
 }
 
 muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* hp, void* workspace,
@@ -1352,12 +1458,11 @@ muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* 
   const int S = hp->ns_steps;
   const float kap = kGramScale;
 
-  std::vector<char> fused(nb, 0);
-  for (int i = 0; i < nb; ++i) {
-    if (batch_empty(batches[i]) || !small_eligible(batches[i])) continue;
-    fused[i] = 1;
-    if ((st = run_small(batches[i], L.nsb[i], ws, hp, sumsq[i], err, true, sms, stream)) != MUON_OK) return st;
-  }
+  std::vector<char> fused;
+  SideFork side;
+  cudaStream_t fstream = stream;
+  if ((st = start_fused(batches, nb, L, ws, hp, sumsq, err, true, sms, stream, fused, side, fstream)) != MUON_OK)
+    return st;
   // G: kappa * s^2 * X X^T (short side) in fp16.
   {
     std::vector<ProblemSpec> g;
@@ -1458,7 +1563,8 @@ muon_status ns_gram_impl(const muon_batch* batches, int nb, const muon_hparams* 
     }
     if ((st = launch_gemms(o, sms, err, stream)) != MUON_OK) return st;
   }
-  return finalize_gemm_row_sums(batches, nb, L, ws, fused, sms, stream);
+  if ((st = finalize_gemm_row_sums(batches, nb, L, ws, fused, sms, stream)) != MUON_OK) return st;
+  return side.close();
 }
 
 extern "C" {

@@ -318,21 +318,21 @@ def test_update_rejects_missing_fans_and_unknown_modes(mn):
 
 def test_testing_options_round_trip_and_range_checks(mn):
     from newton_schulz_ns_b200 import _capi
-    prev = _capi.MuonTestingOptions()
-    assert _capi.lib.muon_testing_set_options(None, ctypes.byref(prev)) == 0
-    assert (prev.fused_small, prev.max_waves, prev.max_problems, prev.pdl) == (1, 32, 1, 1)
-    with mn.testing_options(fused_small=0, max_waves=4, pdl=0):
+
+    def now():
         cur = _capi.MuonTestingOptions()
-        _capi.lib.muon_testing_set_options(None, ctypes.byref(cur))
-        assert (cur.fused_small, cur.max_waves, cur.max_problems, cur.pdl) == (0, 4, 1, 0)
-    cur = _capi.MuonTestingOptions()
-    _capi.lib.muon_testing_set_options(None, ctypes.byref(cur))
-    assert (cur.fused_small, cur.max_waves, cur.max_problems, cur.pdl) == (1, 32, 1, 1)
-    for bad in [(2, 32, 1, 1), (1, -1, 1, 1), (1, 32, 0, 1), (1, 32, 9, 1), (1, 32, 1, 3)]:
+        assert _capi.lib.muon_testing_set_options(None, ctypes.byref(cur)) == 0
+        return (cur.fused_small, cur.max_waves, cur.max_problems, cur.pdl, cur.overlap)
+
+    assert now() == (1, 32, 1, 1, 1)
+    with mn.testing_options(fused_small=0, max_waves=4, pdl=0, overlap=0):
+        assert now() == (0, 4, 1, 0, 0)
+    assert now() == (1, 32, 1, 1, 1)
+    for bad in [(2, 32, 1, 1, 1), (1, -1, 1, 1, 1), (1, 32, 0, 1, 1), (1, 32, 9, 1, 1), (1, 32, 1, 3, 1),
+                (1, 32, 1, 1, 2), (1, 32, 1, 1, -1)]:
         o = _capi.MuonTestingOptions(*bad)
         assert _capi.lib.muon_testing_set_options(ctypes.byref(o), None) == 1
-    _capi.lib.muon_testing_set_options(None, ctypes.byref(cur))
-    assert (cur.fused_small, cur.max_waves, cur.max_problems, cur.pdl) == (1, 32, 1, 1)
+    assert now() == (1, 32, 1, 1, 1)
 
 
 def test_row_sum_partials_take_workspace_only_when_requested(mn):

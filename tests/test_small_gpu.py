@@ -237,3 +237,104 @@ def test_fused_small_step_captured_in_cuda_graph(mn):
     assert mn.workspace_error(ws) == 0
     for e, o in zip(eager, outs):
         assert torch.equal(e, o)
+
+
+def _mixed_batches(mn, seed, with_rows=True):
+    # Fused slices (streamed heads, resident conv slices, a tall transposed
+    # one) beside GEMM-path slices (short side above 128) in one call.
+    shapes = [(8, 128, 4096), (2, 512, 1024), (3, 64, 576), (2, 1024, 512), (2, 700, 96)]
+    Us, outs, rss, bs = [], [], [], []
+    for k, (n, r, c) in enumerate(shapes):
+        U = _seeded(n, r, c, seed + k)
+        _, out = _padded(n, r, c, torch.bfloat16, float("nan"))
+        rs = torch.full((n, r), float("nan"), dtype=torch.float32, device=DEV) if with_rows else None
+        Us.append(U)
+        outs.append(out)
+        rss.append(rs)
+        bs.append(mn.Batch(n, r, c, ns_in=U, ns_out=out, row_sumsq=rs))
+    return Us, outs, rss, bs
+
+
+@pytest.mark.parametrize("variant", ["standard", "gram"])
+def test_overlapped_fused_slices_match_single_stream(mn, variant):
+    # With both kinds of slices in one call the fused ones run on a second
+    # stream beside the GEMM chain; the results (and row sums) are bitwise
+    # those of the one-stream schedule, and match the oracle.
+    Us, outs, rss, bs = _mixed_batches(mn, 610)
+    fn = mn.muon_ns_batched if variant == "standard" else mn.muon_gram_ns_batched
+    ws = mn.allocate_workspace(bs, 1 if variant == "standard" else 2)
+    results = {}
+    for overlap in (1, 0):
+        for o, r in zip(outs, rss):
+            o.fill_(float("nan"))
+            r.fill_(float("nan"))
+        with mn.testing_options(overlap=overlap):
+            fn(bs, mn.Hparams(), ws)
+            torch.cuda.synchronize()
+        assert mn.workspace_error(ws) == 0
+        results[overlap] = ([o.clone() for o in outs], [r.clone() for r in rss])
+    for a, b in zip(results[1][0] + results[1][1], results[0][0] + results[0][1]):
+        assert torch.equal(a, b)
+    for U, out in zip(Us, outs):
+        ref = oracle.ns_batched(f64(U[:1]), variant)
+        assert rel(f64(out[:1])[0], ref[0]) < NS_TOL
+
+
+def test_overlapped_call_is_ordered_before_later_stream_work(mn):
+    # Work enqueued on the call's stream right after it (a copy of every
+    # output, no host synchronization in between) sees the fused slices'
+    # results: the second stream is joined back before the call returns.
+    Us, outs, rss, bs = _mixed_batches(mn, 640)
+    ws = mn.allocate_workspace(bs, 1)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            for o in outs:
+                o.fill_(float("nan"))
+            mn.muon_ns_batched(bs, mn.Hparams(), ws, s)
+            copies = [o.clone() for o in outs] + [r.clone() for r in rss]
+    torch.cuda.synchronize()
+    assert mn.workspace_error(ws) == 0
+    for c, o in zip(copies, outs + rss):
+        assert not torch.isnan(c).any()
+        assert torch.equal(c, o)
+
+
+def test_overlapped_call_first_used_inside_graph_capture(mn):
+    # A thread whose first mixed call is inside stream capture makes its
+    # second stream and events there; the captured graph replays to the
+    # eager result.
+    import threading
+    Us, outs, rss, bs = _mixed_batches(mn, 670)
+    ws = mn.allocate_workspace(bs, 2)
+    hp = mn.Hparams()
+    with mn.testing_options(overlap=0):
+        mn.muon_gram_ns_batched(bs, hp, ws)
+    torch.cuda.synchronize()
+    eager = [o.clone() for o in outs] + [r.clone() for r in rss]
+    box = {}
+
+    def worker():
+        try:
+            torch.cuda.set_device(0)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                mn.muon_gram_ns_batched(bs, hp, ws, torch.cuda.current_stream())
+            for o in outs + rss:
+                o.fill_(float("nan"))
+            torch.cuda.synchronize()
+            g.replay()
+            torch.cuda.synchronize()
+            box["ok"] = True
+        except Exception as e:   # reported in the main thread
+            box["err"] = e
+
+    t = threading.Thread(target=worker)
+    t.start()
+    t.join(120)
+    assert not t.is_alive()
+    assert "err" not in box, box.get("err")
+    assert mn.workspace_error(ws) == 0
+    for e, o in zip(eager, outs + rss):
+        assert torch.equal(e, o)
