@@ -224,3 +224,32 @@ def test_long_k_launch_with_several_waves(mn, cta_pair):
     for t in range(nh):
         want = np.sum(c[:, :, 128 * t:128 * (t + 1)] ** 2, axis=2)
         assert np.allclose(_f64(rss)[:, t], want, rtol=1e-5)
+
+
+@pytest.mark.parametrize("tri", [False, True])
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0)])
+def test_single_and_pair_tiles_are_bitwise_equal(mn, tri, a_mn, b_mn):
+    # Both tile kernels issue the same K-ordered sequence of K = 16 tensor-core
+    # steps into fp32 accumulators and share the epilogue, so the choice of
+    # kernel (single-CTA 128 x 256 or 2-CTA 256 x 256 tiles) never changes a
+    # stored bit; the library may pick either for a slice.
+    S, M, K = 2, 520, 700
+    N = M if tri else 1000
+    A = _rnd((S, K, M) if a_mn else (S, M, K), torch.bfloat16, 21)
+    B = A if tri else _rnd((S, K, N) if b_mn else (S, N, K), torch.bfloat16, 22)
+    bmn = a_mn if tri else b_mn
+    D = _rnd((S, M, N), torch.bfloat16, 23)
+    ss = torch.tensor([2.0, 5.0], device=DEV)
+    rows = {}
+    outs = {}
+    for pair in PAIRS:
+        C = _empty((S, M, N), torch.bfloat16)
+        rss = None if tri else torch.full((S, 2 * ((N + 255) // 256), M), float("nan"), device=DEV)
+        mn.testing_gemm(A, bool(a_mn), B, bool(bmn), C, K=K, tri=tri, D=D, alpha=0.7, beta=1.3, gamma=0.25,
+                        s_pow=1, sumsq=ss, eps=1e-7, row_ss=rss, cta_pair=pair, workspace=_ws())
+        torch.cuda.synchronize()
+        outs[pair] = C.clone()
+        rows[pair] = rss
+    assert torch.equal(outs[1], outs[2])
+    if not tri:
+        assert torch.equal(rows[1], rows[2])
