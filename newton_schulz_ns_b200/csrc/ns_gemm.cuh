@@ -178,6 +178,47 @@ __device__ __forceinline__ float load_elem(const void* base, long long off, int 
   return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[off]);
 }
 
+// Element j of a chunk packed two per word (low half first).
+__device__ __forceinline__ uint16_t half16(const uint32_t (&w32)[16], int j) {
+  return static_cast<uint16_t>(w32[j >> 1] >> ((j & 1) * 16));
+}
+
+// One 32-column chunk of an epilogue row: x = v * f (+ gamma where the
+// column is the row, j == dj), rounded to bf16 or fp16 two at a time into
+// w32, and css += (rounded x)^2 over the first ncol columns in column order.
+template <bool F16>
+__device__ __forceinline__ void round_chunk(const float (&v)[32], float f, float gamma, int dj, int ncol,
+                                            uint32_t (&w32)[16], float& css) {
+  float xr[32];
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    float x0 = v[j] * f, x1 = v[j + 1] * f;
+    if (dj >= 0) {                                     // only chunks that cross the diagonal
+      x0 = (j == dj) ? x0 + gamma : x0;
+      x1 = (j + 1 == dj) ? x1 + gamma : x1;
+    }
+    if constexpr (F16) {
+      const __half2 h = __floats2half2_rn(x0, x1);
+      w32[j >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+      xr[j] = __low2float(h);
+      xr[j + 1] = __high2float(h);
+    } else {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+      w32[j >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+      xr[j] = __low2float(h);
+      xr[j + 1] = __high2float(h);
+    }
+  }
+  if (ncol == 32) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) css += xr[j] * xr[j];
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < ncol) css += xr[j] * xr[j];
+  }
+}
+
 template <int CG>
 __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
   using Cfg = GemmCfg<CG>;
@@ -470,8 +511,13 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
         if (col0 >= pr.N) continue;                       // warp-uniform (every later chunk too)
         const bool full_chunk = col0 + 32 <= pr.N;
         float v[32];
+        if (pr.alpha == 1.0f) {                            // x * 1 == x: skip the multiply (uniform)
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = pr.alpha * __uint_as_float(r[j]);
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = pr.alpha * __uint_as_float(r[j]);
+        }
         if (use_add && row_ok) {
           const long long aoff = add_slice + static_cast<long long>(row) * pr.add_ld + col0;
           if (full_chunk) {
@@ -500,25 +546,18 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
               v[j] += pr.beta * load_elem(pr.addend, aoff + j, pr.add_f16);
           }
         }
-        // Round to the output type once; these are the values stored.
-        uint16_t h16[32];
+        // Round to the output type once (two values per conversion); these
+        // are the values stored.  The identity term touches only chunks that
+        // cross the diagonal (warp-uniform test), and whole chunks of a valid
+        // row sum every square without per-column tests.
+        uint32_t w32[16];
         float css = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float x = v[j] * f;
-          if (pr.gamma != 0.0f && row == col0 + j) x += pr.gamma;
-          float xr;
-          if (pr.out_f16) {
-            const __half hv = __float2half_rn(x);
-            h16[j] = __half_as_ushort(hv);
-            xr = __half2float(hv);
-          } else {
-            const __nv_bfloat16 hv = __float2bfloat16_rn(x);
-            h16[j] = __bfloat16_as_ushort(hv);
-            xr = __bfloat162float(hv);
-          }
-          if (row_ok && col0 + j < pr.N) css += xr * xr;
-        }
+        const bool diag = pr.gamma != 0.0f && col0 < row0 + 32 && row0 < col0 + 32;
+        const int ncol = row_ok ? min(32, pr.N - col0) : 0;  // columns of this row that count
+        if (pr.out_f16)
+          round_chunk<true>(v, f, diag ? pr.gamma : 0.0f, diag ? row - col0 : -1, ncol, w32, css);
+        else
+          round_chunk<false>(v, f, diag ? pr.gamma : 0.0f, diag ? row - col0 : -1, ncol, w32, css);
         if (c < EPI_CHUNKS)
           rss0 += css;
         else
@@ -539,11 +578,7 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
           // Row `lane`, 64 bytes, 16-byte chunks placed by the 64-byte swizzle.
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
-            const uint4 val = make_uint4(
-                static_cast<uint32_t>(h16[8 * w + 0]) | (static_cast<uint32_t>(h16[8 * w + 1]) << 16),
-                static_cast<uint32_t>(h16[8 * w + 2]) | (static_cast<uint32_t>(h16[8 * w + 3]) << 16),
-                static_cast<uint32_t>(h16[8 * w + 4]) | (static_cast<uint32_t>(h16[8 * w + 5]) << 16),
-                static_cast<uint32_t>(h16[8 * w + 6]) | (static_cast<uint32_t>(h16[8 * w + 7]) << 16));
+            const uint4 val = make_uint4(w32[4 * w], w32[4 * w + 1], w32[4 * w + 2], w32[4 * w + 3]);
             *reinterpret_cast<uint4*>(sd + lane * 64 + ((w ^ ((lane >> 1) & 3)) << 4)) = val;
           }
           fence_proxy_async_smem();
@@ -555,12 +590,12 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
           ++stores;
         } else if (row_ok) {
           for (int j = 0; j < 32 && col0 + j < pr.N; ++j)
-            out16[out_slice + static_cast<long long>(row) * pr.out_ld + col0 + j] = h16[j];
+            out16[out_slice + static_cast<long long>(row) * pr.out_ld + col0 + j] = half16(w32, j);
         }
         if (mirror && row_ok) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (col0 + j < pr.N) out16[out_slice + static_cast<long long>(col0 + j) * pr.out_ld + row] = h16[j];
+            if (col0 + j < pr.N) out16[out_slice + static_cast<long long>(col0 + j) * pr.out_ld + row] = half16(w32, j);
         }
 #pragma unroll
         for (int w = 0; w < 4; ++w) add_cur[w] = add_nxt[w];
