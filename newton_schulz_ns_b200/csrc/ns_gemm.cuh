@@ -185,14 +185,19 @@ __device__ __forceinline__ uint16_t half16(const uint32_t (&w32)[16], int j) {
 
 // One 32-column chunk of an epilogue row: x = v * f (+ gamma where the
 // column is the row, j == dj), rounded to bf16 or fp16 two at a time into
-// w32, and css += (rounded x)^2 over the first ncol columns in column order.
-template <bool F16>
-__device__ __forceinline__ void round_chunk(const float (&v)[32], float f, float gamma, int dj, int ncol,
+// w32; with SS, css += (rounded x)^2 over the first ncol columns in column
+// order.  (x * 1 == x: a unit factor is not multiplied.)
+template <bool F16, bool SS>
+__device__ __forceinline__ void round_chunk(float (&v)[32], float f, float gamma, int dj, int ncol,
                                             uint32_t (&w32)[16], float& css) {
+  if (f != 1.0f) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] *= f;
+  }
   float xr[32];
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
-    float x0 = v[j] * f, x1 = v[j + 1] * f;
+    float x0 = v[j], x1 = v[j + 1];
     if (dj >= 0) {                                     // only chunks that cross the diagonal
       x0 = (j == dj) ? x0 + gamma : x0;
       x1 = (j + 1 == dj) ? x1 + gamma : x1;
@@ -209,13 +214,15 @@ __device__ __forceinline__ void round_chunk(const float (&v)[32], float f, float
       xr[j + 1] = __high2float(h);
     }
   }
-  if (ncol == 32) {
+  if constexpr (SS) {
+    if (ncol == 32) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) css += xr[j] * xr[j];
-  } else {
+      for (int j = 0; j < 32; ++j) css += xr[j] * xr[j];
+    } else {
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < ncol) css += xr[j] * xr[j];
+      for (int j = 0; j < 32; ++j)
+        if (j < ncol) css += xr[j] * xr[j];
+    }
   }
 }
 
@@ -554,10 +561,19 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
         float css = 0.0f;
         const bool diag = pr.gamma != 0.0f && col0 < row0 + 32 && row0 < col0 + 32;
         const int ncol = row_ok ? min(32, pr.N - col0) : 0;  // columns of this row that count
-        if (pr.out_f16)
-          round_chunk<true>(v, f, diag ? pr.gamma : 0.0f, diag ? row - col0 : -1, ncol, w32, css);
-        else
-          round_chunk<false>(v, f, diag ? pr.gamma : 0.0f, diag ? row - col0 : -1, ncol, w32, css);
+        const float gm = diag ? pr.gamma : 0.0f;
+        const int dj = diag ? row - col0 : -1;
+        if (pr.row_ss != nullptr) {                       // sums of squares only where they are stored
+          if (pr.out_f16)
+            round_chunk<true, true>(v, f, gm, dj, ncol, w32, css);
+          else
+            round_chunk<false, true>(v, f, gm, dj, ncol, w32, css);
+        } else {
+          if (pr.out_f16)
+            round_chunk<true, false>(v, f, gm, dj, ncol, w32, css);
+          else
+            round_chunk<false, false>(v, f, gm, dj, ncol, w32, css);
+        }
         if (c < EPI_CHUNKS)
           rss0 += css;
         else
