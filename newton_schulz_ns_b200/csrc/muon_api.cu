@@ -210,6 +210,14 @@ struct SideStream {
   unsigned long long ctx = 0;
   cudaStream_t s = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
+  // Released when the thread ends, while their context is still the
+  // current one (handles of a context that is gone are not touched).
+  ~SideStream() {
+    if (s == nullptr || ctx == 0 || ctx != current_ctx_id()) return;
+    (void)cudaEventDestroy(fork);
+    (void)cudaEventDestroy(join);
+    (void)cudaStreamDestroy(s);
+  }
 };
 thread_local SideStream t_side[kMaxDevices];
 
@@ -242,7 +250,9 @@ class SideFork {
       (void)cudaThreadExchangeStreamCaptureMode(&mode);
       if (!ok) {
         (void)cudaGetLastError();
-        t = SideStream{};
+        t.s = nullptr;   // whatever was made is left to the context
+        t.fork = t.join = nullptr;
+        t.ctx = 0;
         return MUON_CUDA_ERROR;
       }
       t.ctx = ctx;
