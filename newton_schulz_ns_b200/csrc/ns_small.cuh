@@ -5,8 +5,8 @@
 //   A = X X^T,  B = b A + c A^2,  X <- a X + B X
 // (Newton-Schulz iteration as the Megatron-Core layer_sharded_muon docs and
 // DeepSpeed issue #8437 describe it; the first step works on the Frobenius-
-// normalized X0 = s U, s = 1 / (||U||_F + eps), folded into the epilogues as
-// on the GEMM path).  With m this small each product is a few MFLOP, so the
+// normalized X0 = s U, s = 1 / (||U||_F + eps), formed in fp16 as the input
+// is read).  With m this small each product is a few MFLOP, so the
 // GEMM path spends its time in launches and pipeline fill.  Here one
 // thread-block cluster of C CTAs (C = 1, 2, 4 or 8) runs all steps of one
 // slice in one launch:
@@ -19,7 +19,7 @@
 //     partial to the CTA that owns the row's 8-row block, with distributed-
 //     shared-memory stores that count their bytes on the owner's mbarrier;
 //     once all C partials of its rows have arrived each owner sums them in
-//     rank order (deterministic), scales and rounds them to bf16 and pushes
+//     rank order (deterministic), scales and rounds them to fp16 and pushes
 //     them into every CTA's copy of A the same way; once all of A's lower
 //     triangle has arrived each CTA fills the upper triangle from it (A is
 //     exactly symmetric, as on the GEMM path);
@@ -36,10 +36,18 @@
 // their lower triangles; the last Q is rounded to bf16 and O = s Q X0 is
 // formed on the resident columns.
 //
-// Precision follows the GEMM path: bf16 operands, fp32 accumulation, A, B
-// and X rounded to bf16 between products.  Operand layouts are the 128-byte
-// swizzled tiles TMA writes (64 columns x 128 rows per 16 KB block): X is
-// read K-major for X X^T and MN-major for B X without any copy.
+// Precision: fp32 accumulation; in the standard form X, A and B are
+// rounded to fp16 between products (every entry is at most about 1 in
+// magnitude: X0 is normalized and the iteration keeps singular values near
+// 1) and the last X to bf16, the output type.  bf16 iterates, as on the GEMM
+// path, lose too much on slices with a very short side: with 3 or 4 rows the
+// few singular values sit where the composed quintic is steep, and a model
+// of bf16 arithmetic lands up to 0.05 from the exact result (fp16: <= 0.008
+// for every short side up to 128).  The Gram form keeps its m x m side in
+// fp16 and its X side in bf16.  Operand layouts are the 128-byte swizzled
+// tiles TMA writes (64 columns x 128 rows per 16 KB block, 16-bit values
+// of either type): X is read K-major for X X^T and MN-major for B X without
+// any copy.
 //
 // 256 threads, one CTA per SM (the shared-memory request reserves the SM):
 // thread 0 issues TMA and MMAs; in the epilogues warp w reads TMEM lanes
@@ -60,9 +68,9 @@ constexpr int SMALL_MAX_STEPS = 16;
 constexpr int SMALL_MAX_CLUSTER = 8;
 constexpr int SMALL_MAX_M = 128;
 constexpr int SMALL_MAX_W = 512;                       // resident columns per CTA
-constexpr int SMALL_BLK = 128 * 128;                   // one 64-column block of 128 bf16 rows
+constexpr int SMALL_BLK = 128 * 128;                   // one 64-column block of 128 rows (16-bit)
 constexpr int SMALL_X_BYTES = SMALL_MAX_W / 64 * SMALL_BLK;   // 128 KB
-constexpr int SMALL_A_BYTES = 2 * SMALL_BLK;                  // A (then B in place): 128 x 128 bf16
+constexpr int SMALL_A_BYTES = 2 * SMALL_BLK;                  // A (then B in place): 128 x 128, 16-bit
 constexpr int SMALL_RECV_BYTES = 128 * 512;                   // C slots of fp32 partial rows
 constexpr int SMALL_SMEM_BYTES = 1024 + SMALL_X_BYTES + SMALL_A_BYTES + SMALL_RECV_BYTES + 64;
 
@@ -146,6 +154,21 @@ __device__ __forceinline__ uint32_t bf16_at(const uint4& u, int e) {
 __device__ __forceinline__ uint4 pack_bf16x8(const float (&o)[8]) {
   return make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
                     pack_bf16x2(o[6], o[7]));
+}
+
+// In place over nbytes (a multiple of 16) of 16-bit values: bf16 x -> fp16 (s x).
+// The standard form's first iterate X0 = s U, s = 1 / (||U||_F + eps), so
+// every entry is at most 1 in magnitude.  The caller orders the stores before
+// tensor-core reads (the fence below, then a CTA barrier).
+__device__ __forceinline__ void to_f16_scaled(uint8_t* p, int nbytes, float s, int tid) {
+  for (int i = tid * 16; i < nbytes; i += SMALL_THREADS * 16) {
+    float f[8];
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(p + i), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] *= s;
+    *reinterpret_cast<uint4*>(p + i) = pack_f16x8(f);
+  }
+  fence_proxy_async_smem();
 }
 
 __device__ __forceinline__ void small_record_error(int* err, volatile int* abort_flag, int code) {
@@ -245,11 +268,12 @@ __device__ __forceinline__ void epi_square(uint32_t taddr, int row, int half, in
 }
 
 // Epilogue of the product on the resident columns for row `row`, columns
-// [half w/2, half w/2 + w/2): X <- f (acc + a X), in place, bf16.  With
-// rss non-null, also the sum of squares of the stored values of those
-// columns (zero outside the slice) is written to *rss for rows below m.
+// [half w/2, half w/2 + w/2): X <- f (acc + a X), in place; X is read as
+// fp16 (x_f16) or bf16 and written as fp16 (out_f16) or bf16.  With rss
+// non-null, also the sum of squares of the stored values of those columns
+// (zero outside the slice) is written to *rss for rows below m.
 __device__ __forceinline__ void epi_columns(uint32_t taddr, int row, int half, int w, int m8, float a, float f,
-                                            uint8_t* Xs, float* rss = nullptr, int m = 0) {
+                                            uint8_t* Xs, bool x_f16, bool out_f16, float* rss = nullptr, int m = 0) {
   const int hw = w >> 1;
   const int cend = half * hw + hw;
   float ss = 0.0f;
@@ -273,18 +297,24 @@ __device__ __forceinline__ void epi_columns(uint32_t taddr, int row, int half, i
       for (int h = 0; h < 8; ++h) {
         if (h < nch) {
           float xf[8], o[8];
-          unpack_bf16x8(xv[h], xf);
+          if (x_f16)
+            unpack_f16x8(xv[h], xf);
+          else
+            unpack_bf16x8(xv[h], xf);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             float x = __uint_as_float(v[h * 8 + e]);
             x += a * xf[e];
             o[e] = x * f;
           }
-          const uint4 pk = pack_bf16x8(o);
+          const uint4 pk = out_f16 ? pack_f16x8(o) : pack_bf16x8(o);
           *reinterpret_cast<uint4*>(Xs + sw128_chunk(row, (c0 >> 3) + h)) = pk;
           if (rss != nullptr) {
             float st[8];
-            unpack_bf16x8(pk, st);
+            if (out_f16)
+              unpack_f16x8(pk, st);
+            else
+              unpack_bf16x8(pk, st);
 #pragma unroll
             for (int e = 0; e < 8; ++e) ss += st[e] * st[e];
           }
@@ -373,13 +403,12 @@ struct SmallCta {
   }
 
   // A = fA * (sum over the cluster of the partials in TMEM [0, 128)), into
-  // every CTA's As (bf16; fp16 in the Gram form), upper triangle mirrored.
+  // every CTA's As (fp16), upper triangle mirrored.
   // Partial rows and A's rows travel as st.async stores that complete bytes
   // on the receiver's mbarrier, so each CTA waits only for the data it needs.
   // (Every CTA's next exchange starts after it holds this exchange's A,
   // which needs every owner to have finished reading its receive slots: the
   // slots and barriers are never overwritten early.)
-  template <bool GRAM>
   __device__ __forceinline__ void exchange(float fA) {
     if (ok && tid == 0) {
       mbar_arrive_expect_tx(recv_bar, recv_bytes);
@@ -451,7 +480,7 @@ struct SmallCta {
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] *= fA;
-        const uint4 pk = GRAM ? pack_f16x8(acc) : pack_bf16x8(acc);
+        const uint4 pk = pack_f16x8(acc);
         const uint32_t dst = a0 + sw128_chunk(8 * b + r8, g);
         const uint32_t abar = smem_u32(a_bar);
         for (int q = 0; q < C; ++q)
@@ -470,9 +499,9 @@ struct SmallCta {
     __syncthreads();
   }
 
-  // A^2 -> TMEM columns [128, 256), then B = c A^2 + b A in place over A.
+  // A^2 -> TMEM columns [128, 256), then B = c A^2 + b A in place over A (fp16).
   __device__ __forceinline__ void form_b(float cb, float cc) {
-    const uint32_t idesc_sq = mma_idesc_f16(1, 0, 0, 128, 128);
+    const uint32_t idesc_sq = mma_idesc_f16(0, 0, 0, 128, 128);
     if (ok) {
       if (tid == 0) {
         fence_proxy_async_smem();
@@ -487,7 +516,7 @@ struct SmallCta {
     }
     if (ok) {
       tc_fence_after();
-      epi_square(tmem + tlane + 128u, row, half, m8, m, cc, cb, As, false, 0.0f, As, false);
+      epi_square(tmem + tlane + 128u, row, half, m8, m, cc, cb, As, true, 0.0f, As, true);
       fence_proxy_async_smem();
     }
     tc_fence_before();
@@ -496,31 +525,41 @@ struct SmallCta {
 };
 
 // The whole iteration, for a kernel whose columns `X` provide
-//   partial(c, k)          : TMEM [0, 128) = this CTA's X_r X_r^T before step k (the
-//                            input's at k = 0; the streaming kernel accumulates the later
-//                            ones during its passes, so it only does k = 0)
-//   apply(c, F, a, f, rss, next) : X_r <- f (F X_r + a X_r) with F a 128 x 128 bf16
-//                            K-major matrix in shared memory; rss (or null): this
-//                            thread's row sum of squares of the stored values; next:
-//                            a later exchange will need this X's partial
-// Standard form: per step exchange, B, apply.  Gram form: one exchange of
-// kappa s^2 X0 X0^T, the m x m iteration on P and Q (fp16, kappa-scaled A,
-// every CTA alike), restarts every P.restart steps (X <- xf Q X, A again
-// from an exchange, Q = I), and O = xf Q X.
+//   to_half(c, s)          : X_r <- fp16(s X_r) before the first product (the
+//                            streaming kernel converts each block as it reads the input)
+//   partial(c, k, h)       : TMEM [0, 128) = this CTA's X_r X_r^T before step k, X in
+//                            fp16 (h) or bf16 (the input's at k = 0; the streaming kernel
+//                            accumulates the later ones during its passes, so it only
+//                            does k = 0)
+//   apply(c, F, a, f, rss, next, h, ho) : X_r <- f (F X_r + a X_r) with F a 128 x 128
+//                            K-major matrix in shared memory, F and X in fp16 (h) or
+//                            bf16, the result stored as fp16 (ho) or bf16; rss (or
+//                            null): this thread's row sum of squares of the stored
+//                            values; next: a later exchange will need this X's partial
+// Standard form: X0 = s U in fp16, then per step exchange, B, apply, all in
+// fp16 (X, A, B; fp32 accumulation) with the last X stored as bf16.  (bf16
+// iterates, as on the GEMM path, miss the 3e-2 bar on slices with a short
+// side of 3 or 4, whose few singular values sit where the composed quintic
+// is steep; fp16 keeps every short side within a fifth of it.)  Gram form:
+// one exchange of kappa s^2 X0 X0^T, the m x m iteration on P and Q (fp16,
+// kappa-scaled A, every CTA alike), restarts every P.restart steps
+// (X <- xf Q X, A again from an exchange, Q = I), and O = xf Q X, the X
+// side in bf16.
 template <bool GRAM, class Cols>
 __device__ __forceinline__ void small_iterate(SmallCta& c, Cols& X, const SmallParams& P, float s, float* row_slot) {
   if (!GRAM) {
+    X.to_half(c, s);
     for (int k = 0; k < P.steps; ++k) {
-      X.partial(c, k);
-      c.template exchange<false>((k == 0) ? s * s : 1.0f);
+      X.partial(c, k, true);
+      c.exchange(1.0f);
       c.form_b(P.b[k], P.c[k]);
       const bool last = k == P.steps - 1;
-      X.apply(c, c.a0, P.a[k], (k == 0) ? s : 1.0f, (last && P.row_ss != nullptr) ? row_slot : nullptr, !last);
+      X.apply(c, c.a0, P.a[k], 1.0f, (last && P.row_ss != nullptr) ? row_slot : nullptr, !last, true, !last);
     }
     return;
   }
-  X.partial(c, 0);
-  c.template exchange<true>(P.kappa * (s * s));
+  X.partial(c, 0, false);
+  c.exchange(P.kappa * (s * s));
   uint8_t* Pb = c.Rv;                             // P (and, at a segment's start, the first Q)
   uint8_t* Qb = c.Rv + SMALL_A_BYTES;             // Q
   const int tid = c.tid;
@@ -540,13 +579,13 @@ __device__ __forceinline__ void small_iterate(SmallCta& c, Cols& X, const SmallP
   for (int k = 0; k < P.steps; ++k) {
     if (restart_at(k)) {
       // X <- xf Q X (Q in bf16)
-      X.apply(c, smem_u32(Qb), 0.0f, xf, nullptr, true);
+      X.apply(c, smem_u32(Qb), 0.0f, xf, nullptr, true, false, false);
       xf = 1.0f;
-      X.partial(c, k);
+      X.partial(c, k, false);
       tc_fence_before();
       __syncthreads();
       cluster_sync();       // no CTA still reads its Q when peers push partial rows over it
-      c.template exchange<true>(kap);
+      c.exchange(kap);
       clear_pq();
       seg_start = k;
     }
@@ -604,7 +643,7 @@ __device__ __forceinline__ void small_iterate(SmallCta& c, Cols& X, const SmallP
     }
   }
   // O = xf Q X (Q in bf16)
-  X.apply(c, smem_u32(Qb), 0.0f, xf, P.row_ss != nullptr ? row_slot : nullptr, false);
+  X.apply(c, smem_u32(Qb), 0.0f, xf, P.row_ss != nullptr ? row_slot : nullptr, false, false, false);
 }
 
 // ---------------------------------------------------------------------------
@@ -614,9 +653,14 @@ struct ResidentCols {
   uint8_t* Xs;
   int w;
 
-  __device__ __forceinline__ void partial(SmallCta& c, int) {
+  __device__ __forceinline__ void to_half(SmallCta& c, float s) {
+    if (c.ok) to_f16_scaled(Xs, (w >> 6) * SMALL_BLK, s, c.tid);
+    __syncthreads();
+  }
+
+  __device__ __forceinline__ void partial(SmallCta& c, int, bool h) {
     if (!c.ok) return;
-    const uint32_t idesc_sq = mma_idesc_f16(1, 0, 0, 128, 128);
+    const uint32_t idesc_sq = mma_idesc_f16(h ? 0u : 1u, 0, 0, 128, 128);
     if (c.tid == 0) {
       fence_proxy_async_smem();
       tc_fence_after();
@@ -630,7 +674,8 @@ struct ResidentCols {
     c.ok = c.wait_mma();
   }
 
-  __device__ __forceinline__ void apply(SmallCta& c, uint32_t f0, float a, float f, float* rss, bool) {
+  __device__ __forceinline__ void apply(SmallCta& c, uint32_t f0, float a, float f, float* rss, bool, bool h,
+                                        bool ho) {
     // F X_r -> TMEM [0, w)
     if (c.ok) {
       if (c.tid == 0) {
@@ -639,7 +684,7 @@ struct ResidentCols {
         const uint32_t x0 = smem_u32(Xs);
         for (int nc = 0; nc < w; nc += 256) {
           const int N = min(256, w - nc);
-          const uint32_t idesc = mma_idesc_f16(1, 0, 1, 128, static_cast<uint32_t>(N));
+          const uint32_t idesc = mma_idesc_f16(h ? 0u : 1u, 0, 1, 128, static_cast<uint32_t>(N));
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t ad = smem_desc_sw128(f0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = smem_desc_sw128(x0 + (nc >> 6) * SMALL_BLK + kk * 16 * 128, SMALL_BLK, 1024);
@@ -653,7 +698,7 @@ struct ResidentCols {
     // X <- f (F X + a X), in place
     if (c.ok) {
       tc_fence_after();
-      epi_columns(c.tmem + c.tlane, c.row, c.half, w, c.m8, a, f, Xs, rss, c.m);
+      epi_columns(c.tmem + c.tlane, c.row, c.half, w, c.m8, a, f, Xs, h, ho, rss, c.m);
     }
     tc_fence_before();
     __syncthreads();
@@ -812,6 +857,7 @@ struct StreamCols {
   int npair, col0, slice, n;
   uint32_t loads = 0;        // pairs loaded so far over all passes: stage g % STAGES, parity (g / STAGES) & 1
   bool src_out = false;      // X lives in ns_out (after the first pass that stored it)
+  float conv = 0.0f;         // nonzero: pairs read from the input become fp16(conv x) first
 
   __device__ __forceinline__ void issue_load(const CUtensorMap* src, int p, uint32_t g) {
     const int st = static_cast<int>(g % STREAM_STAGES);
@@ -833,12 +879,15 @@ struct StreamCols {
   // One pass over this CTA's block pairs.  product = false: partial X X^T of
   // the input only.  product = true: X <- f (F X + a X) pair by pair, stored
   // to ns_out, with the next partial when `next` and row sums when rss != null.
+  // F and X are fp16 (h) or bf16; the stored X (and its partial) fp16 (ho) or bf16.
   __device__ __forceinline__ void pass(SmallCta& c, bool product, uint32_t f0, float a, float f, float* rss,
-                                       bool next) {
+                                       bool next, bool h, bool ho) {
     const CUtensorMap* src = src_out ? map_out : map_in;
     const uint32_t base = loads;
-    const uint32_t idesc_sq = mma_idesc_f16(1, 0, 0, 128, 128);
-    const uint32_t idesc_fx = mma_idesc_f16(1, 0, 1, 128, 128);
+    const uint32_t idesc_sq = mma_idesc_f16(h ? 0u : 1u, 0, 0, 128, 128);
+    const uint32_t idesc_fx = mma_idesc_f16(h ? 0u : 1u, 0, 1, 128, 128);
+    const uint32_t idesc_nx = mma_idesc_f16(ho ? 0u : 1u, 0, 0, 128, 128);
+    const bool convert = conv != 0.0f && !src_out;
     if (c.ok && c.tid == 0)
       for (int p = 0; p < min(STREAM_STAGES, npair); ++p) issue_load(src, p, base + static_cast<uint32_t>(p));
     float ss = 0.0f;
@@ -847,6 +896,10 @@ struct StreamCols {
       if (c.ok) c.ok = wait_load(c, g);
       uint8_t* xp = ring + (g % STREAM_STAGES) * STREAM_PAIR;
       const uint32_t xp0 = smem_u32(xp);
+      if (convert) {                                // the input pair as fp16(conv x), in place
+        if (c.ok) to_f16_scaled(xp, STREAM_PAIR, conv, c.tid);
+        __syncthreads();
+      }
       if (!product) {
         if (c.ok) {
           if (c.tid == 0) {
@@ -881,17 +934,23 @@ struct StreamCols {
           uint32_t v[64];
           tmem_ld_64(c.tmem + c.tlane + 256u + static_cast<uint32_t>(c.half * 64), v);
 #pragma unroll
-          for (int h = 0; h < 8; ++h) {
-            const uint32_t off = sw128_chunk(c.row, c.half * 8 + h);
+          for (int hh = 0; hh < 8; ++hh) {
+            const uint32_t off = sw128_chunk(c.row, c.half * 8 + hh);
             float xf[8], o[8];
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(xp + off), xf);
+            if (h)
+              unpack_f16x8(*reinterpret_cast<const uint4*>(xp + off), xf);
+            else
+              unpack_bf16x8(*reinterpret_cast<const uint4*>(xp + off), xf);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) o[e] = (__uint_as_float(v[h * 8 + e]) + a * xf[e]) * f;
-            const uint4 pk = pack_bf16x8(o);
+            for (int e = 0; e < 8; ++e) o[e] = (__uint_as_float(v[hh * 8 + e]) + a * xf[e]) * f;
+            const uint4 pk = ho ? pack_f16x8(o) : pack_bf16x8(o);
             *reinterpret_cast<uint4*>(xo + off) = pk;
             if (rss != nullptr) {
               float st[8];
-              unpack_bf16x8(pk, st);
+              if (ho)
+                unpack_f16x8(pk, st);
+              else
+                unpack_bf16x8(pk, st);
 #pragma unroll
               for (int e = 0; e < 8; ++e) ss += st[e] * st[e];
             }
@@ -906,7 +965,7 @@ struct StreamCols {
             const uint32_t xo0 = smem_u32(xo);
             for (int kk = 0; kk < 8; ++kk) {
               const uint64_t d = smem_desc_sw128(xo0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
-              tc_mma_f16(c.tmem, d, d, idesc_sq, (p | kk) != 0 ? 1u : 0u);
+              tc_mma_f16(c.tmem, d, d, idesc_nx, (p | kk) != 0 ? 1u : 0u);
             }
           }
           for (int b = 0; b < 2; ++b)
@@ -934,12 +993,15 @@ struct StreamCols {
     __syncthreads();
   }
 
-  __device__ __forceinline__ void partial(SmallCta& c, int k) {
-    if (k == 0) pass(c, false, 0u, 0.0f, 1.0f, nullptr, false);   // later partials come from the passes
+  __device__ __forceinline__ void to_half(SmallCta&, float s) { conv = s; }   // applied as the input is read
+
+  __device__ __forceinline__ void partial(SmallCta& c, int k, bool h) {
+    if (k == 0) pass(c, false, 0u, 0.0f, 1.0f, nullptr, false, h, h);   // later partials come from the passes
   }
 
-  __device__ __forceinline__ void apply(SmallCta& c, uint32_t f0, float a, float f, float* rss, bool next) {
-    pass(c, true, f0, a, f, rss, next);
+  __device__ __forceinline__ void apply(SmallCta& c, uint32_t f0, float a, float f, float* rss, bool next, bool h,
+                                        bool ho) {
+    pass(c, true, f0, a, f, rss, next, h, ho);
   }
 };
 

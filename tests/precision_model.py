@@ -5,9 +5,13 @@ the method.  This model runs the same iteration with every stored matrix
 rounded to bf16 (round-to-nearest-even) and every product accumulated in
 float64 before rounding to float32, which is what bf16 tensor-core operands
 with fp32 accumulation compute up to summation order.  It is used only where
-bf16 arithmetic and the exact method legitimately part ways (rank-deficient
-inputs, whose null space collects rounding noise that the iteration
-amplifies), to check that the device does no worse than that arithmetic.
+the storage precision and the exact method legitimately part ways (rank-
+deficient inputs, whose null space collects rounding noise that the
+iteration amplifies; slices with a very short side, whose few singular
+values sit where the composed quintic is steep), to check that the device
+does no worse than that arithmetic.  The fused small-side kernels store
+their standard-form iterates in fp16 (`ns_standard_f16`), the GEMM path in
+bf16 (`ns_standard_bf16`).
 It shares no code with the CUDA library.
 """
 import numpy as np
@@ -42,6 +46,29 @@ def ns_standard_bf16(U, steps=5, eps=1e-7, abc=(3.4445, -4.7750, 2.0315)):
 
 def _f16(x):
     return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float16).astype(np.float64)
+
+
+def ns_standard_f16(U, steps=5, eps=1e-7, abc=(3.4445, -4.7750, 2.0315)):
+    """Standard iteration of the fused small-side kernels (short side <= 128).
+
+    X0 = fp16(s * bf16(U)) with s = 1 / (||U||_F + eps) in float32; then X, A
+    and B = b A + c A^2 stored in fp16 between products (fp32 accumulation),
+    the last X in bf16.
+    """
+    a, b, c = abc
+    X = np.asarray(U, dtype=np.float64)
+    tr = X.shape[0] > X.shape[1]
+    if tr:
+        X = X.T
+    Xb = _bf16(X)
+    s = float(np.float32(1.0) / (np.sqrt(np.float32(np.sum(Xb * Xb))) + np.float32(eps)))
+    Xh = _f16(_f32(s * Xb))
+    for k in range(steps):
+        A = _f16(_f32(Xh @ Xh.T))
+        B = _f16(_f32(c * _f32(A @ A) + b * A))
+        Y = _f32(_f32(B @ Xh) + a * Xh)
+        Xh = _bf16(Y) if k == steps - 1 else _f16(Y)
+    return Xh.T if tr else Xh
 
 
 def ns_gram_f16(U, steps=5, eps=1e-7, abc=(3.4445, -4.7750, 2.0315), restart=3, kappa=16384.0):

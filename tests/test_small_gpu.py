@@ -13,9 +13,10 @@ at each restart) and iterates on the m x m side in every CTA.  Tall slices
 shapes below cover every cluster split the planner picks (1 to 8 resident
 CTAs of 64 to 512 columns, 4 streaming CTAs of 768 to 4096 columns), ragged
 last blocks, CTAs that hold only padding, and short sides from 1 to 128.
-Bars: 3e-2 relative Frobenius error against the oracle per slice; bitwise
-batch invariance and run-to-run determinism; nothing written outside the
-slice.
+Bars: 3e-2 relative Frobenius error against the oracle per slice (the
+standard form iterates in fp16 here: 1e-2 where it is compared with the
+GEMM path); bitwise batch invariance and run-to-run determinism; nothing
+written outside the slice.
 """
 import numpy as np
 import pytest
@@ -130,10 +131,14 @@ def test_fused_small_agrees_with_gemm_path(mn, shape, variant):
     assert nf < ng
     ref = oracle.ns_batched(f64(U), variant)
     for i in range(2):
-        assert rel(f64(fused)[i], ref[i]) < NS_TOL
         assert rel(f64(gemm)[i], ref[i]) < NS_TOL
-        # Same arithmetic up to the order of fp32 sums: far below the bar.
-        assert rel(f64(fused)[i], f64(gemm)[i]) < 1e-2
+        if variant == "standard":
+            # fp16 iterates on the fused path (bf16 on the GEMM path): well inside the bar
+            assert rel(f64(fused)[i], ref[i]) < 1e-2
+        else:
+            # the same arithmetic up to the order of fp32 sums
+            assert rel(f64(fused)[i], ref[i]) < NS_TOL
+            assert rel(f64(fused)[i], f64(gemm)[i]) < 1e-2
 
 
 @pytest.mark.parametrize("variant", ["standard", "gram"])
