@@ -169,8 +169,11 @@ MUON_API muon_status muon_momentum_norm(const muon_batch* batches, int nb, const
                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
- * Standard quintic Newton-Schulz of every slice, bf16 operands, fp32
- * accumulation on the tensor cores.
+ * Standard quintic Newton-Schulz of every slice, fp32 accumulation on the
+ * tensor cores; X, A and B are stored in bf16 between products, or in fp16
+ * for slices whose short side is at most 128 (the fused path below: with
+ * 3 or 4 rows bf16 rounding alone can move the result past 3e-2 of the
+ * exact one).  The output is bf16.
  * [ds-8437] "Why it happens": normalize, then iterate on X X^T.
  * [mcore-lsm] use_syrk: A = X X^T and B = b*A + c*A^2 are symmetric, one
  * triangle of each is computed.  Per iteration X <- a*X + B X.  A slice with
