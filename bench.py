@@ -161,19 +161,39 @@ def default_variant(wl):
 
 # ----------------------------------------------------------------------------- CPU oracle (baseline)
 
+def small_kernel(r, c):
+    """The fused kernel a slice takes (the library's shape rule), or None for the GEMM path."""
+    m, n = min(r, c), max(r, c)
+    if m > 128:
+        return None
+    if n <= 2048:
+        return "ns_small_kernel"                 # columns resident on <= 4 CTAs
+    if n % 8 == 0 and n <= 16384:
+        return "ns_stream_kernel"                # columns streamed from L2, 4-CTA clusters
+    if n <= 4096:
+        return "ns_small_kernel"                 # resident on 8 CTAs
+    return None
+
+
 def ns_kernels_label(groups):
-    """Which kernels one Newton-Schulz call of these batches runs (the library's shape rule)."""
-    def fused(r, c):
-        m, n = min(r, c), max(r, c)
-        return m <= 128 and n <= 4096
-    kinds = {fused(b.rows, b.cols) for b in groups}
-    if kinds == {True}:
-        name = "ns_small_kernel (fused: one clustered launch per batch)"
-    elif kinds == {False}:
-        name = "ns_gemm_pair_kernel / ns_gemm_kernel"
-    else:
-        name = "ns_small_kernel + ns_gemm_pair_kernel"
-    return name + " (all launches of one Newton-Schulz call)"
+    """Which kernels one Newton-Schulz call of these batches runs."""
+    names = []
+    for b in groups:
+        k = small_kernel(b.rows, b.cols) or "ns_gemm_pair_kernel / ns_gemm_kernel"
+        if k not in names:
+            names.append(k)
+    return " + ".join(names) + " (all launches of one Newton-Schulz call)"
+
+
+def ns_dtype(groups, variant):
+    """The arithmetic type of the path: bf16 on the GEMM path; the fused kernels' standard form
+    iterates in fp16 (bf16 in and out)."""
+    if variant in ("gram", "auto"):
+        return "bf16 (Gram form: fp16 m x m side)"
+    fused = {small_kernel(b.rows, b.cols) is not None for b in groups}
+    if fused == {False}:
+        return "bf16"
+    return "fp16 (bf16 in/out)" if fused == {True} else "bf16 + fp16 (short sides <= 128)"
 
 
 def coefficients_desc(args):
@@ -569,7 +589,7 @@ def run_ours(args, wl, variant, rank, world, local_rank):
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch Philox on the device)",
+        "vs_baseline": None, "dtype": ns_dtype(groups, variant), "data": "synthetic (seeded torch Philox on the device)",
         "config": dict(workload_config(args, wl, variant), parallelism=f"replicas x{world} (no exchange)"),
         "launch": ("CUDA graph of one whole step, replayed for each timed step" if args.graph == "on"
                    else "eager calls"),
