@@ -909,6 +909,11 @@ struct StreamCols {
               tc_mma_f16(c.tmem, d, d, idesc_sq, (p | kk) != 0 ? 1u : 0u);
             }
             tc_commit(c.mma_bar);
+            if (convert) {        // keep fp16 X0 in ns_out: the next pass reads it instead of converting again
+              for (int b = 0; b < 2; ++b)
+                if (col0 + 128 * p + 64 * b < n) tma_store_3d(map_out, xp + b * SMALL_BLK, col0 + 128 * p + 64 * b, 0, slice);
+              bulk_commit_group();
+            }
           }
           c.ok = c.wait_mma();
         }
@@ -974,11 +979,18 @@ struct StreamCols {
         }
       }
       // The stage's pair has been read by its product and by the epilogue
-      // (before the barrier above): load the pair STAGES ahead into it.
-      if (c.ok && c.tid == 0 && p + STREAM_STAGES < npair)
+      // (before the barrier above), and by its store when X0 was kept: load
+      // the pair STAGES ahead into it.
+      if (c.ok && c.tid == 0 && p + STREAM_STAGES < npair) {
+        if (!product && convert) bulk_wait_group_read<0>();
         issue_load(src, p + STREAM_STAGES, g + static_cast<uint32_t>(STREAM_STAGES));
+      }
     }
     loads = base + static_cast<uint32_t>(npair);
+    if (!product && convert) {
+      if (c.tid == 0) bulk_wait_group_all();     // X0 in ns_out before the next pass loads it
+      src_out = true;
+    }
     if (product) {
       // the last partial product, and every store, complete before the next pass or exchange
       if (c.ok) {
