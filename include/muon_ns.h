@@ -195,6 +195,8 @@ MUON_API muon_status muon_momentum_norm(const muon_batch* batches, int nb, const
  * Reads ns_in (left unchanged), sumsq; writes ns_out, and row_sumsq when it
  * is non-NULL (per output row, the sum of squares of the stored bf16 values,
  * summed in a fixed order: tile partials from the last product's epilogue).
+ * No batch's ns_out may share a byte with any batch's ns_in or with another
+ * batch's ns_out (MUON_INVALID_ARG): ns_out also holds intermediate iterates.
  */
 MUON_API muon_status muon_ns_batched(const muon_batch* batches, int nb, const muon_hparams* hp,
                             void* workspace, size_t workspace_bytes, cudaStream_t stream);

@@ -1107,6 +1107,17 @@ ProblemSpec apply_spec(const muon_batch& b, const Mat& f, const Mat& x, void* ou
   return s;
 }
 
+// Byte range [first, last) a view of batch b spans.
+struct ByteRange {
+  uintptr_t first, last;
+};
+ByteRange view_range(const muon_batch& b, const muon_view& v) {
+  const int64_t span = (b.n - 1) * v.batch_stride + (b.rows - 1) * v.ld + b.cols;
+  const uintptr_t p = reinterpret_cast<uintptr_t>(v.ptr);
+  return ByteRange{p, p + static_cast<uintptr_t>(span) * static_cast<uintptr_t>(esize(v.dtype))};
+}
+inline bool overlaps(const ByteRange& a, const ByteRange& b) { return a.first < b.last && b.first < a.last; }
+
 muon_status validate_ns(const muon_batch* bs, int nb, const muon_hparams* hp) {
   if (nb < 0 || (nb > 0 && bs == nullptr)) return MUON_INVALID_ARG;
   muon_status st = check_hp(hp);
@@ -1117,7 +1128,18 @@ muon_status validate_ns(const muon_batch* bs, int nb, const muon_hparams* hp) {
     if (batch_empty(b)) continue;
     if ((st = check_view(b, b.ns_in, {MUON_BF16}, true)) != MUON_OK) return st;
     if ((st = check_view(b, b.ns_out, {MUON_BF16}, true)) != MUON_OK) return st;
-    if (b.ns_in.ptr == b.ns_out.ptr) return MUON_INVALID_ARG;
+  }
+  // The iteration reads ns_in while it writes ns_out (and, on the fused
+  // path, keeps its intermediate iterates there): no output may share a byte
+  // with any input or with another batch's output of the call.
+  for (int i = 0; i < nb; ++i) {
+    if (batch_empty(bs[i])) continue;
+    const ByteRange out = view_range(bs[i], bs[i].ns_out);
+    for (int j = 0; j < nb; ++j) {
+      if (batch_empty(bs[j])) continue;
+      if (overlaps(out, view_range(bs[j], bs[j].ns_in))) return MUON_INVALID_ARG;
+      if (j > i && overlaps(out, view_range(bs[j], bs[j].ns_out))) return MUON_INVALID_ARG;
+    }
   }
   return MUON_OK;
 }

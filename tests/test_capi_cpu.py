@@ -144,6 +144,28 @@ def test_dtype_and_alignment_rules(mn):
 
 
 @no_device
+@pytest.mark.parametrize("fn", ["muon_ns_batched", "muon_gram_ns_batched"])
+def test_newton_schulz_outputs_may_not_overlap_inputs_or_each_other(mn, fn):
+    good = _fake_batch(mn, 2, 64, 576)
+    # ns_out starting one row into ns_in, or on it
+    part = _fake_batch(mn, 2, 64, 576)
+    part.ns_out.ptr = part.ns_in.ptr + 2 * 576
+    same = _fake_batch(mn, 2, 64, 576)
+    same.ns_out.ptr = same.ns_in.ptr
+    # another batch's output on this batch's input, and two outputs on one buffer
+    other = _fake_batch(mn, 1, 64, 576, ptr=0x7F4000000000)
+    other.ns_out.ptr = good.ns_in.ptr + 2 * 576 * 64
+    twin = _fake_batch(mn, 1, 64, 576, ptr=0x7F5000000000)
+    twin.ns_out.ptr = good.ns_out.ptr
+    for bad in ([part], [same], [good, other], [good, twin]):
+        assert _call(mn, fn, bad, 0x7F0000300000, 1 << 30) == 1
+    # adjacent, not overlapping: passes validation (then no device: CUDA error, or not a B200)
+    near = _fake_batch(mn, 2, 64, 576)
+    near.ns_out.ptr = near.ns_in.ptr + 2 * (2 * 64 * 576)
+    assert _call(mn, fn, [near], 0x7F0000300000, 1 << 30) in (6, 7)
+
+
+@no_device
 def test_empty_batches_enqueue_nothing(mn):
     for fn in ("muon_momentum_norm", "muon_ns_batched", "muon_gram_ns_batched", "normuon_update"):
         assert _call(mn, fn, [_fake_batch(mn, 0, 64, 576)], None, 0) == 0
