@@ -65,13 +65,26 @@ def _batch(mn, n, r, c, seed, pad):
     return U, base, base[:, :, :c], rs
 
 
-@pytest.mark.parametrize("variant", ["standard", "gram"])
+def _caller(mn, variant):
+    if variant == "auto":   # Gram for slices with n >= 1.25 m, standard otherwise
+        return lambda bs, hp, ws: mn.muon_ns_auto_batched(bs, hp, ws, 1.25)
+    return mn.muon_ns_batched if variant == "standard" else mn.muon_gram_ns_batched
+
+
+def _oracle_variant(variant, r, c):
+    if variant != "auto":
+        return variant
+    m, n = min(r, c), max(r, c)
+    return "gram" if n > m and n >= 1.25 * m else "standard"
+
+
+@pytest.mark.parametrize("variant", ["standard", "gram", "auto"])
 def test_random_shapes_one_call(mn, variant):
-    fn = mn.muon_ns_batched if variant == "standard" else mn.muon_gram_ns_batched
+    fn = _caller(mn, variant)
     parts = [_batch(mn, n, r, c, 900 + k, 8 * (k % 3)) for k, (n, r, c) in enumerate(SHAPES)]
     bs = [mn.Batch(U.shape[0], U.shape[1], U.shape[2], ns_in=U, ns_out=o, row_sumsq=rs)
           for U, _, o, rs in parts]
-    ws = mn.allocate_workspace(bs, 1 if variant == "standard" else 2)
+    ws = mn.allocate_workspace(bs, -1)
     fn(bs, mn.Hparams(), ws)
     torch.cuda.synchronize()
     assert mn.workspace_error(ws) == 0
@@ -79,7 +92,7 @@ def test_random_shapes_one_call(mn, variant):
     for (U, base, o, rs), (n, r, c) in zip(parts, SHAPES):
         assert torch.isnan(base[:, :, c:].float()).all(), (n, r, c)      # nothing past the slice
         got = f64(o)
-        ref = oracle.ns_batched(f64(U), variant)
+        ref = oracle.ns_batched(f64(U), _oracle_variant(variant, r, c))
         for i in range(n):
             assert rel(got[i], ref[i]) < NS_TOL, ((n, r, c), i, rel(got[i], ref[i]))
         ss = (got.astype(np.float64) ** 2).sum(axis=2)
@@ -89,7 +102,7 @@ def test_random_shapes_one_call(mn, variant):
         U, _, o, rs = parts[k]
         o.fill_(float("nan"))
         rs.fill_(float("nan"))
-        w1 = mn.allocate_workspace([bs[k]], 1 if variant == "standard" else 2)
+        w1 = mn.allocate_workspace([bs[k]], -1)
         fn([bs[k]], mn.Hparams(), w1)
         torch.cuda.synchronize()
         assert mn.workspace_error(w1) == 0
