@@ -888,7 +888,11 @@ struct StreamCols {
     const uint32_t idesc_fx = mma_idesc_f16(h ? 0u : 1u, 0, 1, 128, 128);
     const uint32_t idesc_nx = mma_idesc_f16(ho ? 0u : 1u, 0, 0, 128, 128);
     const bool convert = conv != 0.0f && !src_out;
-    if (c.ok && c.tid == 0)
+    // thread io issues this pass's TMA loads and stores: thread 0 in the
+    // input pass; in an apply pass thread 32 (another warp), so that its TMA
+    // work proceeds beside thread 0's tensor-core issue
+    const int io = product ? 32 : 0;
+    if (c.ok && c.tid == io)
       for (int p = 0; p < min(STREAM_STAGES, npair); ++p) issue_load(src, p, base + static_cast<uint32_t>(p));
     float ss = 0.0f;
     for (int p = 0; p < npair; ++p) {
@@ -919,10 +923,10 @@ struct StreamCols {
         }
       } else {
         uint8_t* xo = Xo + (p & 1) * STREAM_PAIR;
+        if (c.ok && c.tid == io) bulk_wait_group_read<1>();   // the store from xo two pairs ago has read it
         // F X_p -> TMEM [256, 384); its commit also covers the previous pair's partial product
         if (c.ok) {
           if (c.tid == 0) {
-            bulk_wait_group_read<1>();              // the stores from xo two pairs ago have read it
             tc_fence_after();
             for (int kk = 0; kk < 8; ++kk) {
               const uint64_t ad = smem_desc_sw128(f0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
@@ -964,15 +968,15 @@ struct StreamCols {
         }
         tc_fence_before();
         __syncthreads();
-        if (c.ok && c.tid == 0) {
-          if (next) {
-            tc_fence_after();
-            const uint32_t xo0 = smem_u32(xo);
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t d = smem_desc_sw128(xo0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
-              tc_mma_f16(c.tmem, d, d, idesc_nx, (p | kk) != 0 ? 1u : 0u);
-            }
+        if (c.ok && c.tid == 0 && next) {
+          tc_fence_after();
+          const uint32_t xo0 = smem_u32(xo);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t d = smem_desc_sw128(xo0 + (kk >> 2) * SMALL_BLK + (kk & 3) * 32, 16, 1024);
+            tc_mma_f16(c.tmem, d, d, idesc_nx, (p | kk) != 0 ? 1u : 0u);
           }
+        }
+        if (c.ok && c.tid == io) {
           for (int b = 0; b < 2; ++b)
             if (col0 + 128 * p + 64 * b < n) tma_store_3d(map_out, xo + b * SMALL_BLK, col0 + 128 * p + 64 * b, 0, slice);
           bulk_commit_group();
@@ -981,7 +985,7 @@ struct StreamCols {
       // The stage's pair has been read by its product and by the epilogue
       // (before the barrier above), and by its store when X0 was kept: load
       // the pair STAGES ahead into it.
-      if (c.ok && c.tid == 0 && p + STREAM_STAGES < npair) {
+      if (c.ok && c.tid == io && p + STREAM_STAGES < npair) {
         if (!product && convert) bulk_wait_group_read<0>();
         issue_load(src, p + STREAM_STAGES, g + static_cast<uint32_t>(STREAM_STAGES));
       }
@@ -997,7 +1001,7 @@ struct StreamCols {
         if (c.tid == 0) tc_commit(c.mma_bar);
         c.ok = c.wait_mma();
       }
-      if (c.tid == 0) bulk_wait_group_all();
+      if (c.tid == io) bulk_wait_group_all();
       src_out = true;
       if (rss != nullptr && c.row < c.m) *rss = ss;
     }
