@@ -73,13 +73,36 @@ def parse():
     return ap.parse_args()
 
 
-def load_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def _peak_number(v):
+    """A peak as a plain number, or from a record that holds one (value / median / mean / max)."""
+    if isinstance(v, (int, float)) and v > 0:
+        return float(v)
+    if isinstance(v, dict):
+        for k in ("value", "median", "mean", "max"):
+            if isinstance(v.get(k), (int, float)) and v[k] > 0:
+                return float(v[k])
+    return None
+
+
+def load_peaks(path=None):
+    """The measured peaks (hbm_gbs, bf16_tflops, bf16_tflops_sustained) where the measurements file
+    holds them, the fallback figures elsewhere; returns (peaks, {key: "measured" | "fallback"})."""
+    p = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    d = {}
     if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        return d, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
+        try:
+            with open(p) as f:
+                raw = json.load(f)
+            if isinstance(raw, dict):
+                for k in FALLBACK_PEAKS:
+                    v = _peak_number(raw.get(k))
+                    if v is not None:
+                        d[k] = v
+        except (OSError, ValueError):
+            d = {}
+    peaks = dict(FALLBACK_PEAKS)
+    peaks.update(d)
+    return peaks, {k: ("measured" if k in d else "fallback") for k in FALLBACK_PEAKS}
 
 
 AUTO_GRAM_RATIO = 1.25
@@ -604,11 +627,13 @@ def run_ours(args, wl, variant, rank, world, local_rank):
                          "normuon_update": round(upd_mean, 3)},
         "hbm_kernels": {"momentum_gbs": round(momentum_bytes(groups) / (mom_mean / 1e3) / 1e9, 1),
                         "update_gbs": round(update_bytes(groups, wl.normuon) / (upd_mean / 1e3) / 1e9, 1),
-                        "peak_gbs": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])},
+                        "peak_gbs": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
+                        "peak_source": src["hbm_gbs"]},
         "roofline": {"bound": "tensor", "kernel": ns_kernels_label(groups),
                      "achieved": round(achieved, 2), "peak": peak_s, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_s, 4), "frac_of_burst": round(achieved / peak_b, 4),
-                     "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a long step)",
+                     "peak_source": f"{src['bf16_tflops_sustained']} bf16_tflops_sustained (kernel timed inside a long "
+                                    f"step)",
                      "traffic": measured_traffic(wl.key, variant) if args.scale_down == 1 else None,
                      "traffic_unit": "bytes per Newton-Schulz call: ncu dram__bytes_read.sum + write.sum of "
                                      "one-layer launches, scaled by the slices and steps of one call "

@@ -57,3 +57,24 @@ def test_reference_arm_rank_rule():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_peaks_file_read_per_key(tmp_path):
+    import bench
+    full = tmp_path / "full.json"
+    full.write_text('{"hbm_gbs": 6546.6, "bf16_tflops": 1648.7, "bf16_tflops_sustained": 1352.3}')
+    peaks, src = bench.load_peaks(str(full))
+    assert peaks == {"hbm_gbs": 6546.6, "bf16_tflops": 1648.7, "bf16_tflops_sustained": 1352.3}
+    assert set(src.values()) == {"measured"}
+    part = tmp_path / "part.json"       # records with a value field; one key missing
+    part.write_text('{"hbm_gbs": {"value": 6546.6}, "bf16_tflops": {"median": 1648.7}}')
+    peaks, src = bench.load_peaks(str(part))
+    assert peaks["hbm_gbs"] == 6546.6 and peaks["bf16_tflops"] == 1648.7
+    assert peaks["bf16_tflops_sustained"] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+    assert src == {"hbm_gbs": "measured", "bf16_tflops": "measured", "bf16_tflops_sustained": "fallback"}
+    bad = tmp_path / "bad.json"
+    bad.write_text("not json")
+    peaks, src = bench.load_peaks(str(bad))
+    assert peaks == bench.FALLBACK_PEAKS and set(src.values()) == {"fallback"}
+    peaks, src = bench.load_peaks(str(tmp_path / "absent.json"))
+    assert peaks == bench.FALLBACK_PEAKS and set(src.values()) == {"fallback"}
