@@ -410,6 +410,10 @@ struct SmallCta {
   // which needs every owner to have finished reading its receive slots: the
   // slots and barriers are never overwritten early.)
   __device__ __forceinline__ void exchange(float fA) {
+    if (C == 1) {
+      exchange_local(fA);
+      return;
+    }
     if (ok && tid == 0) {
       mbar_arrive_expect_tx(recv_bar, recv_bytes);
       mbar_arrive_expect_tx(a_bar, a_bytes);
@@ -496,6 +500,33 @@ struct SmallCta {
     ++xphase;
     // upper triangle of A from the lower one (local; ends with the async-proxy fence)
     if (ok) mirror_upper(As, G, tid);
+    __syncthreads();
+  }
+
+  // A cluster of one: its partial is the sum, written as A from TMEM (the
+  // same bits as the exchange, which adds the one slot to zero and scales).
+  __device__ __forceinline__ void exchange_local(float fA) {
+    if (ok && half * 64 < m8) {
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld_64(tmem + tlane + static_cast<uint32_t>(half * 64), v);
+      if (row < m8) {
+#pragma unroll
+        for (int gg = 0; gg < 8; ++gg) {
+          const int g = half * 8 + gg;
+          if (g <= (row >> 3)) {
+            float acc[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = (0.0f + __uint_as_float(v[8 * gg + e])) * fA;
+            *reinterpret_cast<uint4*>(As + sw128_chunk(row, g)) = pack_f16x8(acc);
+          }
+        }
+      }
+    }
+    tc_fence_before();        // the TMEM reads above precede the next product's writes
+    ++xphase;
+    __syncthreads();
+    if (ok) mirror_upper(As, G, tid);    // ends with the async-proxy fence
     __syncthreads();
   }
 
