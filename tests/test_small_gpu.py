@@ -85,6 +85,7 @@ SHAPES = [
     (100, 1000),   # resident 4 x 256, ragged
     (128, 128),    # resident 2 x 64
     (3, 5),        # resident 1 x 64, element stores (cols not a multiple of 8)
+    (64, 64),      # resident 1 x 64: a cluster of one, its partial X X^T is A
     (1, 4096),     # streamed; one row: one owner, three CTAs own no block of A
     (128, 4040),   # streamed 4 x 1024, last CTA's last blocks partly padding
     (65, 3000),    # streamed 4 x 768, 9 row blocks of A
@@ -99,6 +100,7 @@ SHAPES = [
     (4096, 128),   # streamed on the transposed copy
     (1000, 100),
     (5, 3),
+    (64, 40),      # a cluster of one on the transposed copy
     (3001, 65),    # resident 8 x 384, element stores on the transposed copy
     (12288, 80),   # streamed on the transposed copy
 ]
