@@ -226,6 +226,11 @@ __device__ __forceinline__ void round_chunk(float (&v)[32], float f, float gamma
   }
 }
 
+// Fetches the line holding p into L1 (no register result, nothing waits).
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
 template <int CG>
 __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
   using Cfg = GemmCfg<CG>;
@@ -471,14 +476,10 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
       const GemmProblem& pr = P.prob[tc.p];
       const int acc = iter & 1;
       const uint32_t acc_par = (iter >> 1) & 1;
-      bool ok = mbar_wait_bounded(&tfull[acc], acc_par, abort_flag, limit);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) {
-        if (lane == 0) record_error(P.err, abort_flag, kErrEpilogue);
-        break;
-      }
-      tc_fence_after();
-
+      // The tile's scale (and, in launches whose epilogue is exposed, the
+      // first addend chunk) is read before the wait for the accumulator: it
+      // does not depend on it, and in launches of one tile per CTA these
+      // loads would otherwise start only after the main loop.
       const int row0 = tc.tm * Cfg::TILE_M + static_cast<int>(rank) * BM + q * 32;
       const int row = row0 + lane;
       const bool row_ok = row < pr.M;
@@ -505,7 +506,23 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
           for (int w = 0; w < 4; ++w) dst[w] = src[w];
         }
       };
-      load_addend(c_begin, add_cur);
+      // Split epilogues: the row's first addend chunk into registers and the
+      // second into L1 before the wait (the loop loads each next chunk one
+      // chunk ahead); long-K launches load the first chunk after it.
+      if (split) {
+        load_addend(c_begin, add_cur);
+        if (use_add && row_ok && c_begin + 1 < c_end && tc.tn * BN + (c_begin + 1) * 32 + 32 <= pr.N)
+          prefetch_l1(reinterpret_cast<const uint16_t*>(pr.addend) + add_slice + static_cast<long long>(row) * pr.add_ld +
+                      tc.tn * BN + (c_begin + 1) * 32);
+      }
+      bool ok = mbar_wait_bounded(&tfull[acc], acc_par, abort_flag, limit);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) record_error(P.err, abort_flag, kErrEpilogue);
+        break;
+      }
+      tc_fence_after();
+      if (!split) load_addend(c_begin, add_cur);
 
       for (int c = c_begin; c < c_end; ++c) {
         if (c + 1 < c_end) load_addend(c + 1, add_nxt);
@@ -625,11 +642,15 @@ __device__ __forceinline__ void ns_gemm_body(const GemmParams& P) {
           rs[pr.M] = rss1;
         }
       }
-      tc_fence_before();
-      if (CG == 2)
-        mbar_arrive_leader(&tempty[acc]);
-      else
-        mbar_arrive(&tempty[acc]);
+      // The MMA issuer reuses this accumulator only for a later tile of
+      // this CTA; after the last one nothing waits for it.
+      if (t + units < P.total_tiles) {
+        tc_fence_before();
+        if (CG == 2)
+          mbar_arrive_leader(&tempty[acc]);
+        else
+          mbar_arrive(&tempty[acc]);
+      }
     }
     // Every store has landed before the kernel (and its shared memory) ends.
     if (lane == 0) bulk_wait_group_all();
